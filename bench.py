@@ -1,0 +1,425 @@
+#!/usr/bin/env python
+"""Throughput of the flow-map block draft + prefix verify step on B200.
+
+One step = one speculative round of the hot path for every sequence of the
+workload: append the round's new target-feature rows to the context cache
+(fm_project_context), draft one K=16 block per noise sample (fm_draft) and
+verify it against target logits (fm_verify_greedy / fm_verify_sample).
+Inputs are seeded synthetic arrays (fm_synth) with the workload's shapes;
+the target model itself is not run: synthetic target logits stand in for
+its scores.
+
+Prints one JSON line (rank 0).  `value` is drafted 16-token blocks per
+second over all ranks (each rank runs its own replica: weak scaling, no
+collective on the data path); `verified_tokens_per_s` counts accepted
+tokens plus the target's correction/bonus token.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the fp64 CPU oracle on host cores
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import fm_synth as fs  # noqa: E402
+
+METRIC = "drafted 16-token blocks/s + verified tokens/s on 1 B200; % of HBM/TC roofline"
+DEFAULT_WORKLOAD = "qwen3_8b_bs1"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="fm", choices=["fm", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(fs.WORKLOADS))
+    ap.add_argument("--rounds", type=int, default=0, help="distinct seeded rounds cycled (0: auto)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, torch_dev: int, period=0.02):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.period, self.stop_ev = period, threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            bus = torch.cuda.get_device_properties(torch_dev).pci_bus_id
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover
+            self.err = str(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_ev.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self.stop_ev.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- algorithmic bytes
+def algorithmic_bytes(w: fs.Workload):
+    """Bytes each kernel class must move per step (weights, activations, caches)."""
+    s = w.shape
+    e = 2 if w.dtype == "bf16" else 4
+    M = w.M
+    V, d, F, nb = s.V, s.d, s.mlp, s.n_blocks
+    steps = len(w.t_grid) - 1
+    ctx_rows = w.ctx + w.new_rows
+    n_part = (V + 127) // 128
+    embed = V * d * e + M * V * e + 2 * M * d * 4                     # E, noise/D, x and z
+    lm = V * d * e + M * d * e + M * n_part * 8                        # W_lm, h, argmax partials
+    if any(t > 0 for t in w.temps) or steps > 1:
+        lm = V * d * e + M * d * e + M * V * 4                         # logits written
+    dit = nb * (3 * d * d + d * d + 2 * d * F) * e                     # block weights
+    attn = nb * w.B * ctx_rows * 2 * d * e                             # context keys/values
+    ctx = (w.B * w.new_rows * (s.n_taps * s.hidden * e + d * 4)
+           + s.n_taps * s.hidden * d * e + nb * 2 * d * d * e)        # hidden, fc, K/V weights
+    verify = w.B * w.n_noise * (s.K + 1) * V * 4
+    return {"embed": embed * steps, "lm_head": lm * steps, "dit_gemm": dit * steps,
+            "attn": attn * steps, "context": ctx, "verify": verify,
+            "embed_per_launch": embed, "lm_head_per_launch": lm}
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_fm(args, w, rank, world, local_rank):
+    import torch
+    import step_flow_map_b200 as fmb
+    from step_flow_map_b200.host import Context, to_device
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    s = w.shape
+    B, N, K, V = w.B, w.n_noise, s.K, s.V
+    seqs = list(range(B))
+    sampled = [b for b in seqs if w.temps[b] > 0]
+    greedy = [b for b in seqs if w.temps[b] == 0]
+    # contiguous halves only (greedy first, then sampled), as in the mixed workload
+    assert sampled == list(range(len(greedy), B)) or not sampled
+    t_setup = time.time()
+    W = fs.make_weights(s, w.dtype)
+    max_new = max(1, min(1024, w.ctx))
+    ctx = Context(s, w.dtype, W, max_ctx=w.ctx + max(w.new_rows, 1) + 8, max_seqs=B,
+                  max_noise=N, max_new=max(max_new, w.new_rows))
+    del W
+    for b in seqs:
+        h = fs.prefill_hidden(w, b)
+        for p0 in range(0, w.ctx, max_new):
+            ctx.project([b], to_device(h[p0:p0 + max_new][None], w.dtype), [p0])
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+
+    per_round_mb = (B * N * K * V * (2 if w.dtype == "bf16" else 4) + B * N * (K + 1) * V * 4) / 2**20
+    R = args.rounds or min(w.rounds, args.steps + args.warmup, 32, max(1, int(4096 // per_round_mb)))
+    R = max(1, R)
+    need_logits = bool(sampled)
+    tokens = torch.empty((B, N, K), dtype=torch.int32, device="cuda")
+    dlog = torch.empty((B, N, K, V), dtype=torch.float32, device="cuda") if need_logits else None
+    rounds = []
+    for i in range(R):
+        r = i + 100000 * rank
+        ri = fs.round_inputs(w, r)
+        rd = {"noise": to_device(ri.noise, w.dtype),
+              "hidden": to_device(ri.new_hidden, w.dtype) if w.new_rows else None,
+              "u_draft": to_device(ri.u_draft), "u_accept": to_device(ri.u_accept),
+              "u_res": to_device(ri.u_res)}
+        # untimed pass: the drafted block the synthetic target scores
+        if w.new_rows:
+            ctx.project(seqs, rd["hidden"], [w.ctx] * B)
+        lg = torch.empty((B, N, K, V), dtype=torch.float32, device="cuda")
+        fmb.fm_draft(ctx.ctx, seqs, rd["noise"], N, w.t_grid, w.temps, rd["u_draft"], tokens, lg,
+                     stream)
+        tgt = fs.target_logits(w, r, tokens.cpu().numpy(), lg.cpu().numpy())
+        del lg
+        rd["target"] = to_device(tgt)
+        rounds.append(rd)
+    n_acc_all = torch.zeros((args.steps + args.warmup, B), dtype=torch.int32, device="cuda")
+    branch = torch.empty(B, dtype=torch.int32, device="cuda")
+    out_tok = torch.empty((B, K + 1), dtype=torch.int32, device="cuda")
+    g, h0 = len(greedy), len(greedy)
+
+    def step(rd, k, n_acc):
+        if w.new_rows:
+            fmb.fm_project_context(ctx.ctx, seqs, rd["hidden"], w.new_rows, [w.ctx] * B, stream)
+        fmb.fm_draft(ctx.ctx, seqs, rd["noise"], N, w.t_grid, w.temps, rd["u_draft"], tokens, dlog,
+                     stream)
+        tgt = rd["target"]
+        if g:
+            fmb.fm_verify_greedy(ctx.ctx, tgt, tokens, g, N, K, V, n_acc, branch, out_tok, stream)
+        if sampled:
+            ns = B - g
+            fmb.fm_verify_sample(ctx.ctx, tgt[h0:], dlog[h0:], tokens[h0:], ns, N, K, V,
+                                 w.temps[h0], rd["u_accept"][h0:], rd["u_res"][h0:],
+                                 n_acc[h0:], branch[h0:], out_tok[h0:], stream)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    setup_s = time.time() - t_setup
+    for k in range(args.warmup):
+        step(rounds[k % R], k, n_acc_all[k])
+    ab = algorithmic_bytes(w)
+    prof_classes = ["embed", "lm_head"]
+    mask = sum(1 << fmb.FM_PROF[c] for c in prof_classes)
+    barrier()
+    fmb.fm_profile(ctx.ctx, mask)
+    fmb.fm_profile_read(ctx.ctx, reset=True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        ev0.record(stream)
+        for k in range(args.steps):
+            step(rounds[(args.warmup + k) % R], k, n_acc_all[args.warmup + k])
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    prof_ms, launches = fmb.fm_profile_read(ctx.ctx, reset=True)
+    fmb.fm_profile(ctx.ctx, 0)
+    barrier()
+    ms = max_over_ranks(ev0.elapsed_time(ev1))
+    n_sum = int(n_acc_all[args.warmup:].sum().item())
+    verified = n_sum + args.steps * B           # accepted + one target token per sequence
+    if dist is not None:
+        t = torch.tensor([float(verified)], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t)
+        verified = float(t.item())
+    else:
+        verified *= world
+    sec = ms / 1e3
+    blocks = B * N * args.steps * world
+    value = blocks / sec
+    tok_per_s = verified / sec
+
+    # roofline of the dominant kernel (largest timed share)
+    pk, pk_kind = peaks()
+    per_class = {}
+    for c in prof_classes:
+        i = fmb.FM_PROF[c]
+        n_launch = launches[i]
+        if prof_ms[i] > 0 and n_launch > 0:
+            avg = prof_ms[i] / (args.steps * (len(w.t_grid) - 1))
+            per_class[c] = {"ms_per_launch": avg, "bytes_per_launch": ab[f"{c}_per_launch"],
+                            "gbs": ab[f"{c}_per_launch"] / (avg / 1e3) / 1e9,
+                            "share_of_step": prof_ms[i] / ms}
+    dom = max(per_class, key=lambda c: per_class[c]["share_of_step"]) if per_class else None
+    roof = None
+    if dom:
+        a = per_class[dom]["gbs"]
+        roof = {"kernel": dom, "bound": "hbm", "achieved": round(a, 1), "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": round(a / pk["hbm_gbs"], 4), "traffic": None,
+                "peak_kind": pk_kind + " hbm_gbs (burst copy)"}
+    step_bytes = sum(ab[k] for k in ("embed", "lm_head", "dit_gemm", "attn", "context", "verify"))
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "blocks/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w.dtype, "data": "synthetic (seeded fm_synth inputs; no trained weights)",
+        "config": {"workload": w.name, "sequences_per_gpu": B, "noise_drafts": N, "K": K, "V": V,
+                   "d": s.d, "n_blocks": s.n_blocks, "context_rows": w.ctx + w.new_rows,
+                   "num_steps": len(w.t_grid) - 1, "temperatures": sorted(set(w.temps)),
+                   "distinct_rounds": R, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2: every step streams ~%.2f GB" % (step_bytes / 1e9)},
+        "verified_tokens_per_s": round(tok_per_s, 1),
+        "mean_accepted": round(n_sum / (args.steps * B), 3),
+        "step_hbm_gbs": round(step_bytes / (ms / args.steps / 1e3) / 1e9, 1),
+        "step_hbm_frac": round(step_bytes / (ms / args.steps / 1e3) / 1e9 / pk["hbm_gbs"], 4),
+        "roofline": roof, "kernels": per_class,
+        "gpu_launches": int(sum(launches)),
+        "clocks": clk.summary(), "setup_s": round(setup_s, 1),
+    }
+
+    # end to end: host inputs in pinned memory, copies inside the timed region
+    if not args.no_e2e:
+        RE = min(R, 8)
+        pin = []
+        for i in range(RE):
+            rd = rounds[i]
+            pin.append({k: (v.cpu().pin_memory() if v is not None else None) for k, v in rd.items()})
+        dev_in = {k: (torch.empty_like(v) if v is not None else None) for k, v in rounds[0].items()}
+        host_n = torch.empty((args.steps, B), dtype=torch.int32).pin_memory()
+        host_tok = torch.empty((args.steps, B, K + 1), dtype=torch.int32).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in pin[0].values() if v is not None)
+        d2h = B * 4 + B * (K + 1) * 4
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for k in range(args.steps):
+            src = pin[k % RE]
+            for key, v in src.items():
+                if v is not None:
+                    dev_in[key].copy_(v, non_blocking=True)
+            step(dev_in, k, n_acc_all[args.warmup + k])
+            host_n[k].copy_(n_acc_all[args.warmup + k], non_blocking=True)
+            host_tok[k].copy_(out_tok, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = max_over_ranks(e0.elapsed_time(e1))
+        line["e2e"] = {"value": round(B * N * args.steps * world / (ems / 1e3), 3),
+                       "unit": "blocks/s", "h2d_bytes_per_step": int(h2d),
+                       "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ems / args.steps, 5)}
+    ctx.close()
+    if dist is not None:
+        dist.destroy_process_group()
+    return line
+
+
+# ---------------------------------------------------------------- oracle (CPU) arm
+def oracle_rounds(w: fs.Workload, budget_s: float, max_rounds: int, warmup: int = 0):
+    """Time the fp64 oracle doing whole rounds of sequence 0 (context rows,
+    draft, verify); returns (seconds per block, rounds timed, cores)."""
+    from oracle import flashmap as om
+    s = w.shape
+    W = {k: v.astype(np.float64) for k, v in fs.make_weights(s, w.dtype).items()}
+    base = fs.prefill_hidden(w, 0)
+    C0, kv0 = om.project_context(W, s.n_blocks, base)
+    times = []
+    for r in range(warmup + max_rounds):
+        ri = fs.round_inputs(dataclasses_replace_B1(w), r)
+        t0 = time.perf_counter()
+        if w.new_rows:
+            _, kvn = om.project_context(W, s.n_blocks, ri.new_hidden[0])
+            kv = [(np.concatenate([a, an]), np.concatenate([b, bn]))
+                  for (a, b), (an, bn) in zip(kv0, kvn)]
+        else:
+            kv = kv0
+        res = om.draft(W, s, kv, ri.noise[0], w.t_grid, w.temps[0], ri.u_draft[0])
+        t1 = time.perf_counter()
+        tgt = fs.target_logits(dataclasses_replace_B1(w), r, res["tokens"][None],
+                               res["logits"][None].astype(np.float32))
+        t2 = time.perf_counter()
+        if w.temps[0] == 0:
+            om.verify_greedy(tgt[0], res["tokens"])
+        else:
+            om.verify_sample(tgt[0], res["logits"].astype(np.float32), res["tokens"], w.temps[0],
+                             ri.u_accept[0], ri.u_res[0])
+        t3 = time.perf_counter()
+        if r >= warmup:
+            times.append((t1 - t0) + (t3 - t2))
+        if r >= warmup and sum(times) > budget_s:
+            break
+    cores = len(os.sched_getaffinity(0))
+    return times, cores
+
+
+def dataclasses_replace_B1(w):
+    import dataclasses
+    return dataclasses.replace(w, B=1, temps=w.temps[:1])
+
+
+def run_reference(args, w):
+    wr = dataclasses_replace_B1(w)
+    times, cores = oracle_rounds(w, budget_s=1e9, max_rounds=args.steps, warmup=args.warmup)
+    sec = sum(times)
+    blocks = len(times) * wr.n_noise
+    v = blocks / sec
+    sample = (f"{len(times)} whole rounds of sequence 0 of {w.name} (context rows, "
+              f"{wr.n_noise} noise draft(s) x K={w.shape.K}, verify) per timed step set")
+    return {"impl": "reference", "metric": METRIC, "value": round(v, 5), "unit": "blocks/s",
+            "n_gpus": 1, "steps": len(times), "warmup": args.warmup,
+            "ms_per_step": round(sec / len(times) * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded fm_synth inputs; no trained weights)",
+            "config": {"workload": w.name, "sequences_per_gpu": 1},
+            "cpu_baseline": {"value": round(v, 5), "unit": "blocks/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(v, 5), "unit": "blocks/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    w = fs.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, w)), flush=True)
+        return 0
+    line = run_fm(args, w, rank, world, local_rank)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            times, cores = oracle_rounds(w, budget_s=args.cpu_seconds, max_rounds=64, warmup=0)
+            line["cpu_baseline"] = {
+                "value": round(len(times) * w.n_noise / sum(times), 5), "unit": "blocks/s",
+                "cores": cores, "kind": "oracle",
+                "sample": f"{len(times)} rounds of sequence 0 of {w.name}, fp64 numpy/BLAS, "
+                          f"~{args.cpu_seconds:.0f} s budget"}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -20,7 +20,7 @@ Princeton выпустили FlashMap", section "Как работает FlashMa
 Seeds: weights use ``1000 + tensor_index``; round ``r`` draws its noise from
 ``2000 + r``, its new context rows from ``3000 + r``, its target-logit
 perturbation from ``4000 + r`` and its uniforms from ``5000 + r``.  The
-prefill context uses seed 2999.  Every draw is PCG64 through a
+prefill context of sequence b uses seed 2999, stream b.  Every draw is PCG64 through a
 ``SeedSequence``, split into fixed chunks so that large tensors can be drawn
 on several threads with identical results.
 """
@@ -216,10 +216,10 @@ class RoundInputs:
     extra: dict = field(default_factory=dict)
 
 
-def prefill_hidden(w: Workload) -> np.ndarray:
-    """Prefill context: [B, ctx, n_taps, hidden] target hidden states, N(0,1)."""
+def prefill_hidden(w: Workload, b: int) -> np.ndarray:
+    """Prefill context of sequence b: [ctx, n_taps, hidden] target hidden states, N(0,1)."""
     s = w.shape
-    return _store(normal(2999, (w.B, w.ctx, s.n_taps, s.hidden)), w.dtype)
+    return _store(normal(2999, (w.ctx, s.n_taps, s.hidden), sub=b), w.dtype)
 
 
 def round_inputs(w: Workload, r: int) -> RoundInputs:

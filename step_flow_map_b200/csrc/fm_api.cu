@@ -1,0 +1,692 @@
+// C ABI of the flow-map drafter and verifier: context management and the
+// orchestration of the kernels of one draft / verify call.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <vector>
+
+#include "flashmap.h"
+#include "fm_simt.cuh"
+#include "fm_misc.cuh"
+#include "fm_verify.cuh"
+#include "fm_tc.cuh"
+
+using fm::bf16;
+
+// ------------------------------------------------------------------ errors
+static thread_local char g_err[1024] = "no error";
+
+static fm_status set_err(fm_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+#define FM_CUDA(call)                                                               \
+  do {                                                                              \
+    cudaError_t e_ = (call);                                                        \
+    if (e_ != cudaSuccess)                                                          \
+      return set_err(FM_ERR_CUDA, "%s failed: %s (%s:%d)", #call,                   \
+                     cudaGetErrorString(e_), __FILE__, __LINE__);                   \
+  } while (0)
+#define FM_LAUNCHED() FM_CUDA(cudaGetLastError())
+#define FM_TRY(expr)                  \
+  do {                                \
+    fm_status s_ = (expr);            \
+    if (s_ != FM_OK) return s_;       \
+  } while (0)
+
+extern "C" const char* fm_last_error(void) { return g_err; }
+
+// ------------------------------------------------------------------ context
+namespace {
+
+constexpr int N_MOD_SLOTS = 8;
+
+struct ModSlot {
+  bool valid = false;
+  float s = 0.f, t = 0.f;
+  float* buf = nullptr;  // [n_blocks][6][d] then [2][d], fp32
+  unsigned long long stamp = 0;
+};
+
+}  // namespace
+
+struct fm_ctx {
+  fm_config cfg;
+  int dev = 0, sms = 148;
+  size_t esz = 4;
+  fm_weights w;
+  std::vector<const void*> wqkv, wo, wup, wdown, wada;
+  std::vector<void*> owned;  // every cudaMalloc of the context
+  void* Et = nullptr;        // E transposed, [d][V]
+  std::vector<void*> Kc, Vc; // per block [max_seqs][max_ctx][d]
+  std::vector<int> ctx_len;  // host copy of each slot's context length
+  ModSlot mods[N_MOD_SLOTS];
+  unsigned long long clock = 0;
+  float *P = nullptr, *phi = nullptr, *tv = nullptr;  // tv: 5 x d time-MLP scratch
+  int M_max = 0, R_max = 0;
+  float *x = nullptr, *z = nullptr, *logits = nullptr;
+  void *h = nullptr, *qkv = nullptr, *o = nullptr, *u = nullptr, *D = nullptr;
+  float* part_v = nullptr;
+  int* part_i = nullptr;
+  int n_part = 0;
+  float* splitk = nullptr;
+  size_t splitk_elems = 0;
+  unsigned* tile_cnt = nullptr;
+  int tile_cnt_n = 0;
+  float* c_raw = nullptr;
+  void* c_norm = nullptr;
+  int v_chunks = 1;
+  float* vg_pv = nullptr;
+  int* vg_pi = nullptr;
+  unsigned* vg_cnt = nullptr;
+  float* vs_pm = nullptr;
+  double* vs_ps = nullptr;
+  double* vs_resid = nullptr;
+  bool use_tc = false;
+  fm::TcMaps tc;  // tensor maps of the weight operands (tensor-core path)
+  // launch counts and optional device timing per kernel class
+  long long launches[FM_PROF_N] = {};
+  int prof_mask = 0;
+  std::vector<cudaEvent_t> ev_a, ev_b;
+  std::vector<int> ev_cls;
+  size_t ev_used = 0;
+};
+
+namespace {
+
+fm_status dalloc(fm_ctx* c, void** p, size_t bytes) {
+  *p = nullptr;
+  if (bytes == 0) bytes = 16;
+  cudaError_t e = cudaMalloc(p, bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    *p = nullptr;
+    return set_err(FM_ERR_OOM, "cudaMalloc(%zu bytes) failed: %s", bytes, cudaGetErrorString(e));
+  }
+  c->owned.push_back(*p);
+  return FM_OK;
+}
+template <typename P>
+fm_status dalloc_t(fm_ctx* c, P** p, size_t count) {
+  void* v = nullptr;
+  fm_status s = dalloc(c, &v, count * sizeof(P));
+  *p = (P*)v;
+  return s;
+}
+
+// Records an event pair around the launches of one operation when its class
+// is being timed.
+struct Prof {
+  fm_ctx* c;
+  cudaStream_t st;
+  long slot = -1;
+  Prof(fm_ctx* c_, int cls, cudaStream_t st_) : c(c_), st(st_) {
+    if (((c->prof_mask >> cls) & 1) && c->ev_used < c->ev_a.size()) {
+      slot = (long)c->ev_used++;
+      c->ev_cls[slot] = cls;
+      cudaEventRecord(c->ev_a[slot], st);
+    }
+  }
+  ~Prof() {
+    if (slot >= 0) cudaEventRecord(c->ev_b[slot], st);
+  }
+};
+
+#define FM_KERNEL(c, cls, ...)   \
+  do {                           \
+    __VA_ARGS__;                 \
+    (c)->launches[cls]++;        \
+    FM_LAUNCHED();               \
+  } while (0)
+
+int grid_1d(size_t n, int threads, int cap = 148 * 16) {
+  size_t b = (n + threads - 1) / threads;
+  if (b > (size_t)cap) b = cap;
+  return b < 1 ? 1 : (int)b;
+}
+
+// ------------------------------------------------------------------ GEMM dispatch
+// Y[M][N] = A[M][Kd] . W(n,k), W K-major ([N][ldw]) or N-major ([Kd][ldw]).
+template <typename TA, typename TW, class Epi>
+fm_status gemm_simt(fm_ctx* c, int cls, const TA* A, int lda, const TW* W, int ldw, bool wk, int M,
+                    int N, int Kd, Epi epi, cudaStream_t st) {
+  Prof prof(c, cls, st);
+  dim3 grid((N + fm::SG_BN - 1) / fm::SG_BN, (M + fm::SG_BM - 1) / fm::SG_BM, 1);
+  long tiles = (long)grid.x * grid.y;
+  int splits = 1;
+  if (tiles < 2L * c->sms && Kd >= 512) {
+    splits = (int)((2L * c->sms + tiles - 1) / tiles);
+    splits = std::min(splits, Kd / 256);
+    splits = std::min(splits, 64);
+    while (splits > 1 && (size_t)splits * M * N > c->splitk_elems) --splits;
+    if (splits < 1) splits = 1;
+  }
+  int k_split = Kd;
+  if (splits > 1) {
+    k_split = (Kd + splits - 1) / splits;
+    k_split = (k_split + fm::SG_BK - 1) / fm::SG_BK * fm::SG_BK;
+    splits = (Kd + k_split - 1) / k_split;
+  }
+  grid.z = splits;
+  if (wk)
+    FM_KERNEL(c, cls, fm::k_gemm_simt<TA, TW, true, Epi><<<grid, 256, 0, st>>>(
+                          A, lda, W, ldw, M, N, Kd, k_split, c->splitk, epi));
+  else
+    FM_KERNEL(c, cls, fm::k_gemm_simt<TA, TW, false, Epi><<<grid, 256, 0, st>>>(
+                          A, lda, W, ldw, M, N, Kd, k_split, c->splitk, epi));
+  if (splits > 1)
+    FM_KERNEL(c, cls, fm::k_splitk_apply<Epi><<<grid_1d((size_t)M * N, 256), 256, 0, st>>>(
+                          c->splitk, splits, M, N, epi));
+  return FM_OK;
+}
+
+// Weight GEMM for the DiT, fc and LM head: tensor cores for bf16 when the
+// shape allows, CUDA cores otherwise.
+template <typename T, class Epi>
+fm_status gemm_w(fm_ctx* c, int cls, const T* A, int lda, const T* W, int M, int N, int Kd,
+                 Epi epi, cudaStream_t st, const fm::TcMap* map = nullptr) {
+  if constexpr (sizeof(T) == 2) {
+    if (c->use_tc && map && map->valid) {
+      Prof prof(c, cls, st);
+      int n_launch = 0;
+      fm_status s = fm::tc_gemm(c->tc, *map, (const bf16*)A, lda, M, N, Kd, epi, c->splitk,
+                                c->splitk_elems, c->tile_cnt, c->tile_cnt_n, c->sms, st, g_err,
+                                sizeof(g_err), &n_launch);
+      c->launches[cls] += n_launch;
+      return s;
+    }
+  }
+  return gemm_simt<T, T, Epi>(c, cls, A, lda, W, Kd, true, M, N, Kd, epi, st);
+}
+
+// ------------------------------------------------------------------ conditioning
+template <typename T>
+fm_status compute_mods(fm_ctx* c, float s, float t, float* out, cudaStream_t st) {
+  const int d = c->cfg.d, nb = c->cfg.n_blocks;
+  float* tv = c->tv;  // 5 slots of d
+  auto gemv = [&](const void* W, int n_out, int n_in, const float* x, float* y, const float* add,
+                  int act) -> fm_status {
+    int threads = 256, blocks = (n_out * 32 + threads - 1) / threads;
+    FM_KERNEL(c, FM_PROF_OTHER,
+              fm::k_gemv<T><<<blocks, threads, 0, st>>>((const T*)W, n_out, n_in, x, y, add, act));
+    return FM_OK;
+  };
+  FM_KERNEL(c, FM_PROF_OTHER, fm::k_time_features<<<1, 256, 0, st>>>((double)s, (double)t, c->phi));
+  FM_TRY(gemv(c->w.W_ts1, d, 256, c->phi, tv, nullptr, 1));                // SiLU(W1 phi(s))
+  FM_TRY(gemv(c->w.W_ts2, d, d, tv, tv + d, nullptr, 0));                 // TE_s(s)
+  FM_TRY(gemv(c->w.W_tt1, d, 256, c->phi + 256, tv + 2 * d, nullptr, 1)); // SiLU(W1 phi(t))
+  FM_TRY(gemv(c->w.W_tt2, d, d, tv + 2 * d, tv + 3 * d, tv + d, 0));      // c = TE_s + TE_t
+  FM_KERNEL(c, FM_PROF_OTHER, fm::k_silu_vec<<<(d + 255) / 256, 256, 0, st>>>(tv + 3 * d, tv + 4 * d, d));
+  for (int l = 0; l < nb; ++l)
+    FM_TRY(gemv(c->wada[l], 6 * d, d, tv + 4 * d, out + (size_t)l * 6 * d, nullptr, 0));
+  FM_TRY(gemv(c->w.W_ada_f, 2 * d, d, tv + 4 * d, out + (size_t)nb * 6 * d, nullptr, 0));
+  return FM_OK;
+}
+
+template <typename T>
+fm_status get_mods(fm_ctx* c, float s, float t, const float** out, cudaStream_t st) {
+  for (auto& m : c->mods)
+    if (m.valid && m.s == s && m.t == t) {
+      m.stamp = ++c->clock;
+      *out = m.buf;
+      return FM_OK;
+    }
+  ModSlot* victim = &c->mods[0];
+  for (auto& m : c->mods) {
+    if (!m.valid) { victim = &m; break; }
+    if (m.stamp < victim->stamp) victim = &m;
+  }
+  victim->valid = false;
+  FM_TRY(compute_mods<T>(c, s, t, victim->buf, st));
+  victim->valid = true;
+  victim->s = s;
+  victim->t = t;
+  victim->stamp = ++c->clock;
+  *out = victim->buf;
+  return FM_OK;
+}
+
+// ------------------------------------------------------------------ load
+template <typename T>
+fm_status load_impl(fm_ctx* c, cudaStream_t st) {
+  const fm_config& g = c->cfg;
+  const int d = g.d;
+  FM_TRY(dalloc(c, &c->Et, (size_t)g.V * d * sizeof(T)));
+  {
+    dim3 grid((d + 31) / 32, (g.V + 31) / 32), block(32, 8);
+    FM_KERNEL(c, FM_PROF_OTHER, fm::k_transpose<T><<<grid, block, 0, st>>>((const T*)c->w.E, (T*)c->Et, g.V, d));
+  }
+  c->Kc.resize(g.n_blocks);
+  c->Vc.resize(g.n_blocks);
+  for (int l = 0; l < g.n_blocks; ++l) {
+    size_t n = (size_t)g.max_seqs * g.max_ctx * d * sizeof(T);
+    FM_TRY(dalloc(c, &c->Kc[l], n));
+    FM_TRY(dalloc(c, &c->Vc[l], n));
+  }
+  c->ctx_len.assign(g.max_seqs, 0);
+  for (auto& m : c->mods) FM_TRY(dalloc_t(c, &m.buf, (size_t)(g.n_blocks * 6 + 2) * d));
+  FM_TRY(dalloc_t(c, &c->P, (size_t)g.K * d));
+  FM_TRY(dalloc_t(c, &c->phi, 512));
+  FM_TRY(dalloc_t(c, &c->tv, (size_t)5 * d));
+  {
+    std::vector<float> P((size_t)g.K * d);
+    for (int i = 0; i < g.K; ++i)
+      for (int k = 0; k < d / 2; ++k) {
+        double w = pow(10000.0, -2.0 * k / d);
+        P[(size_t)i * d + 2 * k] = (float)sin(i * w);
+        P[(size_t)i * d + 2 * k + 1] = (float)cos(i * w);
+      }
+    FM_CUDA(cudaMemcpyAsync(c->P, P.data(), P.size() * sizeof(float), cudaMemcpyHostToDevice, st));
+    FM_CUDA(cudaStreamSynchronize(st));
+  }
+  const int call_seqs = std::min(g.max_seqs, FM_MAX_CALL_SEQS);
+  c->M_max = call_seqs * g.max_noise * g.K;
+  c->R_max = call_seqs * g.max_new;
+  const size_t M = c->M_max;
+  FM_TRY(dalloc_t(c, &c->x, M * d));
+  FM_TRY(dalloc_t(c, &c->z, M * d));
+  FM_TRY(dalloc(c, &c->h, M * d * sizeof(T)));
+  FM_TRY(dalloc(c, &c->qkv, M * 3 * d * sizeof(T)));
+  FM_TRY(dalloc(c, &c->o, M * d * sizeof(T)));
+  FM_TRY(dalloc(c, &c->u, M * g.mlp * sizeof(T)));
+  FM_TRY(dalloc_t(c, &c->logits, M * g.V));
+  FM_TRY(dalloc(c, &c->D, M * g.V * sizeof(T)));
+  c->n_part = (g.V + 127) / 128;
+  FM_TRY(dalloc_t(c, &c->part_v, M * c->n_part));
+  FM_TRY(dalloc_t(c, &c->part_i, M * c->n_part));
+  c->splitk_elems = std::max<size_t>((size_t)1 << 22, 8 * M * (size_t)std::max(3 * d, g.mlp));
+  FM_TRY(dalloc_t(c, &c->splitk, c->splitk_elems));
+  c->tile_cnt_n = 1 << 16;
+  FM_TRY(dalloc_t(c, &c->tile_cnt, c->tile_cnt_n));
+  FM_CUDA(cudaMemsetAsync(c->tile_cnt, 0, c->tile_cnt_n * sizeof(unsigned), st));
+  FM_TRY(dalloc_t(c, &c->c_raw, (size_t)c->R_max * d));
+  FM_TRY(dalloc(c, &c->c_norm, (size_t)c->R_max * d * sizeof(T)));
+  // verify workspaces: rows = B*N*(K+1) target + B*N*K draft rows
+  c->v_chunks = 64;
+  const size_t vrows = (size_t)g.max_seqs * g.max_noise * (2 * g.K + 1);
+  FM_TRY(dalloc_t(c, &c->vg_pv, vrows * c->v_chunks));
+  FM_TRY(dalloc_t(c, &c->vg_pi, vrows * c->v_chunks));
+  FM_TRY(dalloc_t(c, &c->vg_cnt, (size_t)g.max_seqs));
+  FM_CUDA(cudaMemsetAsync(c->vg_cnt, 0, g.max_seqs * sizeof(unsigned), st));
+  FM_TRY(dalloc_t(c, &c->vs_pm, vrows * c->v_chunks));
+  FM_TRY(dalloc_t(c, &c->vs_ps, vrows * c->v_chunks));
+  FM_TRY(dalloc_t(c, &c->vs_resid, (size_t)g.max_seqs * 2 * g.V));
+  if constexpr (sizeof(T) == 2) {
+    c->use_tc = fm::tc_supported(g.d, g.mlp, g.V, g.n_taps * g.target_hidden);
+    if (c->use_tc) {
+      if (!fm::tc_make_maps(c->tc, c->w.W_lm, c->Et, c->w.W_fc, c->wqkv.data(), c->wo.data(),
+                            c->wup.data(), c->wdown.data(), g.n_blocks, g.d, g.mlp, g.V,
+                            g.n_taps * g.target_hidden, g_err, sizeof(g_err)))
+        return FM_ERR_CUDA;
+    }
+  }
+  // the grids every draft uses
+  const float grids[3][2] = {{0.f, 1.f}, {0.f, 0.5f}, {0.5f, 1.f}};
+  for (auto& gp : grids) {
+    const float* tmp;
+    FM_TRY(get_mods<T>(c, gp[0], gp[1], &tmp, st));
+  }
+  FM_CUDA(cudaStreamSynchronize(st));
+  return FM_OK;
+}
+
+// ------------------------------------------------------------------ context projection
+template <typename T>
+fm_status project_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* hidden,
+                       int n_new, const int32_t* pos0, cudaStream_t st) {
+  const fm_config& g = c->cfg;
+  const int d = g.d, R = n_seqs * n_new, in = g.n_taps * g.target_hidden;
+  FM_TRY(gemm_w<T>(c, FM_PROF_CONTEXT, (const T*)hidden, in, (const T*)c->w.W_fc, R, d, in,
+                   fm::EpiStoreF32{c->c_raw, d}, st, &c->tc.fc));
+  {
+    Prof prof(c, FM_PROF_CONTEXT, st);
+    FM_KERNEL(c, FM_PROF_CONTEXT, fm::k_adaln<float, T><<<R, 256, 0, st>>>(
+                                      c->c_raw, d, nullptr, nullptr, (T*)c->c_norm));
+  }
+  fm::EpiCtxKV<T> epi;
+  epi.d = d;
+  epi.max_ctx = g.max_ctx;
+  epi.map.n_seqs = n_seqs;
+  epi.map.n_new = n_new;
+  for (int q = 0; q < n_seqs; ++q) {
+    epi.map.slot[q] = seq_ids[q];
+    epi.map.pos0[q] = pos0[q];
+  }
+  for (int l = 0; l < g.n_blocks; ++l) {
+    epi.Kc = (T*)c->Kc[l];
+    epi.Vc = (T*)c->Vc[l];
+    const T* Wkv = (const T*)c->wqkv[l] + (size_t)d * d;  // key and value thirds
+    FM_TRY(gemm_w<T>(c, FM_PROF_CONTEXT, (const T*)c->c_norm, d, Wkv, R, 2 * d, d, epi, st,
+                     &c->tc.kv[l]));
+  }
+  for (int q = 0; q < n_seqs; ++q) c->ctx_len[seq_ids[q]] = pos0[q] + n_new;
+  return FM_OK;
+}
+
+// ------------------------------------------------------------------ draft
+template <typename T>
+fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* noise,
+                     int n_noise, const float* t_grid, int num_steps, const float* temps,
+                     const double* u_draft, int32_t* tokens, float* draft_logits,
+                     cudaStream_t st) {
+  const fm_config& g = c->cfg;
+  const int d = g.d, K = g.K, V = g.V, nb = g.n_blocks, F = g.mlp;
+  const int M = n_seqs * n_noise * K;
+  T* h = (T*)c->h;
+  T* qkv = (T*)c->qkv;
+  T* o = (T*)c->o;
+  T* u = (T*)c->u;
+  fm::AttnArgs aa;
+  aa.n_seqs = n_seqs;
+  aa.n_noise = n_noise;
+  aa.K = K;
+  aa.d = d;
+  aa.n_heads = g.n_heads;
+  aa.max_ctx = g.max_ctx;
+  aa.scale = (float)(1.0 / sqrt((double)(d / g.n_heads)));
+  for (int q = 0; q < n_seqs; ++q) {
+    aa.slot[q] = seq_ids[q];
+    aa.len[q] = c->ctx_len[seq_ids[q]];
+  }
+  bool any_sample = false;
+  fm::TempArgs ta;
+  ta.n_noise = n_noise;
+  ta.K = K;
+  for (int q = 0; q < n_seqs; ++q) {
+    ta.temp[q] = temps[q];
+    any_sample |= temps[q] > 0.f;
+  }
+  float* logits = draft_logits ? draft_logits : c->logits;
+  for (int k = 0; k < num_steps; ++k) {
+    const float s = t_grid[k], t = t_grid[k + 1];
+    const bool last = (k == num_steps - 1);
+    const float* mods;
+    FM_TRY(get_mods<T>(c, s, t, &mods, st));
+    // input embedding (first step: x0 E; later: flow-map update through E)
+    fm::EpiEmbed emb{c->x, num_steps > 1 ? c->z : nullptr, c->P, d, K,
+                     k == 0 ? -1.f : (float)((double)(t - s) / (1.0 - (double)s))};
+    if (k == 0) emb.alpha = -1.f;
+    const T* A = (k == 0) ? (const T*)noise : (const T*)c->D;
+    if (c->use_tc && c->tc.embed.valid) {
+      FM_TRY(gemm_w<T>(c, FM_PROF_EMBED, A, V, (const T*)c->Et, M, d, V, emb, st, &c->tc.embed));
+    } else {
+      FM_TRY((gemm_simt<T, T, fm::EpiEmbed>(c, FM_PROF_EMBED, A, V, (const T*)c->w.E, d, false, M,
+                                             d, V, emb, st)));
+    }
+    for (int l = 0; l < nb; ++l) {
+      const float* ml = mods + (size_t)l * 6 * d;
+      {
+        Prof prof(c, FM_PROF_NORM, st);
+        FM_KERNEL(c, FM_PROF_NORM, fm::k_adaln<float, T><<<M, 256, 0, st>>>(c->x, d, ml, ml + d, h));
+      }
+      FM_TRY(gemm_w<T>(c, FM_PROF_DIT_GEMM, h, d, (const T*)c->wqkv[l], M, 3 * d, d,
+                       fm::EpiStore<T>{qkv, 3 * d}, st, &c->tc.qkv[l]));
+      {
+        Prof prof(c, FM_PROF_ATTN, st);
+        dim3 grid(n_seqs, g.n_heads, n_noise);
+        FM_KERNEL(c, FM_PROF_ATTN, fm::k_attn_simt<T><<<grid, 128, 0, st>>>(
+                                       qkv, (const T*)c->Kc[l], (const T*)c->Vc[l], o, aa));
+      }
+      FM_TRY(gemm_w<T>(c, FM_PROF_DIT_GEMM, o, d, (const T*)c->wo[l], M, d, d,
+                       fm::EpiResidual{c->x, ml + 2 * d, d}, st, &c->tc.o[l]));
+      {
+        Prof prof(c, FM_PROF_NORM, st);
+        FM_KERNEL(c, FM_PROF_NORM, fm::k_adaln<float, T><<<M, 256, 0, st>>>(c->x, d, ml + 3 * d,
+                                                                            ml + 4 * d, h));
+      }
+      FM_TRY(gemm_w<T>(c, FM_PROF_DIT_GEMM, h, d, (const T*)c->wup[l], M, F, d,
+                       fm::EpiGelu<T>{u, F}, st, &c->tc.up[l]));
+      FM_TRY(gemm_w<T>(c, FM_PROF_DIT_GEMM, u, F, (const T*)c->wdown[l], M, d, F,
+                       fm::EpiResidual{c->x, ml + 5 * d, d}, st, &c->tc.down[l]));
+    }
+    const float* mf = mods + (size_t)nb * 6 * d;
+    {
+      Prof prof(c, FM_PROF_NORM, st);
+      FM_KERNEL(c, FM_PROF_NORM, fm::k_adaln<float, T><<<M, 256, 0, st>>>(c->x, d, mf, mf + d, h));
+    }
+    // LM head: greedy-only final steps keep the logits on chip when possible
+    const bool need_logits = !last || any_sample || draft_logits != nullptr;
+    bool have_partials = false;
+    if (c->use_tc && c->tc.lm.valid && !need_logits) {
+      Prof prof(c, FM_PROF_LM_HEAD, st);
+      int n_launch = 0;
+      FM_TRY(fm::tc_lm_head_argmax(c->tc, (const bf16*)h, d, M, V, c->part_v, c->part_i,
+                                   c->n_part, c->sms, st, g_err, sizeof(g_err), &n_launch));
+      c->launches[FM_PROF_LM_HEAD] += n_launch;
+      have_partials = true;
+    } else {
+      FM_TRY(gemm_w<T>(c, FM_PROF_LM_HEAD, h, d, (const T*)c->w.W_lm, M, V, d,
+                       fm::EpiStoreF32{logits, V}, st, &c->tc.lm));
+    }
+    Prof prof(c, FM_PROF_NORM, st);
+    if (!last) {
+      FM_KERNEL(c, FM_PROF_NORM, fm::k_softmax_rows<T><<<M, 1024, 0, st>>>(logits, V, (T*)c->D));
+    } else {
+      FM_KERNEL(c, FM_PROF_NORM,
+                fm::k_select_tokens<<<M, 1024, 0, st>>>(
+                    have_partials ? nullptr : logits, V, have_partials ? c->part_v : nullptr,
+                    have_partials ? c->part_i : nullptr, c->n_part, u_draft, ta, tokens));
+    }
+  }
+  return FM_OK;
+}
+
+fm_status check_cfg(const fm_config* g) {
+  if (!g) return set_err(FM_ERR_ARG, "cfg is NULL");
+  if (g->V < 2 || g->d < 2 || g->n_blocks < 1 || g->n_heads < 1 || g->mlp < 1 || g->K < 1 ||
+      g->target_hidden < 1 || g->n_taps < 1 || g->max_ctx < 1 || g->max_seqs < 1 ||
+      g->max_noise < 1 || g->max_new < 1)
+    return set_err(FM_ERR_ARG, "config sizes must be positive");
+  if (g->d % g->n_heads || (g->d / g->n_heads) > fm::SA_MAXDH || (g->d & 1))
+    return set_err(FM_ERR_ARG, "d must be even and d/n_heads <= %d", fm::SA_MAXDH);
+  if (g->K > fm::SA_MAXQ) return set_err(FM_ERR_UNSUPPORTED, "K must be <= %d", fm::SA_MAXQ);
+  if (g->max_noise > 32) return set_err(FM_ERR_UNSUPPORTED, "max_noise must be <= 32");
+  if (g->max_noise * (g->K + 1) > fm::VG_MAX_ROWS)
+    return set_err(FM_ERR_UNSUPPORTED, "max_noise*(K+1) must be <= %d", fm::VG_MAX_ROWS);
+  if (g->dtype != FM_F32 && g->dtype != FM_BF16) return set_err(FM_ERR_ARG, "bad dtype");
+  return FM_OK;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ ABI
+extern "C" fm_status fm_load_weights(fm_ctx** out, const fm_config* cfg, const fm_weights* w,
+                                     fm_stream stream) {
+  if (!out) return set_err(FM_ERR_ARG, "out is NULL");
+  *out = nullptr;
+  FM_TRY(check_cfg(cfg));
+  if (!w || !w->E || !w->W_lm || !w->W_fc || !w->W_ts1 || !w->W_ts2 || !w->W_tt1 || !w->W_tt2 ||
+      !w->W_ada_f || !w->W_qkv || !w->W_o || !w->W_up || !w->W_down || !w->W_ada)
+    return set_err(FM_ERR_ARG, "a weight pointer is NULL");
+  fm_ctx* c = new fm_ctx();
+  c->cfg = *cfg;
+  c->w = *w;
+  c->esz = cfg->dtype == FM_BF16 ? 2 : 4;
+  for (int l = 0; l < cfg->n_blocks; ++l) {
+    if (!w->W_qkv[l] || !w->W_o[l] || !w->W_up[l] || !w->W_down[l] || !w->W_ada[l]) {
+      delete c;
+      return set_err(FM_ERR_ARG, "block %d weight pointer is NULL", l);
+    }
+    c->wqkv.push_back(w->W_qkv[l]);
+    c->wo.push_back(w->W_o[l]);
+    c->wup.push_back(w->W_up[l]);
+    c->wdown.push_back(w->W_down[l]);
+    c->wada.push_back(w->W_ada[l]);
+  }
+  c->w.W_qkv = c->w.W_o = c->w.W_up = c->w.W_down = c->w.W_ada = nullptr;
+  cudaError_t e = cudaGetDevice(&c->dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&c->sms, cudaDevAttrMultiProcessorCount, c->dev);
+  if (e != cudaSuccess) {
+    delete c;
+    return set_err(FM_ERR_CUDA, "no CUDA device: %s", cudaGetErrorString(e));
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  fm_status s = cfg->dtype == FM_BF16 ? load_impl<bf16>(c, st) : load_impl<float>(c, st);
+  if (s != FM_OK) {
+    char keep[sizeof(g_err)];
+    memcpy(keep, g_err, sizeof(keep));
+    fm_free(c);
+    memcpy(g_err, keep, sizeof(keep));
+    return s;
+  }
+  *out = c;
+  return FM_OK;
+}
+
+extern "C" void fm_free(fm_ctx* c) {
+  if (!c) return;
+  cudaDeviceSynchronize();
+  for (void* p : c->owned) cudaFree(p);
+  for (auto e : c->ev_a) cudaEventDestroy(e);
+  for (auto e : c->ev_b) cudaEventDestroy(e);
+  fm::tc_free_maps(c->tc);
+  delete c;
+}
+
+extern "C" fm_status fm_project_context(fm_ctx* c, const int32_t* seq_ids, int n_seqs,
+                                        const void* hidden, int n_new, const int32_t* pos0,
+                                        fm_stream stream) {
+  if (!c || !seq_ids || !hidden || !pos0) return set_err(FM_ERR_ARG, "NULL argument");
+  const fm_config& g = c->cfg;
+  if (n_seqs < 1 || n_seqs > FM_MAX_CALL_SEQS || n_seqs > g.max_seqs)
+    return set_err(FM_ERR_ARG, "n_seqs=%d out of range", n_seqs);
+  if (n_new < 1 || n_new > g.max_new) return set_err(FM_ERR_ARG, "n_new=%d out of range", n_new);
+  std::vector<char> seen(g.max_seqs, 0);
+  for (int q = 0; q < n_seqs; ++q) {
+    if (seq_ids[q] < 0 || seq_ids[q] >= g.max_seqs || seen[seq_ids[q]])
+      return set_err(FM_ERR_ARG, "seq_ids[%d]=%d invalid or repeated", q, seq_ids[q]);
+    seen[seq_ids[q]] = 1;
+    if (pos0[q] < 0 || pos0[q] + n_new > g.max_ctx)
+      return set_err(FM_ERR_ARG, "pos0[%d]=%d: rows exceed max_ctx=%d", q, pos0[q], g.max_ctx);
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  return g.dtype == FM_BF16 ? project_impl<bf16>(c, seq_ids, n_seqs, hidden, n_new, pos0, st)
+                            : project_impl<float>(c, seq_ids, n_seqs, hidden, n_new, pos0, st);
+}
+
+extern "C" fm_status fm_draft(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* noise,
+                              int n_noise, const float* t_grid, int num_steps,
+                              const float* temperature, const double* u_draft, int32_t* tokens,
+                              float* draft_logits, fm_stream stream) {
+  if (!c || !seq_ids || !noise || !t_grid || !temperature || !tokens)
+    return set_err(FM_ERR_ARG, "NULL argument");
+  const fm_config& g = c->cfg;
+  if (n_seqs < 1 || n_seqs > FM_MAX_CALL_SEQS || n_seqs > g.max_seqs)
+    return set_err(FM_ERR_ARG, "n_seqs=%d out of range", n_seqs);
+  if (n_noise < 1 || n_noise > g.max_noise)
+    return set_err(FM_ERR_ARG, "n_noise=%d out of range", n_noise);
+  if (num_steps < 1 || num_steps > FM_MAX_STEPS)
+    return set_err(FM_ERR_ARG, "num_steps=%d out of range", num_steps);
+  if (t_grid[0] != 0.f || t_grid[num_steps] != 1.f)
+    return set_err(FM_ERR_ARG, "t_grid must start at 0 and end at 1");
+  for (int k = 0; k < num_steps; ++k)
+    if (!(t_grid[k] < t_grid[k + 1])) return set_err(FM_ERR_ARG, "t_grid must increase");
+  for (int q = 0; q < n_seqs; ++q) {
+    if (seq_ids[q] < 0 || seq_ids[q] >= g.max_seqs)
+      return set_err(FM_ERR_ARG, "seq_ids[%d]=%d invalid", q, seq_ids[q]);
+    if (!(temperature[q] >= 0.f)) return set_err(FM_ERR_ARG, "temperature[%d] < 0", q);
+    if (temperature[q] > 0.f && !u_draft)
+      return set_err(FM_ERR_ARG, "u_draft is NULL but sequence %d samples", q);
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  return g.dtype == FM_BF16
+             ? draft_impl<bf16>(c, seq_ids, n_seqs, noise, n_noise, t_grid, num_steps, temperature,
+                                u_draft, tokens, draft_logits, st)
+             : draft_impl<float>(c, seq_ids, n_seqs, noise, n_noise, t_grid, num_steps,
+                                 temperature, u_draft, tokens, draft_logits, st);
+}
+
+static fm_status check_verify(fm_ctx* c, const void* tgt, const void* draft, int B, int N, int K,
+                              int V, const void* n_acc, const void* branch, const void* out) {
+  if (!c || !tgt || !draft || !n_acc || !branch || !out) return set_err(FM_ERR_ARG, "NULL argument");
+  const fm_config& g = c->cfg;
+  if (B < 1 || B > g.max_seqs) return set_err(FM_ERR_ARG, "B=%d out of range", B);
+  if (N < 1 || N > g.max_noise) return set_err(FM_ERR_ARG, "N=%d out of range", N);
+  if (K != g.K || V != g.V) return set_err(FM_ERR_UNSUPPORTED, "K/V differ from the configuration");
+  return FM_OK;
+}
+
+static int verify_chunks(fm_ctx* c, long rows, int V) {
+  long want = (2L * c->sms + rows - 1) / rows;
+  int ch = (int)std::min<long>(want, c->v_chunks);
+  ch = std::min(ch, std::max(1, V / 1024));
+  return std::max(ch, 1);
+}
+
+extern "C" fm_status fm_verify_greedy(fm_ctx* c, const float* target_logits, const int32_t* draft,
+                                      int B, int N, int K, int V, int32_t* n_acc,
+                                      int32_t* branch, int32_t* out_tokens, fm_stream stream) {
+  FM_TRY(check_verify(c, target_logits, draft, B, N, K, V, n_acc, branch, out_tokens));
+  cudaStream_t st = (cudaStream_t)stream;
+  const long rows = (long)B * N * (K + 1);
+  const int ch = verify_chunks(c, rows, V);
+  Prof prof(c, FM_PROF_VERIFY, st);
+  FM_KERNEL(c, FM_PROF_VERIFY, fm::k_verify_greedy<<<(unsigned)(rows * ch), fm::VG_THREADS, 0, st>>>(
+      target_logits, draft, B, N, K, V, ch, c->vg_pv, c->vg_pi, c->vg_cnt, n_acc, branch,
+      out_tokens));
+  return FM_OK;
+}
+
+extern "C" fm_status fm_verify_sample(fm_ctx* c, const float* target_logits,
+                                      const float* draft_logits, const int32_t* draft, int B, int N,
+                                      int K, int V, float temperature, const double* u_accept,
+                                      const double* u_res, int32_t* n_acc, int32_t* branch,
+                                      int32_t* out_tokens, fm_stream stream) {
+  FM_TRY(check_verify(c, target_logits, draft, B, N, K, V, n_acc, branch, out_tokens));
+  if (!(temperature > 0.f)) return set_err(FM_ERR_ARG, "temperature must be > 0");
+  if (!u_accept || !u_res) return set_err(FM_ERR_ARG, "uniforms are NULL");
+  cudaStream_t st = (cudaStream_t)stream;
+  const int n_tgt = B * N * (K + 1);
+  const int n_rows = n_tgt + (draft_logits ? B * N * K : 0);
+  const int ch = verify_chunks(c, n_rows, V);
+  Prof prof(c, FM_PROF_VERIFY, st);
+  FM_KERNEL(c, FM_PROF_VERIFY, fm::k_row_stats<<<(unsigned)((long)n_rows * ch), fm::VS_THREADS, 0, st>>>(
+      target_logits, draft_logits, n_tgt, n_rows, V, ch, temperature, c->vs_pm, c->vs_ps));
+  FM_KERNEL(c, FM_PROF_VERIFY, fm::k_verify_sample_decide<<<B, fm::VS_DECIDE_THREADS, 0, st>>>(
+      target_logits, draft_logits, draft, B, N, K, V, temperature, u_accept, u_res, c->vs_pm,
+      c->vs_ps, ch, c->vs_resid, n_acc, branch, out_tokens));
+  return FM_OK;
+}
+
+extern "C" fm_status fm_profile(fm_ctx* c, int mask) {
+  if (!c) return set_err(FM_ERR_ARG, "NULL context");
+  if (mask && c->ev_a.empty()) {
+    const size_t n = 65536;
+    c->ev_a.resize(n);
+    c->ev_b.resize(n);
+    c->ev_cls.assign(n, 0);
+    for (size_t i = 0; i < n; ++i) {
+      FM_CUDA(cudaEventCreate(&c->ev_a[i]));
+      FM_CUDA(cudaEventCreate(&c->ev_b[i]));
+    }
+  }
+  c->prof_mask = mask & ((1 << FM_PROF_N) - 1);
+  c->ev_used = 0;
+  return FM_OK;
+}
+
+extern "C" fm_status fm_profile_read(fm_ctx* c, double* ms, int64_t* launches, int reset) {
+  if (!c) return set_err(FM_ERR_ARG, "NULL context");
+  if (ms) {
+    for (int k = 0; k < FM_PROF_N; ++k) ms[k] = 0.0;
+    for (size_t i = 0; i < c->ev_used; ++i) {
+      FM_CUDA(cudaEventSynchronize(c->ev_b[i]));
+      float t = 0.f;
+      FM_CUDA(cudaEventElapsedTime(&t, c->ev_a[i], c->ev_b[i]));
+      ms[c->ev_cls[i]] += t;
+    }
+  }
+  if (launches)
+    for (int k = 0; k < FM_PROF_N; ++k) launches[k] = c->launches[k];
+  if (reset) {
+    for (int k = 0; k < FM_PROF_N; ++k) c->launches[k] = 0;
+    c->ev_used = 0;
+  }
+  return FM_OK;
+}

@@ -1,0 +1,103 @@
+// Shared device helpers: storage types, conversions, warp/block reductions.
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <math.h>
+
+namespace fm {
+
+typedef __nv_bfloat16 bf16;
+
+template <typename T> __device__ __forceinline__ float to_f(T v);
+template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f<bf16>(bf16 v) { return __bfloat162float(v); }
+
+template <typename T> __device__ __forceinline__ T from_f(float v);
+template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ bf16 from_f<bf16>(float v) { return __float2bfloat16_rn(v); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// (value, index) argmax with ties to the lowest index; NaN never wins
+// because every comparison with NaN is false.
+struct ArgMax {
+  float v;
+  int i;
+};
+__device__ __forceinline__ bool am_better(float v, int i, float bv, int bi) {
+  return v > bv || (v == bv && i < bi);
+}
+__device__ __forceinline__ ArgMax warp_argmax(ArgMax a) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    float v = __shfl_xor_sync(0xffffffffu, a.v, o);
+    int i = __shfl_xor_sync(0xffffffffu, a.i, o);
+    if (am_better(v, i, a.v, a.i)) { a.v = v; a.i = i; }
+  }
+  return a;
+}
+
+// Block-wide reductions; `sh` needs 32 slots.  Every thread gets the result.
+__device__ __forceinline__ float block_sum(float v, float* sh) {
+  int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  v = warp_sum(v);
+  __syncthreads();
+  if (lane == 0) sh[w] = v;
+  __syncthreads();
+  v = (lane < nw) ? sh[lane] : 0.f;
+  v = warp_sum(v);
+  return v;
+}
+__device__ __forceinline__ double block_sum_d(double v, double* sh) {
+  int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  v = warp_sum_d(v);
+  __syncthreads();
+  if (lane == 0) sh[w] = v;
+  __syncthreads();
+  v = (lane < nw) ? sh[lane] : 0.0;
+  v = warp_sum_d(v);
+  return v;
+}
+__device__ __forceinline__ float block_max(float v, float* sh) {
+  int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  v = warp_max(v);
+  __syncthreads();
+  if (lane == 0) sh[w] = v;
+  __syncthreads();
+  v = (lane < nw) ? sh[lane] : -INFINITY;
+  v = warp_max(v);
+  return v;
+}
+__device__ __forceinline__ ArgMax block_argmax(ArgMax a, float* shv, int* shi) {
+  int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  a = warp_argmax(a);
+  __syncthreads();
+  if (lane == 0) { shv[w] = a.v; shi[w] = a.i; }
+  __syncthreads();
+  if (lane < nw) { a.v = shv[lane]; a.i = shi[lane]; } else { a.v = -INFINITY; a.i = 0x7fffffff; }
+  a = warp_argmax(a);
+  return a;
+}
+
+__device__ __forceinline__ float gelu_tanh(float u) {
+  const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
+  return 0.5f * u * (1.f + tanhf(k0 * (u + 0.044715f * u * u * u)));
+}
+__device__ __forceinline__ float silu(float u) { return u / (1.f + expf(-u)); }
+
+}  // namespace fm

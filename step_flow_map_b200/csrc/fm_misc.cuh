@@ -1,0 +1,228 @@
+// Row kernels of the drafter: time conditioning, modulated LayerNorm,
+// softmax, token selection, and a tiled transpose.
+#pragma once
+#include "fm_common.cuh"
+
+namespace fm {
+
+// ------------------------------------------------------------------ conditioning
+// 256-wide time features of s and t: [cos(1000 tau f_j), sin(1000 tau f_j)],
+// f_j = 10000^(-j/128), evaluated in fp64.
+__global__ void k_time_features(double s, double t, float* __restrict__ phi) {
+  int e = threadIdx.x;  // 0..255
+  int j = e & 127;
+  double f = exp(-log(10000.0) * (double)j / 128.0);
+  for (int w = 0; w < 2; ++w) {
+    double a = 1000.0 * (w == 0 ? s : t) * f;
+    phi[w * 256 + e] = (float)(e < 128 ? cos(a) : sin(a));
+  }
+}
+
+// y[o] = act(sum_i W[o][i] * x[i]) (+ add[o]); one warp per output row.
+// act: 0 = identity, 1 = SiLU.  x may be pre-activated by the caller.
+template <typename T>
+__global__ void k_gemv(const T* __restrict__ W, int n_out, int n_in, const float* __restrict__ x,
+                       float* __restrict__ y, const float* __restrict__ add, int act) {
+  int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= n_out) return;
+  const T* row = W + (size_t)warp * n_in;
+  float s = 0.f;
+  for (int i = lane; i < n_in; i += 32) s = fmaf(to_f(row[i]), x[i], s);
+  s = warp_sum(s);
+  if (lane == 0) {
+    if (act == 1) s = silu(s);
+    if (add) s += add[warp];
+    y[warp] = s;
+  }
+}
+
+__global__ void k_silu_vec(const float* __restrict__ x, float* __restrict__ y, int n) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = silu(x[i]);
+}
+
+// ------------------------------------------------------------------ LayerNorm
+// out[m] = LN0(x[m]) * (1 + scale) + shift, LN0 without affine part, eps 1e-6,
+// mean and variance in fp32 by two passes over the row held in registers.
+// shift/scale may be null (plain LN0).  One CTA of 256 threads per row.
+template <typename TI, typename TO>
+__global__ void __launch_bounds__(256)
+k_adaln(const TI* __restrict__ x, int d, const float* __restrict__ shift,
+        const float* __restrict__ scale, TO* __restrict__ out) {
+  __shared__ float sh[32];
+  const int m = blockIdx.x;
+  const TI* row = x + (size_t)m * d;
+  float s = 0.f;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) s += to_f(row[c]);
+  const float mean = block_sum(s, sh) / (float)d;
+  float v = 0.f;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    float t = to_f(row[c]) - mean;
+    v = fmaf(t, t, v);
+  }
+  const float var = block_sum(v, sh) / (float)d;
+  const float rstd = rsqrtf(var + 1e-6f);
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    float y = (to_f(row[c]) - mean) * rstd;
+    if (scale) y = y * (1.f + scale[c]) + shift[c];
+    out[(size_t)m * d + c] = from_f<TO>(y);
+  }
+}
+
+// ------------------------------------------------------------------ softmax rows
+// D[m] = softmax(logits[m]) at temperature 1, stored as dtype (the flow-map
+// denoiser output used by the next step's embedding).
+template <typename TO>
+__global__ void __launch_bounds__(1024)
+k_softmax_rows(const float* __restrict__ logits, int V, TO* __restrict__ D) {
+  __shared__ float sh[32];
+  const float* row = logits + (size_t)blockIdx.x * V;
+  float mx = -INFINITY;
+  for (int v = threadIdx.x; v < V; v += blockDim.x) mx = fmaxf(mx, row[v]);
+  mx = block_max(mx, sh);
+  float s = 0.f;
+  for (int v = threadIdx.x; v < V; v += blockDim.x) s += __expf(row[v] - mx);
+  s = block_sum(s, sh);
+  const float inv = 1.f / s;
+  TO* out = D + (size_t)blockIdx.x * V;
+  for (int v = threadIdx.x; v < V; v += blockDim.x) out[v] = from_f<TO>(__expf(row[v] - mx) * inv);
+}
+
+// ------------------------------------------------------------------ inverse CDF
+// Smallest v whose running sum of w(v), in vocabulary order, exceeds
+// `target`; if rounding leaves none, the last v with w(v) > 0.  Each thread
+// owns one contiguous chunk; chunk sums are scanned across the block in fp64
+// and the owning chunk is rescanned.  All threads return the answer.
+template <class WF>
+__device__ int block_inverse_cdf(const WF& w, int V, double target) {
+  __shared__ double wsum[32];
+  __shared__ int found;
+  __shared__ int lastpos;
+  const int nt = blockDim.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int chunk = (V + nt - 1) / nt;
+  const int v0 = min(V, tid * chunk), v1 = min(V, v0 + chunk);
+  double local = 0.0;
+  int last = -1;
+  for (int v = v0; v < v1; ++v) {
+    double x = w(v);
+    local += x;
+    if (x > 0.0) last = v;
+  }
+  // inclusive warp scan, then across warps
+  double incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    double y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (tid == 0) { found = 0x7fffffff; lastpos = -1; }
+  if (lane == 31) wsum[wid] = incl;
+  __syncthreads();
+  if (wid == 0) {
+    int nw = (nt + 31) >> 5;
+    double t = (lane < nw) ? wsum[lane] : 0.0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      double y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    if (lane < nw) wsum[lane] = t;  // inclusive totals per warp
+  }
+  __syncthreads();
+  if (wid > 0) incl += wsum[wid - 1];
+  double prev = __shfl_up_sync(0xffffffffu, incl, 1);
+  if (lane == 0) prev = (wid > 0) ? wsum[wid - 1] : 0.0;
+  if (incl > target && v1 > v0) atomicMin(&found, tid);
+  if (last >= 0) atomicMax(&lastpos, last);
+  __syncthreads();
+  __shared__ int pick_sh;
+  const int owner = found;
+  if (owner != 0x7fffffff) {
+    if (tid == owner) {
+      double r = 0.0;
+      int pick = -1, lp = -1;
+      for (int v = v0; v < v1; ++v) {
+        double x = w(v);
+        r += x;
+        if (x > 0.0) lp = v;
+        if (prev + r > target) { pick = v; break; }
+      }
+      if (pick < 0) pick = lp >= 0 ? lp : v0;  // rounding tie at the chunk end
+      pick_sh = pick;
+    }
+  } else if (tid == 0) {
+    pick_sh = lastpos >= 0 ? lastpos : 0;
+  }
+  __syncthreads();
+  const int ans = pick_sh;
+  __syncthreads();
+  return ans;
+}
+
+// ------------------------------------------------------------------ token choice
+struct TempArgs {
+  int n_noise, K;
+  float temp[256];  // per call-sequence; 0 = greedy
+};
+
+// One CTA per row.  Greedy rows: argmax of the fp32 logits (ties lowest) or,
+// when `part_v` is given, of the per-tile partial maxima the LM-head
+// epilogue left.  Sampled rows: inverse CDF of softmax(logits / T) at u.
+__global__ void __launch_bounds__(1024)
+k_select_tokens(const float* __restrict__ logits, int V, const float* __restrict__ part_v,
+                const int* __restrict__ part_i, int n_part, const double* __restrict__ u,
+                TempArgs ta, int* __restrict__ tokens) {
+  __shared__ float shv[32];
+  __shared__ int shi[32];
+  __shared__ double shd[32];
+  const int m = blockIdx.x;
+  const int q = m / (ta.n_noise * ta.K);
+  const float T = ta.temp[q];
+  if (T == 0.f) {
+    ArgMax a{-INFINITY, 0x7fffffff};
+    if (part_v) {
+      for (int p = threadIdx.x; p < n_part; p += blockDim.x) {
+        float v = part_v[(size_t)m * n_part + p];
+        int i = part_i[(size_t)m * n_part + p];
+        if (am_better(v, i, a.v, a.i)) { a.v = v; a.i = i; }
+      }
+    } else {
+      const float* row = logits + (size_t)m * V;
+      for (int v = threadIdx.x; v < V; v += blockDim.x)
+        if (am_better(row[v], v, a.v, a.i)) { a.v = row[v]; a.i = v; }
+    }
+    a = block_argmax(a, shv, shi);
+    if (threadIdx.x == 0) tokens[m] = (a.i == 0x7fffffff) ? 0 : a.i;
+    return;
+  }
+  const float* row = logits + (size_t)m * V;
+  float mx = -INFINITY;
+  for (int v = threadIdx.x; v < V; v += blockDim.x) mx = fmaxf(mx, row[v]);
+  mx = block_max(mx, shv);
+  const double dm = (double)mx, dT = (double)T;
+  auto wf = [&](int v) { return exp(((double)row[v] - dm) / dT); };
+  double s = 0.0;
+  for (int v = threadIdx.x; v < V; v += blockDim.x) s += wf(v);
+  s = block_sum_d(s, shd);
+  int tok = block_inverse_cdf(wf, V, u[m] * s);
+  if (threadIdx.x == 0) tokens[m] = tok;
+}
+
+// ------------------------------------------------------------------ transpose
+// out[c][r] = in[r][c] for in [R][C]; 32 x 32 tiles.
+template <typename T>
+__global__ void k_transpose(const T* __restrict__ in, T* __restrict__ out, int R, int C) {
+  __shared__ T tile[32][33];
+  int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < R && c < C) tile[i][threadIdx.x] = in[(size_t)r * C + c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += 8) {
+    int c = c0 + i, r = r0 + threadIdx.x;
+    if (r < R && c < C) out[(size_t)c * R + r] = tile[threadIdx.x][i];
+  }
+}
+
+}  // namespace fm

@@ -13,7 +13,7 @@ def _case(shape, seed_round=0, ctx=6):
     w = dataclasses.replace(fs.WORKLOADS["tiny_f32"], shape=shape, ctx=ctx)
     W = fs.make_weights(shape, "f32", std=0.02)
     W = {k: v * 5.0 for k, v in W.items()}   # larger weights: non-trivial gates
-    hid = fs.prefill_hidden(w)[0]
+    hid = fs.prefill_hidden(w, 0)
     ri = fs.round_inputs(w, seed_round)
     return W, hid, ri.noise[0, 0]
 
@@ -40,7 +40,7 @@ def test_loops_match_vectorised_tiny_config():
     shape = w.shape
     W = fs.make_weights(shape, "f32")
     Wd = {k: np.asarray(v, dtype=np.float64) for k, v in W.items()}
-    hid = fs.prefill_hidden(w)[0]
+    hid = fs.prefill_hidden(w, 0)
     X0 = fs.round_inputs(w, 0).noise[0, 0]
     _, kv = fm.project_context(Wd, shape.n_blocks, hid)
     res = fm.draft(Wd, shape, kv, X0[None], w.t_grid)
