@@ -20,6 +20,7 @@ tokens plus the target's correction/bonus token.
 from __future__ import annotations
 
 import argparse
+import faulthandler
 import json
 import os
 import statistics
@@ -161,7 +162,9 @@ def run_fm(args, w, rank, world, local_rank):
     # contiguous halves only (greedy first, then sampled), as in the mixed workload
     assert sampled == list(range(len(greedy), B)) or not sampled
     t_setup = time.time()
+    log(f"{w.name}: generating weights")
     W = fs.make_weights(s, w.dtype)
+    log("loading context")
     max_new = max(1, min(1024, w.ctx))
     ctx = Context(s, w.dtype, W, max_ctx=w.ctx + max(w.new_rows, 1) + 8, max_seqs=B,
                   max_noise=N, max_new=max(max_new, w.new_rows))
@@ -171,6 +174,7 @@ def run_fm(args, w, rank, world, local_rank):
         for p0 in range(0, w.ctx, max_new):
             ctx.project([b], to_device(h[p0:p0 + max_new][None], w.dtype), [p0])
     torch.cuda.synchronize()
+    log("prefill done")
     stream = torch.cuda.current_stream()
 
     per_round_mb = (B * N * K * V * (2 if w.dtype == "bf16" else 4) + B * N * (K + 1) * V * 4) / 2**20
@@ -229,6 +233,7 @@ def run_fm(args, w, rank, world, local_rank):
         return float(t.item())
 
     setup_s = time.time() - t_setup
+    log(f"{R} rounds prepared in {setup_s:.1f} s; timing")
     for k in range(args.warmup):
         step(rounds[k % R], k, n_acc_all[k])
     ab = algorithmic_bytes(w)
@@ -300,6 +305,7 @@ def run_fm(args, w, rank, world, local_rank):
     }
 
     # end to end: host inputs in pinned memory, copies inside the timed region
+    log(f"device-resident: {ms / args.steps:.4f} ms/step")
     if not args.no_e2e:
         RE = min(R, 8)
         pin = []
@@ -397,7 +403,12 @@ def run_reference(args, w):
                     "d2h_bytes_per_step": 0}}
 
 
+def log(msg):
+    print(f"[bench] {msg}", file=sys.stderr, flush=True)
+
+
 def main():
+    faulthandler.enable()
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -411,6 +422,7 @@ def main():
     line = run_fm(args, w, rank, world, local_rank)
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline:
+            log("timing the oracle on host cores")
             times, cores = oracle_rounds(w, budget_s=args.cpu_seconds, max_rounds=64, warmup=0)
             line["cpu_baseline"] = {
                 "value": round(len(times) * w.n_noise / sum(times), 5), "unit": "blocks/s",

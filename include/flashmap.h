@@ -185,6 +185,12 @@ fm_status fm_verify_sample(fm_ctx *ctx, const float *target_logits, const float 
                            int32_t *n_acc, int32_t *branch, int32_t *out_tokens,
                            fm_stream stream);
 
+/* Reads and clears the context's device error word: FM_OK, or
+ * FM_ERR_TIMEOUT when a bounded wait inside a kernel gave up (the kernel
+ * then stopped early and its outputs are invalid).  Waits for the work
+ * queued on `stream`. */
+fm_status fm_device_status(fm_ctx *ctx, fm_stream stream);
+
 /* Kernel classes for launch counting and optional device timing. */
 #define FM_PROF_EMBED 0     /* soft-embedding GEMM x.E (and D.E of later steps) */
 #define FM_PROF_DIT_GEMM 1  /* QKV, O, MLP GEMMs of the DiT blocks */

@@ -124,7 +124,7 @@ def project_context(W: dict, n_blocks: int, hidden: np.ndarray):
     thirds of W_qkv,l (the same projections the block rows use).
     """
     L = hidden.shape[0]
-    flat = np.asarray(hidden, dtype=np.float64).reshape(L, -1)
+    flat = np.asarray(hidden, dtype=np.float64).reshape(L, hidden.shape[1] * hidden.shape[2])
     C = layer_norm0(flat @ W["W_fc"].T)
     d = C.shape[1]
     kv = []

@@ -24,7 +24,7 @@ FM_MAX_STEPS = 8
 
 EXPORTS = (
     "fm_load_weights", "fm_free", "fm_last_error", "fm_project_context",
-    "fm_draft", "fm_verify_greedy", "fm_verify_sample", "fm_profile", "fm_profile_read",
+    "fm_draft", "fm_verify_greedy", "fm_verify_sample", "fm_profile", "fm_profile_read", "fm_device_status",
 )
 FM_PROF = {"embed": 0, "dit_gemm": 1, "attn": 2, "norm": 3, "lm_head": 4, "context": 5,
            "verify": 6, "other": 7}
@@ -83,6 +83,8 @@ def load_library(path: str = LIB_PATH):
     lib.fm_verify_greedy.argtypes = [p, p, p, i, i, i, i, p, p, p, st]
     lib.fm_verify_sample.restype = i
     lib.fm_verify_sample.argtypes = [p, p, p, p, i, i, i, i, f, p, p, p, p, p, st]
+    lib.fm_device_status.restype = i
+    lib.fm_device_status.argtypes = [p, st]
     lib.fm_profile.restype = i
     lib.fm_profile.argtypes = [p, i]
     lib.fm_profile_read.restype = i
@@ -192,3 +194,8 @@ def fm_profile_read(ctx, reset: bool = False):
     n = (ctypes.c_int64 * FM_PROF_N)()
     _check(load_library().fm_profile_read(ctx, ms, n, int(bool(reset))))
     return list(ms), list(n)
+
+
+def fm_device_status(ctx, stream=None) -> None:
+    """Raise FlashmapError(FM_ERR_TIMEOUT) if a kernel's bounded wait gave up."""
+    _check(load_library().fm_device_status(ctx, _stream(stream)))

@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <vector>
@@ -317,8 +318,11 @@ fm_status load_impl(fm_ctx* c, cudaStream_t st) {
   FM_TRY(dalloc_t(c, &c->vs_pm, vrows * c->v_chunks));
   FM_TRY(dalloc_t(c, &c->vs_ps, vrows * c->v_chunks));
   FM_TRY(dalloc_t(c, &c->vs_resid, (size_t)g.max_seqs * 2 * g.V));
+  FM_TRY(dalloc_t(c, &c->tc.err, 1));
+  FM_CUDA(cudaMemsetAsync(c->tc.err, 0, sizeof(int), st));
   if constexpr (sizeof(T) == 2) {
-    c->use_tc = fm::tc_supported(g.d, g.mlp, g.V, g.n_taps * g.target_hidden);
+    const char* off = getenv("FM_DISABLE_TC");  // diagnostic: force the CUDA-core GEMMs
+    c->use_tc = fm::tc_supported(g.d, g.mlp, g.V, g.n_taps * g.target_hidden) && !(off && *off == '1');
     if (c->use_tc) {
       if (!fm::tc_make_maps(c->tc, c->w.W_lm, c->Et, c->w.W_fc, c->wqkv.data(), c->wo.data(),
                             c->wup.data(), c->wdown.data(), g.n_blocks, g.d, g.mlp, g.V,
@@ -409,9 +413,14 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
     const float* mods;
     FM_TRY(get_mods<T>(c, s, t, &mods, st));
     // input embedding (first step: x0 E; later: flow-map update through E)
-    fm::EpiEmbed emb{c->x, num_steps > 1 ? c->z : nullptr, c->P, d, K,
-                     k == 0 ? -1.f : (float)((double)(t - s) / (1.0 - (double)s))};
-    if (k == 0) emb.alpha = -1.f;
+    // the state entering step k moved by the previous step's flow-map update,
+    // alpha = (t_k - t_{k-1}) / (1 - t_{k-1})
+    float alpha = -1.f;
+    if (k > 0) {
+      const double sp = t_grid[k - 1], tp = t_grid[k];
+      alpha = (float)((tp - sp) / (1.0 - sp));
+    }
+    fm::EpiEmbed emb{c->x, num_steps > 1 ? c->z : nullptr, c->P, d, K, alpha};
     const T* A = (k == 0) ? (const T*)noise : (const T*)c->D;
     if (c->use_tc && c->tc.embed.valid) {
       FM_TRY(gemm_w<T>(c, FM_PROF_EMBED, A, V, (const T*)c->Et, M, d, V, emb, st, &c->tc.embed));
@@ -687,6 +696,20 @@ extern "C" fm_status fm_profile_read(fm_ctx* c, double* ms, int64_t* launches, i
   if (reset) {
     for (int k = 0; k < FM_PROF_N; ++k) c->launches[k] = 0;
     c->ev_used = 0;
+  }
+  return FM_OK;
+}
+
+extern "C" fm_status fm_device_status(fm_ctx* c, fm_stream stream) {
+  if (!c) return set_err(FM_ERR_ARG, "NULL context");
+  int v = 0;
+  cudaStream_t st = (cudaStream_t)stream;
+  FM_CUDA(cudaMemcpyAsync(&v, c->tc.err, sizeof(int), cudaMemcpyDeviceToHost, st));
+  FM_CUDA(cudaStreamSynchronize(st));
+  if (v) {
+    FM_CUDA(cudaMemsetAsync(c->tc.err, 0, sizeof(int), st));
+    FM_CUDA(cudaStreamSynchronize(st));
+    return set_err(FM_ERR_TIMEOUT, "a bounded wait inside a tensor-core kernel gave up (code %d)", v);
   }
   return FM_OK;
 }

@@ -1,34 +1,583 @@
-// Tensor-core (tcgen05) weight GEMM: placeholder until the sm_100a kernel lands.
+// Tensor-core weight GEMM for sm_100a: tcgen05.mma with TMEM accumulators,
+// operands staged in shared memory by TMA.
+//
+// Y[M][N] = A[M][K] . W[N][K]^T with both operands K-major bf16 and fp32
+// accumulation.  The drafter's GEMMs stream a large weight through a few
+// activation rows (M = 16 at concurrency 1), so the weight takes the MMA's
+// 128-row side ("swap-AB"): each tile is D[128 features][BN rows] =
+// W_tile[128][K] . A_tile[BN][K]^T.  Few output tiles (x.E has 16 at d=2048)
+// are spread over all SMs by splitting K; the last CTA to finish a tile
+// (arrival counter, no waiting) sums the fp32 partials in split order and
+// runs the epilogue, so results do not depend on scheduling.
+//
+// Roles per CTA (192 threads, one CTA per SM, persistent over work units):
+//   warp 0     TMA producer (one lane) filling a ring of smem stages
+//   warp 1     TMEM allocator and MMA issuer (one lane)
+//   warps 2-5  epilogue: TMEM -> registers -> epilogue functor
+// Two TMEM accumulators let the epilogue of one unit overlap the MMAs of the
+// next.  Every mbarrier wait is bounded in time; on expiry the CTA records
+// an error code, lets in-flight copies land, frees its TMEM and exits.
 #pragma once
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <stdio.h>
+
+#include <type_traits>
 #include <vector>
+
 #include "fm_common.cuh"
 
 namespace fm {
 
+constexpr int TC_BM = 128;       // weight rows (output features) per tile
+constexpr int TC_BK = 64;        // reduction elements per stage: one 128-byte swizzle row
+constexpr int TC_THREADS = 192;
+constexpr unsigned long long TC_TIMEOUT_NS = 2000000000ull;
+constexpr int TC_ERR_TIMEOUT = 1;
+
+// ------------------------------------------------------------------ host-side maps
 struct TcMap {
   bool valid = false;
+  CUtensorMap map;
+  int N = 0, Kd = 0;
 };
 struct TcMaps {
   TcMap embed, lm, fc;
   std::vector<TcMap> qkv, kv, o, up, down;
-  TcMaps() : qkv(64), kv(64), o(64), up(64), down(64) {}
+  int* err = nullptr;  // device error word shared by all tensor-core launches
 };
 
-inline bool tc_supported(int, int, int, int) { return false; }
-inline bool tc_make_maps(TcMaps&, const void*, const void*, const void*, const void* const*,
-                         const void* const*, const void* const*, const void* const*, int, int, int,
-                         int, int, char*, size_t) {
+// ------------------------------------------------------------------ device helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ unsigned long long gtimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Waits for the phase with the given parity; false when it timed out or
+// another role of the CTA already gave up.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try(bar, parity)) return true;
+  const unsigned long long t0 = gtimer();
+  while (!mbar_try(bar, parity)) {
+    if (*abort) return false;
+    if (gtimer() - t0 > TC_TIMEOUT_NS) {
+      *abort = 1;
+      return false;
+    }
+  }
+  return true;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4}], [%2];" ::"r"(dst),
+      "l"((unsigned long long)map), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+// 16 consecutive fp32 columns of this thread's TMEM lane; the wait is part of
+// the same statement so the registers are complete when it returns.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand written by TMA with the
+// 128-byte swizzle, rows of 64 bf16, 8-row groups 1024 bytes apart.
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor: bf16 x bf16 -> fp32, both K-major, M = 128, N = BN.
+template <int BN>
+__host__ __device__ constexpr uint32_t idesc_bf16() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+// ------------------------------------------------------------------ epilogue for the LM head
+// Per activation row and 128-token tile: the largest logit and its lowest
+// index.  The logits themselves never reach HBM.
+struct EpiArgmax {
+  float* part_v;  // [M][n_part]
+  int* part_i;
+  int n_part;
+};
+template <class E>
+struct is_argmax : std::false_type {};
+template <>
+struct is_argmax<EpiArgmax> : std::true_type {};
+
+struct TcArgs {
+  int M, N, Kd;
+  int n_tiles, m_tiles, splits, k_blocks, units;
+  float* partial;       // [splits][tiles][128][BN] fp32 (splits > 1)
+  unsigned* tile_cnt;   // [tiles], zero between launches
+  int* err;
+};
+
+template <int BN>
+struct TcCfg {
+  static constexpr int A_BYTES = TC_BM * TC_BK * 2;  // 16 KB
+  static constexpr int B_BYTES = BN * TC_BK * 2;
+  static constexpr int STAGE = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (200 * 1024) / STAGE > 12 ? 12 : (200 * 1024) / STAGE;
+  static constexpr int TMEM_COLS = (2 * BN) < 32 ? 32 : 2 * BN;
+  static constexpr int SMEM = STAGES * STAGE + 1024 /*align*/ + 256 /*barriers*/ + 8 * BN * 4;
+};
+
+template <int BN, class Epi>
+__device__ __forceinline__ void tc_finish_chunk(const Epi& epi, const TcArgs& a, int n0, int m0,
+                                                int r, int j0, const float* v, float* red_v,
+                                                int* red_i, int q) {
+  const int n = n0 + r;
+  if constexpr (is_argmax<Epi>::value) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      ArgMax am{n < a.N ? v[j] : -INFINITY, n < a.N ? n : 0x7fffffff};
+      am = warp_argmax(am);
+      if (lane == 0) {
+        red_v[q * BN + j0 + j] = am.v;
+        red_i[q * BN + j0 + j] = am.i;
+      }
+    }
+  } else {
+    if (n >= a.N) return;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int m = m0 + j0 + j;
+      if (m < a.M) epi(m, n, v[j]);
+    }
+  }
+}
+
+template <int BN, class Epi>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+k_tc_gemm(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUtensorMap mapA,
+          TcArgs a, Epi epi) {
+  using C = TcCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sA = base;
+  uint8_t* sB = base + C::STAGES * C::A_BYTES;
+  uint64_t* bars = (uint64_t*)(base + C::STAGES * C::STAGE);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + C::STAGES;
+  uint64_t* tfull = bars + 2 * C::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = (uint32_t*)(tempty + 2);
+  volatile int* abort = (volatile int*)(tmem_slot + 1);
+  int* s_last = (int*)(tmem_slot + 2);
+  volatile int* s_ok = (volatile int*)(tmem_slot + 3);
+  float* red_v = (float*)(base + C::STAGES * C::STAGE + 256);
+  int* red_i = (int*)(red_v + 4 * BN);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&tfull[i]), 1);
+      mbar_init(smem_u32(&tempty[i]), 128);
+    }
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int tiles = a.n_tiles * a.m_tiles;
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"((unsigned long long)&mapW) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"((unsigned long long)&mapA) : "memory");
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int u = blockIdx.x; u < a.units && !*abort; u += gridDim.x) {
+        const int mt = u % a.m_tiles, rest = u / a.m_tiles;
+        const int z = rest % a.splits, nt = rest / a.splits;
+        const int kb0 = (int)((long)z * a.k_blocks / a.splits);
+        const int kb1 = (int)((long)(z + 1) * a.k_blocks / a.splits);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort)) break;
+          const uint32_t fb = smem_u32(&full[stage]);
+          mbar_expect_tx(fb, C::STAGE);
+          tma_load_2d(smem_u32(sA + stage * C::A_BYTES), &mapW, kb * TC_BK, nt * TC_BM, fb);
+          tma_load_2d(smem_u32(sB + stage * C::B_BYTES), &mapA, kb * TC_BK, mt * BN, fb);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16<BN>();
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      for (int u = blockIdx.x; u < a.units && !*abort; u += gridDim.x) {
+        const int z = (u / a.m_tiles) % a.splits;
+        const int kb0 = (int)((long)z * a.k_blocks / a.splits);
+        const int kb1 = (int)((long)(z + 1) * a.k_blocks / a.splits);
+        if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1, abort)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + acc * BN;
+        bool ok = true;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(smem_u32(&full[stage]), phase, abort)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t ad = desc_sw128(smem_u32(sA + stage * C::A_BYTES));
+          const uint64_t bd = desc_sw128(smem_u32(sB + stage * C::B_BYTES));
+#pragma unroll
+          for (int k = 0; k < TC_BK / 16; ++k)
+            tc_mma(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          tc_commit(smem_u32(&empty[stage]));
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        tc_commit(smem_u32(&tfull[acc]));
+        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5 = TMEM lane quadrants 2, 3, 0, 1)
+    const int q = warp & 3;
+    const int r = q * 32 + lane;          // feature row within the tile
+    const int et = threadIdx.x - 64;      // 0..127
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int u = blockIdx.x; u < a.units && !*abort; u += gridDim.x) {
+      const int mt = u % a.m_tiles, rest = u / a.m_tiles;
+      const int z = rest % a.splits, nt = rest / a.splits;
+      const int n0 = nt * TC_BM, m0 = mt * BN;
+      const int tile = nt * a.m_tiles + mt;
+      // one waiter, then a barrier the 128 threads always reach together
+      if (et == 0) *s_ok = mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort) ? 1 : 0;
+      named_sync(1, 128);
+      if (!*s_ok) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + acc * BN;
+      float v[16];
+      if (a.splits == 1) {
+        for (int j0 = 0; j0 < BN; j0 += 16) {
+          tmem_ld16(taddr + j0, v);
+          tc_finish_chunk<BN>(epi, a, n0, m0, r, j0, v, red_v, red_i, q);
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&tempty[acc]));
+      } else {
+        float* mine = a.partial + (((size_t)z * tiles + tile) * TC_BM + r) * BN;
+        for (int j0 = 0; j0 < BN; j0 += 16) {
+          tmem_ld16(taddr + j0, v);
+#pragma unroll
+          for (int j = 0; j < 16; j += 4)
+            *(float4*)(mine + j0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&tempty[acc]));
+        __threadfence();
+        named_sync(1, 128);
+        if (et == 0) {
+          unsigned prev = atomicAdd(&a.tile_cnt[tile], 1u);
+          *s_last = (prev == (unsigned)(a.splits - 1));
+        }
+        named_sync(1, 128);
+        const int last = *s_last;
+        if (last) {
+          __threadfence();
+          for (int j0 = 0; j0 < BN; j0 += 16) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = 0.f;
+            for (int zz = 0; zz < a.splits; ++zz) {
+              const float* p = a.partial + (((size_t)zz * tiles + tile) * TC_BM + r) * BN + j0;
+#pragma unroll
+              for (int j = 0; j < 16; j += 4) {
+                float4 t = __ldcg((const float4*)(p + j));
+                v[j] += t.x; v[j + 1] += t.y; v[j + 2] += t.z; v[j + 3] += t.w;
+              }
+            }
+            tc_finish_chunk<BN>(epi, a, n0, m0, r, j0, v, red_v, red_i, q);
+          }
+          if (et == 0) a.tile_cnt[tile] = 0u;
+        }
+        if (!last) {
+          if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+          continue;
+        }
+      }
+      if constexpr (is_argmax<Epi>::value) {
+        named_sync(1, 128);
+        for (int j = et; j < BN; j += 128) {
+          float bv = red_v[j];
+          int bi = red_i[j];
+          for (int qq = 1; qq < 4; ++qq)
+            if (am_better(red_v[qq * BN + j], red_i[qq * BN + j], bv, bi)) {
+              bv = red_v[qq * BN + j];
+              bi = red_i[qq * BN + j];
+            }
+          const int m = m0 + j;
+          if (m < a.M) {
+            epi.part_v[(size_t)m * epi.n_part + nt] = bv;
+            epi.part_i[(size_t)m * epi.n_part + nt] = bi;
+          }
+        }
+        named_sync(1, 128);
+      }
+      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+    }
+  }
+
+  // ---------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (*abort) {
+    if (threadIdx.x == 0) atomicExch(a.err, TC_ERR_TIMEOUT);
+    // let copies and MMAs already issued land before the memory goes away
+    const unsigned long long t0 = gtimer();
+    while (gtimer() - t0 < 50000ull) {
+    }
+    __syncthreads();
+  }
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+inline PFN_cuTensorMapEncodeTiled_v12000 tc_encoder(char* err, size_t errlen) {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p) {
+      snprintf(err, errlen, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorString(e));
+      return nullptr;
+    }
+    fn = (PFN_cuTensorMapEncodeTiled_v12000)p;
+  }
+  return fn;
+}
+
+// 2-D K-major bf16 map of a [rows][ld] matrix with `Kd` used columns; box 64 x box_rows.
+inline bool tc_encode(CUtensorMap* m, const void* ptr, int Kd, int rows, int ld, int box_rows,
+                      char* err, size_t errlen) {
+  auto enc = tc_encoder(err, errlen);
+  if (!enc) return false;
+  if (((uintptr_t)ptr & 15) || (ld % 8)) {
+    snprintf(err, errlen, "tensor map: base %p / leading dim %d not 16-byte aligned", ptr, ld);
+    return false;
+  }
+  cuuint64_t dims[2] = {(cuuint64_t)Kd, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {(cuuint32_t)TC_BK, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(err, errlen, "cuTensorMapEncodeTiled failed (%d) for %d x %d ld %d", (int)r, rows, Kd, ld);
+    return false;
+  }
+  return true;
+}
+
+inline bool tc_supported(int d, int mlp, int V, int in_fc) {
+  return d % 128 == 0 && mlp % 128 == 0 && V % 128 == 0 && d % 8 == 0 && mlp % 8 == 0 &&
+         V % 8 == 0 && in_fc % 8 == 0;
+}
+
+inline bool tc_weight_map(TcMap& t, const void* W, int N, int Kd, char* err, size_t errlen) {
+  t.N = N;
+  t.Kd = Kd;
+  t.valid = tc_encode(&t.map, W, Kd, N, Kd, TC_BM, err, errlen);
+  return t.valid;
+}
+
+inline bool tc_make_maps(TcMaps& m, const void* W_lm, const void* Et, const void* W_fc,
+                         const void* const* wqkv, const void* const* wo, const void* const* wup,
+                         const void* const* wdown, int nb, int d, int mlp, int V, int in_fc,
+                         char* err, size_t errlen) {
+  if (!tc_weight_map(m.lm, W_lm, V, d, err, errlen)) return false;
+  if (!tc_weight_map(m.embed, Et, d, V, err, errlen)) return false;
+  if (!tc_weight_map(m.fc, W_fc, d, in_fc, err, errlen)) return false;
+  m.qkv.resize(nb);
+  m.kv.resize(nb);
+  m.o.resize(nb);
+  m.up.resize(nb);
+  m.down.resize(nb);
+  for (int l = 0; l < nb; ++l) {
+    if (!tc_weight_map(m.qkv[l], wqkv[l], 3 * d, d, err, errlen)) return false;
+    if (!tc_weight_map(m.kv[l], (const bf16*)wqkv[l] + (size_t)d * d, 2 * d, d, err, errlen))
+      return false;
+    if (!tc_weight_map(m.o[l], wo[l], d, d, err, errlen)) return false;
+    if (!tc_weight_map(m.up[l], wup[l], mlp, d, err, errlen)) return false;
+    if (!tc_weight_map(m.down[l], wdown[l], d, mlp, err, errlen)) return false;
+  }
   return true;
 }
 inline void tc_free_maps(TcMaps&) {}
-template <class Epi>
-fm_status tc_gemm(const TcMaps&, const TcMap&, const bf16*, int, int, int, int, Epi, float*, size_t,
-                  unsigned*, int, int, cudaStream_t, char*, size_t, int*) {
-  return FM_ERR_UNSUPPORTED;
+
+inline int tc_pick_bn(int M) {
+  if (M <= 16) return 16;
+  if (M <= 32) return 32;
+  if (M <= 64) return 64;
+  if (M <= 128) return 128;
+  return 256;
 }
-inline fm_status tc_lm_head_argmax(const TcMaps&, const bf16*, int, int, int, float*, int*, int,
-                                   int, cudaStream_t, char*, size_t, int*) {
-  return FM_ERR_UNSUPPORTED;
+
+template <int BN, class Epi>
+fm_status tc_launch(const TcMap& wm, const bf16* A, int lda, int M, Epi epi, float* partial,
+                    size_t partial_elems, unsigned* tile_cnt, int tile_cnt_n, int sms, int* err_word,
+                    cudaStream_t st, char* err, size_t errlen, int* n_launch) {
+  using C = TcCfg<BN>;
+  TcArgs a;
+  a.M = M;
+  a.N = wm.N;
+  a.Kd = wm.Kd;
+  a.n_tiles = (wm.N + TC_BM - 1) / TC_BM;
+  a.m_tiles = (M + BN - 1) / BN;
+  a.k_blocks = (wm.Kd + TC_BK - 1) / TC_BK;
+  const int tiles = a.n_tiles * a.m_tiles;
+  int splits = 1;
+  if (tiles < sms) {
+    splits = sms / tiles;
+    splits = splits > a.k_blocks ? a.k_blocks : splits;
+    while (splits > 1 && (size_t)splits * tiles * TC_BM * BN > partial_elems) --splits;
+  }
+  if (splits > 1 && tiles > tile_cnt_n) splits = 1;
+  a.splits = splits < 1 ? 1 : splits;
+  a.units = tiles * a.splits;
+  a.partial = partial;
+  a.tile_cnt = tile_cnt;
+  a.err = err_word;
+  CUtensorMap mapA;
+  if (!tc_encode(&mapA, A, wm.Kd, M, lda, BN, err, errlen)) return FM_ERR_CUDA;
+  {
+    cudaError_t e = cudaFuncSetAttribute(k_tc_gemm<BN, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM);
+    if (e != cudaSuccess) {
+      snprintf(err, errlen, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+      return FM_ERR_CUDA;
+    }
+  }
+  const int grid = a.units < sms ? a.units : sms;
+  k_tc_gemm<BN, Epi><<<grid, TC_THREADS, C::SMEM, st>>>(wm.map, mapA, a, epi);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    snprintf(err, errlen, "tensor-core GEMM launch: %s", cudaGetErrorString(e));
+    return FM_ERR_CUDA;
+  }
+  if (n_launch) ++*n_launch;
+  return FM_OK;
+}
+
+template <class Epi>
+fm_status tc_gemm(const TcMaps& maps, const TcMap& wm, const bf16* A, int lda, int M, int N, int Kd,
+                  Epi epi, float* partial, size_t partial_elems, unsigned* tile_cnt, int tile_cnt_n,
+                  int sms, cudaStream_t st, char* err, size_t errlen, int* n_launch) {
+  if (N != wm.N || Kd != wm.Kd) {
+    snprintf(err, errlen, "tensor-core GEMM: shape %d x %d does not match its weight map %d x %d", N,
+             Kd, wm.N, wm.Kd);
+    return FM_ERR_ARG;
+  }
+  switch (tc_pick_bn(M)) {
+    case 16: return tc_launch<16>(wm, A, lda, M, epi, partial, partial_elems, tile_cnt, tile_cnt_n, sms, maps.err, st, err, errlen, n_launch);
+    case 32: return tc_launch<32>(wm, A, lda, M, epi, partial, partial_elems, tile_cnt, tile_cnt_n, sms, maps.err, st, err, errlen, n_launch);
+    case 64: return tc_launch<64>(wm, A, lda, M, epi, partial, partial_elems, tile_cnt, tile_cnt_n, sms, maps.err, st, err, errlen, n_launch);
+    case 128: return tc_launch<128>(wm, A, lda, M, epi, partial, partial_elems, tile_cnt, tile_cnt_n, sms, maps.err, st, err, errlen, n_launch);
+    default: return tc_launch<256>(wm, A, lda, M, epi, partial, partial_elems, tile_cnt, tile_cnt_n, sms, maps.err, st, err, errlen, n_launch);
+  }
+}
+
+inline fm_status tc_lm_head_argmax(const TcMaps& maps, const bf16* h, int lda, int M, int V,
+                                   float* part_v, int* part_i, int n_part, int sms, cudaStream_t st,
+                                   char* err, size_t errlen, int* n_launch) {
+  EpiArgmax epi{part_v, part_i, n_part};
+  // no split-K: the vocabulary supplies enough tiles
+  return tc_gemm(maps, maps.lm, h, lda, M, V, maps.lm.Kd, epi, nullptr, 0, nullptr, 0, sms, st, err,
+                 errlen, n_launch);
 }
 
 }  // namespace fm

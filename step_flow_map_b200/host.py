@@ -19,12 +19,13 @@ FM_DTYPE = {"f32": FM_F32, "bf16": FM_BF16}
 def to_device(a, dtype: str = "f32", device="cuda") -> torch.Tensor:
     """Host array -> contiguous device tensor of storage type ``dtype``.
 
-    For bf16 the values must already be bf16-representable; the cast is
-    then exact.
+    fp64 arrays (uniforms) stay fp64; integer arrays keep their type; other
+    floating arrays become ``dtype``.  For bf16 the values must already be
+    bf16-representable; the cast is then exact.
     """
     t = torch.from_numpy(np.ascontiguousarray(a))
-    if t.dtype == torch.float64:
-        t = t.to(torch.float32)
+    if t.dtype == torch.float64:   # uniforms cross the ABI as fp64
+        return t.to(device=device).contiguous()
     t = t.to(device=device, dtype=TORCH_DTYPE[dtype] if t.is_floating_point() else t.dtype)
     return t.contiguous()
 

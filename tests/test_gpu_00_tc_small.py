@@ -1,0 +1,83 @@
+"""Tensor-core (tcgen05) GEMM path on a small bf16 drafter, against the oracle.
+
+Runs before the full-size tests: every GEMM of the draft (context fc and
+keys/values, x.E with split-K, QKV/O/MLP, LM head with stored logits and
+with the fused argmax) goes through the tensor-core kernel at several
+activation-row counts (BN = 16, 64, 256 with a ragged tail).
+"""
+import dataclasses
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import fm_synth as fs
+from oracle import flashmap as om
+from step_flow_map_b200 import fm_device_status
+from step_flow_map_b200.host import Context, to_device
+
+import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+SMALL = fs.Shape(V=1024, d=128, n_blocks=2, n_heads=1, mlp=256, K=16, hidden=64)
+
+
+def _workload(B, N, t_grid=(0.0, 1.0), temps=None, ctx=40):
+    return dataclasses.replace(fs.WORKLOADS["qwen3_8b_bs1"], name="small_bf16", shape=SMALL,
+                               B=B, n_noise=N, ctx=ctx, new_rows=17, t_grid=t_grid,
+                               temps=temps or tuple([0.0] * B))
+
+
+def _run(w, env_off=False, logits=True):
+    if env_off:
+        os.environ["FM_DISABLE_TC"] = "1"
+    try:
+        ctx = gu.make_ctx(w, max_new=64)
+    finally:
+        os.environ.pop("FM_DISABLE_TC", None)
+    seqs = list(range(w.B))
+    gu.gpu_prefill(ctx, w, seqs, max_new=64)
+    gu.gpu_new_rows(ctx, w, 0, seqs)
+    ri = fs.round_inputs(w, 0)
+    tok, lg = ctx.draft(seqs, to_device(ri.noise, "bf16"), w.t_grid, w.temps,
+                        u_draft=to_device(ri.u_draft), logits=logits)
+    torch.cuda.synchronize()
+    fm_device_status(ctx.ctx)
+    out = (gu.to_np(tok), None if lg is None else gu.to_np(lg))
+    ctx.close()
+    return out, ri
+
+
+@pytest.mark.parametrize("B,N", [(1, 1), (1, 4), (9, 2)])
+def test_tc_draft_matches_oracle(B, N):
+    w = _workload(B, N)
+    (tok, lg), ri = _run(w)
+    for b in sorted({0, B - 1}):
+        ref = gu.oracle_draft(w, b, 0)
+        gu.assert_logits_close(lg[b], ref["logits"], "bf16", f"seq {b}")
+        gu.assert_tokens_on_margin(tok[b], ref["logits"], f"seq {b}")
+    # the fused LM-head argmax (no logits written) picks the same tokens
+    (tok2, none), _ = _run(w, logits=False)
+    assert none is None
+    np.testing.assert_array_equal(tok2, tok)
+
+
+def test_tc_matches_cuda_core_path():
+    w = _workload(2, 1)
+    (tok_tc, lg_tc), _ = _run(w)
+    (tok_cc, lg_cc), _ = _run(w, env_off=True)
+    np.testing.assert_allclose(lg_tc, lg_cc, atol=2e-2, rtol=1e-2)
+
+
+def test_tc_two_step():
+    w = _workload(1, 2, t_grid=(0.0, 0.5, 1.0), temps=(1.0,))
+    (tok, lg), ri = _run(w)
+    ref = gu.oracle_draft(w, 0, 0)
+    gu.assert_logits_close(lg[0], ref["logits"], "bf16", "two-step")
+    for j in range(w.n_noise):
+        for i in range(w.shape.K):
+            y, sure = gu.sampled_token_sure(ref["logits"][j, i], 1.0, ri.u_draft[0, j, i])
+            if sure:
+                assert tok[0, j, i] == y
