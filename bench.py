@@ -77,8 +77,10 @@ class ClockSampler:
             import pynvml
             import torch
             pynvml.nvmlInit()
-            bus = torch.cuda.get_device_properties(torch_dev).pci_bus_id
-            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            pr = torch.cuda.get_device_properties(torch_dev)
+            bus = "%08X:%02X:%02X.0" % (int(pr.pci_domain_id), int(pr.pci_bus_id),
+                                        int(pr.pci_device_id))
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
             self.nv = pynvml
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
             self.ok = True

@@ -13,6 +13,7 @@
 #include "fm_misc.cuh"
 #include "fm_verify.cuh"
 #include "fm_tc.cuh"
+#include "fm_attn.cuh"
 
 using fm::bf16;
 
@@ -86,6 +87,10 @@ struct fm_ctx {
   float* vg_pv = nullptr;
   int* vg_pi = nullptr;
   unsigned* vg_cnt = nullptr;
+  float* attn_part = nullptr;   // split-KV attention partials
+  unsigned* attn_cnt = nullptr;
+  size_t attn_part_elems = 0;
+  int attn_pairs_max = 0;
   float* vs_pm = nullptr;
   double* vs_ps = nullptr;
   double* vs_resid = nullptr;
@@ -306,6 +311,11 @@ fm_status load_impl(fm_ctx* c, cudaStream_t st) {
   c->tile_cnt_n = 1 << 16;
   FM_TRY(dalloc_t(c, &c->tile_cnt, c->tile_cnt_n));
   FM_CUDA(cudaMemsetAsync(c->tile_cnt, 0, c->tile_cnt_n * sizeof(unsigned), st));
+  c->attn_pairs_max = call_seqs * g.n_heads;
+  c->attn_part_elems = (size_t)(2 * c->sms + 2 * c->attn_pairs_max) * g.max_noise * 16 * (fm::AM_DH + 2);
+  FM_TRY(dalloc_t(c, &c->attn_part, c->attn_part_elems));
+  FM_TRY(dalloc_t(c, &c->attn_cnt, (size_t)c->attn_pairs_max));
+  FM_CUDA(cudaMemsetAsync(c->attn_cnt, 0, c->attn_pairs_max * sizeof(unsigned), st));
   FM_TRY(dalloc_t(c, &c->c_raw, (size_t)c->R_max * d));
   FM_TRY(dalloc(c, &c->c_norm, (size_t)c->R_max * d * sizeof(T)));
   // verify workspaces: rows = B*N*(K+1) target + B*N*K draft rows
@@ -373,6 +383,36 @@ fm_status project_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void
   return FM_OK;
 }
 
+// ------------------------------------------------------------------ attention
+template <int N>
+fm_status attn_mma_launch(fm_ctx* c, const fm::AttnMmaArgs& am, dim3 grid, const bf16* qkv,
+                          const bf16* Kc, const bf16* Vc, bf16* o, cudaStream_t st) {
+  constexpr int smem = fm::attn_mma_smem<N>();
+  FM_CUDA(cudaFuncSetAttribute(fm::k_attn_mma<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  FM_KERNEL(c, FM_PROF_ATTN, fm::k_attn_mma<N><<<grid, fm::AM_THREADS, smem, st>>>(qkv, Kc, Vc, o, am));
+  return FM_OK;
+}
+
+// Split count: about two CTAs per SM over all (sequence, head) pairs, at
+// most one 64-row chunk per split when the context is short.
+fm_status attn_mma(fm_ctx* c, int n_noise, fm::AttnMmaArgs am, const bf16* qkv, const bf16* Kc,
+                   const bf16* Vc, bf16* o, int n_seqs, int max_len, cudaStream_t st) {
+  const int pairs = n_seqs * am.n_heads;
+  int s_ctx = (2 * c->sms + pairs - 1) / pairs - 1;
+  s_ctx = std::min(s_ctx, (max_len + fm::AM_CHUNK - 1) / fm::AM_CHUNK);
+  s_ctx = std::max(s_ctx, 1);
+  while (s_ctx > 1 &&
+         (size_t)pairs * (s_ctx + 1) * n_noise * 16 * (fm::AM_DH + 2) > c->attn_part_elems)
+    --s_ctx;
+  am.n_ctx_splits = s_ctx;
+  dim3 grid(pairs, s_ctx + 1);
+  switch (n_noise) {
+    case 1: return attn_mma_launch<1>(c, am, grid, qkv, Kc, Vc, o, st);
+    case 2: return attn_mma_launch<2>(c, am, grid, qkv, Kc, Vc, o, st);
+    default: return attn_mma_launch<4>(c, am, grid, qkv, Kc, Vc, o, st);
+  }
+}
+
 // ------------------------------------------------------------------ draft
 template <typename T>
 fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* noise,
@@ -397,6 +437,27 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
   for (int q = 0; q < n_seqs; ++q) {
     aa.slot[q] = seq_ids[q];
     aa.len[q] = c->ctx_len[seq_ids[q]];
+  }
+  // tensor-core (mma.sync) split-KV attention for bf16, head width 128
+  const bool use_mma_attn = sizeof(T) == 2 && d / g.n_heads == fm::AM_DH && K == 16 &&
+                            (n_noise == 1 || n_noise == 2 || n_noise == 4);
+  fm::AttnMmaArgs am;
+  int max_len = 0;
+  if (use_mma_attn) {
+    am.n_seqs = n_seqs;
+    am.n_noise = n_noise;
+    am.K = K;
+    am.d = d;
+    am.n_heads = g.n_heads;
+    am.max_ctx = g.max_ctx;
+    am.scale_log2 = (float)(1.4426950408889634 / sqrt((double)fm::AM_DH));
+    am.part = c->attn_part;
+    am.cnt = c->attn_cnt;
+    for (int q = 0; q < n_seqs; ++q) {
+      am.slot[q] = seq_ids[q];
+      am.len[q] = c->ctx_len[seq_ids[q]];
+      max_len = std::max(max_len, am.len[q]);
+    }
   }
   bool any_sample = false;
   fm::TempArgs ta;
@@ -438,9 +499,14 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
                        fm::EpiStore<T>{qkv, 3 * d}, st, &c->tc.qkv[l]));
       {
         Prof prof(c, FM_PROF_ATTN, st);
-        dim3 grid(n_seqs, g.n_heads, n_noise);
-        FM_KERNEL(c, FM_PROF_ATTN, fm::k_attn_simt<T><<<grid, 128, 0, st>>>(
-                                       qkv, (const T*)c->Kc[l], (const T*)c->Vc[l], o, aa));
+        if (use_mma_attn) {
+          FM_TRY(attn_mma(c, n_noise, am, (const bf16*)qkv, (const bf16*)c->Kc[l],
+                          (const bf16*)c->Vc[l], (bf16*)o, n_seqs, max_len, st));
+        } else {
+          dim3 grid(n_seqs, g.n_heads, n_noise);
+          FM_KERNEL(c, FM_PROF_ATTN, fm::k_attn_simt<T><<<grid, 128, 0, st>>>(
+                                         qkv, (const T*)c->Kc[l], (const T*)c->Vc[l], o, aa));
+        }
       }
       FM_TRY(gemm_w<T>(c, FM_PROF_DIT_GEMM, o, d, (const T*)c->wo[l], M, d, d,
                        fm::EpiResidual{c->x, ml + 2 * d, d}, st, &c->tc.o[l]));

@@ -1,0 +1,331 @@
+// Split-KV attention of the block queries (bf16, head width 128).
+//
+// For each (sequence, head) the N*16 block queries of the sequence's noise
+// drafts attend, without a mask, over [context rows; the draft's own 16
+// block rows] (the drafter's attention; the pages give 16 heads of a
+// 2048-wide DiT -- page "FlashMap并行草拟加速大模型解码", section
+// "一步生成整块，训练时做了什么").  The context rows are shared by every draft of
+// the sequence, so one CTA streams a context slice once for all N drafts.
+//
+// Grid: (sequence*head, n_ctx_splits + 1).  Split s < n_ctx_splits covers a
+// contiguous slice of context rows; the last split covers each draft's own
+// block rows.  Every CTA keeps an online softmax in registers (mma.sync
+// m16n8k16 bf16 -> fp32), merges its four warps in shared memory and writes
+// an unnormalised partial (row max m, row sum l, O).  The last CTA of a
+// (sequence, head) -- arrival counter, no waiting -- merges the partials in
+// split order and writes O / l as bf16.
+#pragma once
+#include "fm_common.cuh"
+
+namespace fm {
+
+constexpr int AM_DH = 128;            // head width
+constexpr int AM_CHUNK = 64;          // context rows per smem stage
+constexpr int AM_LD = AM_DH + 8;      // padded smem row (272 bytes): conflict-free ldmatrix
+constexpr int AM_THREADS = 128;
+
+struct AttnMmaArgs {
+  int n_seqs, n_noise, K, d, n_heads, max_ctx, n_ctx_splits;
+  float scale_log2;    // log2(e) / sqrt(dh)
+  float* part;         // [pairs][n_ctx_splits + 1][N*16][AM_DH + 2]
+  unsigned* cnt;       // [pairs], zero between launches
+  int slot[256];
+  int len[256];
+};
+
+__device__ __forceinline__ void cp_async16(uint32_t saddr, const void* g) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(g) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *(uint32_t*)&v;
+}
+
+// Online-softmax state of one warp: 16 query rows (this thread: rows g, g+8).
+struct AttnState {
+  float o[16][4];
+  float m[2], l[2];
+};
+
+// Scores of one warp's 16 queries (A fragments qa) against `nk` keys at
+// smem rows ks (row-major [key][AM_LD]), then the online update with the
+// matching value rows vs.  NT = number of 8-key tiles (nk <= 8*NT).
+template <int NT>
+__device__ __forceinline__ void attn_block(AttnState& st, const uint32_t (&qa)[8][4],
+                                           const bf16* ks, const bf16* vs, int nk, float sl2) {
+  const int lane = threadIdx.x & 31, t = lane & 3;
+  float s[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < AM_DH / 16; ++kk) {
+#pragma unroll
+    for (int n = 0; n < NT; n += 2) {
+      const int key = n * 8 + (lane & 7) + ((lane >> 4) << 3);
+      const int col = kk * 16 + ((lane >> 3) & 1) * 8;
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4((uint32_t)__cvta_generic_to_shared(ks + key * AM_LD + col), b0, b1, b2, b3);
+      mma_bf16(s[n], qa[kk], b0, b1);
+      mma_bf16(s[n + 1], qa[kk], b2, b3);
+    }
+  }
+  // mask keys beyond nk, scale to log2 units, row maxima over the quad
+  float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+  for (int n = 0; n < NT; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int key = n * 8 + 2 * t + (e & 1);
+      s[n][e] = key < nk ? s[n][e] * sl2 : -INFINITY;
+      mx[e >> 1] = fmaxf(mx[e >> 1], s[n][e]);
+    }
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+    mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+  }
+  float corr[2], mnew[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    mnew[r] = fmaxf(st.m[r], mx[r]);
+    corr[r] = (mnew[r] == -INFINITY) ? 1.f : exp2f(st.m[r] - mnew[r]);
+    st.m[r] = mnew[r];
+    st.l[r] *= corr[r];
+  }
+#pragma unroll
+  for (int n = 0; n < 16; ++n) {
+    st.o[n][0] *= corr[0]; st.o[n][1] *= corr[0];
+    st.o[n][2] *= corr[1]; st.o[n][3] *= corr[1];
+  }
+#pragma unroll
+  for (int n = 0; n < NT; ++n)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float mm = mnew[e >> 1];
+      s[n][e] = (mm == -INFINITY) ? 0.f : exp2f(s[n][e] - mm);
+      st.l[e >> 1] += s[n][e];
+    }
+  // O += P V, 16 keys per k-step
+#pragma unroll
+  for (int kb = 0; kb < NT / 2; ++kb) {
+    uint32_t pa[4];
+    pa[0] = pack_bf16(s[2 * kb][0], s[2 * kb][1]);
+    pa[1] = pack_bf16(s[2 * kb][2], s[2 * kb][3]);
+    pa[2] = pack_bf16(s[2 * kb + 1][0], s[2 * kb + 1][1]);
+    pa[3] = pack_bf16(s[2 * kb + 1][2], s[2 * kb + 1][3]);
+#pragma unroll
+    for (int n = 0; n < 16; n += 2) {
+      const int key = kb * 16 + (lane & 15);
+      const int col = n * 8 + (lane >> 4) * 8;
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t((uint32_t)__cvta_generic_to_shared(vs + key * AM_LD + col), b0, b1, b2, b3);
+      mma_bf16(st.o[n], pa, b0, b1);
+      mma_bf16(st.o[n + 1], pa, b2, b3);
+    }
+  }
+}
+
+// Loads rows [r0, r0+nr) of a [rows][ld] bf16 matrix (dh columns from col0)
+// into smem [nr][AM_LD]; rows past nr up to `pad_to` are zero-filled.
+__device__ __forceinline__ void load_rows(bf16* dst, const bf16* src, size_t ld, int nr, int pad_to) {
+  for (int e = threadIdx.x; e < pad_to * (AM_DH / 8); e += blockDim.x) {
+    const int r = e / (AM_DH / 8), c8 = (e % (AM_DH / 8)) * 8;
+    bf16* dp = dst + r * AM_LD + c8;
+    if (r < nr) cp_async16((uint32_t)__cvta_generic_to_shared(dp), src + (size_t)r * ld + c8);
+    else *(uint4*)dp = make_uint4(0, 0, 0, 0);
+  }
+}
+
+template <int N>
+__global__ void __launch_bounds__(AM_THREADS)
+k_attn_mma(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc, const bf16* __restrict__ Vc,
+           bf16* __restrict__ out, AttnMmaArgs a) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  bf16* sQ = (bf16*)smem_raw;                       // [N*16][AM_LD]
+  bf16* sK = sQ + N * 16 * AM_LD;                   // [2][AM_CHUNK][AM_LD]
+  bf16* sV = sK + 2 * AM_CHUNK * AM_LD;             // [2][AM_CHUNK][AM_LD]
+  __shared__ int s_last;
+  constexpr int WPM = 4 / N;                        // warps sharing one 16-query tile
+  const int pair = blockIdx.x, split = blockIdx.y;
+  const int b = pair / a.n_heads, h = pair - b * a.n_heads;
+  const int d3 = 3 * a.d, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int mt = warp % N, sub = warp / N;          // query tile, key sub-slice
+  const int row0 = b * a.n_noise * a.K;             // first block row of the sequence
+  const int S_all = a.n_ctx_splits + 1;
+  const int NQ = N * 16;
+
+  // queries of all drafts of the sequence
+  load_rows(sQ, qkv + (size_t)row0 * d3 + h * AM_DH, d3, NQ, NQ);
+  cp_commit();
+
+  AttnState st;
+#pragma unroll
+  for (int n = 0; n < 16; ++n) st.o[n][0] = st.o[n][1] = st.o[n][2] = st.o[n][3] = 0.f;
+  st.m[0] = st.m[1] = -INFINITY;
+  st.l[0] = st.l[1] = 0.f;
+
+  uint32_t qa[8][4];
+  auto load_q = [&]() {
+    cp_wait<0>();
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const int r = mt * 16 + (lane & 15), c = kk * 16 + (lane >> 4) * 8;
+      ldsm_x4((uint32_t)__cvta_generic_to_shared(sQ + r * AM_LD + c), qa[kk][0], qa[kk][1],
+              qa[kk][2], qa[kk][3]);
+    }
+  };
+
+  if (split < a.n_ctx_splits) {
+    const int L = a.len[b];
+    const int k0 = (int)((long)split * L / a.n_ctx_splits);
+    const int k1 = (int)((long)(split + 1) * L / a.n_ctx_splits);
+    const size_t base = (size_t)a.slot[b] * a.max_ctx * a.d + h * AM_DH;
+    const int n_chunks = (k1 - k0 + AM_CHUNK - 1) / AM_CHUNK;
+    if (n_chunks > 0) {
+      const int nr = min(AM_CHUNK, k1 - k0);
+      load_rows(sK, Kc + base + (size_t)k0 * a.d, a.d, nr, AM_CHUNK);
+      load_rows(sV, Vc + base + (size_t)k0 * a.d, a.d, nr, AM_CHUNK);
+    }
+    cp_commit();
+    load_q();
+    for (int c = 0; c < n_chunks; ++c) {
+      const int buf = c & 1;
+      if (c + 1 < n_chunks) {
+        const int r0 = k0 + (c + 1) * AM_CHUNK, nr = min(AM_CHUNK, k1 - r0);
+        load_rows(sK + (buf ^ 1) * AM_CHUNK * AM_LD, Kc + base + (size_t)r0 * a.d, a.d, nr, AM_CHUNK);
+        load_rows(sV + (buf ^ 1) * AM_CHUNK * AM_LD, Vc + base + (size_t)r0 * a.d, a.d, nr, AM_CHUNK);
+      }
+      cp_commit();
+      cp_wait<1>();
+      __syncthreads();
+      const int nk_chunk = min(AM_CHUNK, k1 - (k0 + c * AM_CHUNK));
+      constexpr int KW = AM_CHUNK / WPM;            // keys of this warp within the chunk
+      const int kw0 = sub * KW;
+      const int nk = max(0, min(KW, nk_chunk - kw0));
+      const bf16* ks = sK + buf * AM_CHUNK * AM_LD + kw0 * AM_LD;
+      const bf16* vs = sV + buf * AM_CHUNK * AM_LD + kw0 * AM_LD;
+      if (nk > 0) attn_block<KW / 8>(st, qa, ks, vs, nk, a.scale_log2);
+      __syncthreads();
+    }
+  } else {
+    // each draft's own block rows: keys/values of rows row0 + mt*16 .. +16
+    if (sub == 0) {
+      // warps sub==0 (one per draft) load their 16 rows into their own slice
+      bf16* kd = sK + mt * 16 * AM_LD;
+      bf16* vd = sV + mt * 16 * AM_LD;
+      const bf16* kg = qkv + (size_t)(row0 + mt * 16) * d3 + a.d + h * AM_DH;
+      const bf16* vg = kg + a.d;
+      for (int e = lane; e < 16 * (AM_DH / 8); e += 32) {
+        const int r = e / (AM_DH / 8), c8 = (e % (AM_DH / 8)) * 8;
+        cp_async16((uint32_t)__cvta_generic_to_shared(kd + r * AM_LD + c8), kg + (size_t)r * d3 + c8);
+        cp_async16((uint32_t)__cvta_generic_to_shared(vd + r * AM_LD + c8), vg + (size_t)r * d3 + c8);
+      }
+    }
+    cp_commit();
+    load_q();
+    if (sub == 0) attn_block<2>(st, qa, sK + mt * 16 * AM_LD, sV + mt * 16 * AM_LD, 16, a.scale_log2);
+    __syncthreads();
+  }
+
+  // ---- merge the warps of each query tile in smem, write this split's partial
+  float l_tot[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    l_tot[r] = st.l[r];
+    l_tot[r] += __shfl_xor_sync(0xffffffffu, l_tot[r], 1);
+    l_tot[r] += __shfl_xor_sync(0xffffffffu, l_tot[r], 2);
+  }
+  float* sO = (float*)sK;                           // [4 warps][16][AM_DH + 2] fp32 (reuse)
+  const int g = lane >> 2, t = lane & 3;
+  float* wo = sO + warp * 16 * (AM_DH + 2);
+#pragma unroll
+  for (int n = 0; n < 16; ++n) {
+    const int c = n * 8 + 2 * t;
+    wo[g * (AM_DH + 2) + c] = st.o[n][0];
+    wo[g * (AM_DH + 2) + c + 1] = st.o[n][1];
+    wo[(g + 8) * (AM_DH + 2) + c] = st.o[n][2];
+    wo[(g + 8) * (AM_DH + 2) + c + 1] = st.o[n][3];
+  }
+  if (t == 0) {
+    wo[g * (AM_DH + 2) + AM_DH] = st.m[0];
+    wo[g * (AM_DH + 2) + AM_DH + 1] = l_tot[0];
+    wo[(g + 8) * (AM_DH + 2) + AM_DH] = st.m[1];
+    wo[(g + 8) * (AM_DH + 2) + AM_DH + 1] = l_tot[1];
+  }
+  __syncthreads();
+  float* part = a.part + ((size_t)pair * S_all + split) * NQ * (AM_DH + 2);
+  for (int e = threadIdx.x; e < NQ * AM_DH; e += blockDim.x) {
+    const int q = e / AM_DH, c = e % AM_DH;
+    const int tile = q / 16, rr = q % 16;
+    float M = -INFINITY;
+    for (int s2 = 0; s2 < WPM; ++s2) M = fmaxf(M, sO[((s2 * N + tile) * 16 + rr) * (AM_DH + 2) + AM_DH]);
+    float o = 0.f, l = 0.f;
+    for (int s2 = 0; s2 < WPM; ++s2) {
+      const float* w = sO + ((s2 * N + tile) * 16 + rr) * (AM_DH + 2);
+      const float f = (w[AM_DH] == -INFINITY) ? 0.f : exp2f(w[AM_DH] - M);
+      o += f * w[c];
+      l += f * w[AM_DH + 1];
+    }
+    part[q * (AM_DH + 2) + c] = o;
+    if (c == 0) {
+      part[q * (AM_DH + 2) + AM_DH] = M;
+      part[q * (AM_DH + 2) + AM_DH + 1] = l;
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(&a.cnt[pair], 1u) == (unsigned)(S_all - 1));
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // ---- last CTA of this (sequence, head): merge the splits in order
+  const float* pp = a.part + (size_t)pair * S_all * NQ * (AM_DH + 2);
+  for (int e = threadIdx.x; e < NQ * AM_DH; e += blockDim.x) {
+    const int q = e / AM_DH, c = e % AM_DH;
+    float M = -INFINITY;
+    for (int s2 = 0; s2 < S_all; ++s2) M = fmaxf(M, __ldcg(pp + ((size_t)s2 * NQ + q) * (AM_DH + 2) + AM_DH));
+    float o = 0.f, l = 0.f;
+    for (int s2 = 0; s2 < S_all; ++s2) {
+      const float* w = pp + ((size_t)s2 * NQ + q) * (AM_DH + 2);
+      const float ms = __ldcg(w + AM_DH);
+      const float f = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
+      o += f * __ldcg(w + c);
+      l += f * __ldcg(w + AM_DH + 1);
+    }
+    const int j = q / 16, i = q % 16;
+    out[(size_t)(row0 + j * a.K + i) * a.d + h * AM_DH + c] = __float2bfloat16_rn(o / l);
+  }
+  if (threadIdx.x == 0) a.cnt[pair] = 0u;
+}
+
+template <int N>
+constexpr int attn_mma_smem() {
+  return (N * 16 + 4 * AM_CHUNK) * AM_LD * 2;
+}
+
+}  // namespace fm

@@ -237,7 +237,7 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUte
   uint32_t* tmem_slot = (uint32_t*)(tempty + 2);
   volatile int* abort = (volatile int*)(tmem_slot + 1);
   int* s_last = (int*)(tmem_slot + 2);
-  volatile int* s_ok = (volatile int*)(tmem_slot + 3);
+  volatile int* s_ok = (volatile int*)(tmem_slot + 3);  // two slots
   float* red_v = (float*)(base + C::STAGES * C::STAGE + 256);
   int* red_i = (int*)(red_v + 4 * BN);
 
@@ -325,15 +325,19 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUte
     const int et = threadIdx.x - 64;      // 0..127
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int u = blockIdx.x; u < a.units && !*abort; u += gridDim.x) {
+    int it = 0;
+    // the loop condition must not read `abort`: all 128 threads leave together
+    for (int u = blockIdx.x; u < a.units; u += gridDim.x, ++it) {
       const int mt = u % a.m_tiles, rest = u / a.m_tiles;
       const int z = rest % a.splits, nt = rest / a.splits;
       const int n0 = nt * TC_BM, m0 = mt * BN;
       const int tile = nt * a.m_tiles + mt;
-      // one waiter, then a barrier the 128 threads always reach together
-      if (et == 0) *s_ok = mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort) ? 1 : 0;
+      // one waiter, then a barrier the 128 threads always reach together; the
+      // flag alternates between two slots so a late reader never sees the
+      // next unit's value
+      if (et == 0) s_ok[it & 1] = mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort) ? 1 : 0;
       named_sync(1, 128);
-      if (!*s_ok) break;
+      if (!s_ok[it & 1]) break;
       tc_fence_after();
       const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + acc * BN;
       float v[16];

@@ -81,8 +81,9 @@ def assert_tokens_on_margin(got_tokens, want_logits, what=""):
     return int(sure.sum())
 
 
-def sampled_token_sure(logits_row, T, u, frac=0.01):
-    """Oracle token of inverse-CDF sampling and whether u sits well inside its cell."""
+def sampled_token_sure(logits_row, T, u, frac=1e-6):
+    """Oracle token of inverse-CDF sampling and whether u*total sits more than
+    frac*total inside its CDF cell."""
     z = np.asarray(logits_row, dtype=np.float64)
     wts = np.exp((z - z.max()) / T)
     c = np.cumsum(wts)
@@ -92,6 +93,19 @@ def sampled_token_sure(logits_row, T, u, frac=0.01):
     hi = c[y]
     t = u * tot
     return y, (t - lo) > frac * tot and (hi - t) > frac * tot
+
+
+def sampled_token_near(logits_row, T, u, token, tol=2e-4):
+    """True when the oracle's CDF cell of `token` lies within tol*total of u*total:
+    a draw from logits that differ from the oracle's by the bf16 tolerance."""
+    z = np.asarray(logits_row, dtype=np.float64)
+    wts = np.exp((z - z.max()) / T)
+    c = np.cumsum(wts)
+    tot = c[-1]
+    lo = c[token - 1] if token > 0 else 0.0
+    hi = c[token]
+    t = u * tot
+    return lo - tol * tot <= t <= hi + tol * tot
 
 
 def to_np(t: torch.Tensor) -> np.ndarray:
