@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(fs.WORKLOADS))
     ap.add_argument("--rounds", type=int, default=0, help="distinct seeded rounds cycled (0: auto)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of CUDA graphs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     return ap.parse_args()
@@ -203,24 +204,24 @@ def run_fm(args, w, rank, world, local_rank):
         del lg
         rd["target"] = to_device(tgt)
         rounds.append(rd)
-    n_acc_all = torch.zeros((args.steps + args.warmup, B), dtype=torch.int32, device="cuda")
+    n_acc_round = torch.zeros((R, B), dtype=torch.int32, device="cuda")
     branch = torch.empty(B, dtype=torch.int32, device="cuda")
     out_tok = torch.empty((B, K + 1), dtype=torch.int32, device="cuda")
     g, h0 = len(greedy), len(greedy)
 
-    def step(rd, k, n_acc):
+    def step(rd, n_acc, st):
         if w.new_rows:
-            fmb.fm_project_context(ctx.ctx, seqs, rd["hidden"], w.new_rows, [w.ctx] * B, stream)
+            fmb.fm_project_context(ctx.ctx, seqs, rd["hidden"], w.new_rows, [w.ctx] * B, st)
         fmb.fm_draft(ctx.ctx, seqs, rd["noise"], N, w.t_grid, w.temps, rd["u_draft"], tokens, dlog,
-                     stream)
+                     st)
         tgt = rd["target"]
         if g:
-            fmb.fm_verify_greedy(ctx.ctx, tgt, tokens, g, N, K, V, n_acc, branch, out_tok, stream)
+            fmb.fm_verify_greedy(ctx.ctx, tgt, tokens, g, N, K, V, n_acc, branch, out_tok, st)
         if sampled:
             ns = B - g
             fmb.fm_verify_sample(ctx.ctx, tgt[h0:], dlog[h0:], tokens[h0:], ns, N, K, V,
                                  w.temps[h0], rd["u_accept"][h0:], rd["u_res"][h0:],
-                                 n_acc[h0:], branch[h0:], out_tok[h0:], stream)
+                                 n_acc[h0:], branch[h0:], out_tok[h0:], st)
 
     def barrier():
         torch.cuda.synchronize()
@@ -237,25 +238,49 @@ def run_fm(args, w, rank, world, local_rank):
     setup_s = time.time() - t_setup
     log(f"{R} rounds prepared in {setup_s:.1f} s; timing")
     for k in range(args.warmup):
-        step(rounds[k % R], k, n_acc_all[k])
+        step(rounds[k % R], n_acc_round[k % R], stream)
     ab = algorithmic_bytes(w)
     prof_classes = ["embed", "lm_head"]
     mask = sum(1 << fmb.FM_PROF[c] for c in prof_classes)
     barrier()
+    # one CUDA graph per distinct round; the dominant kernels carry CUDA-event
+    # pairs inside the graphs, so their timings come from the timed replays
     fmb.fm_profile(ctx.ctx, mask)
     fmb.fm_profile_read(ctx.ctx, reset=True)
+    graphs = []
+    if not args.no_graph:
+        for i in range(R):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr):
+                step(rounds[i], n_acc_round[i], torch.cuda.current_stream())
+            graphs.append(gr)
+        _, cap_launches = fmb.fm_profile_read(ctx.ctx)
+        launches_per_step = sum(cap_launches) / R
+        for gr in graphs:          # one untimed replay each
+            gr.replay()
+        barrier()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local_rank) as clk:
         ev0.record(stream)
         for k in range(args.steps):
-            step(rounds[(args.warmup + k) % R], k, n_acc_all[args.warmup + k])
+            i = (args.warmup + k) % R
+            if graphs:
+                graphs[i].replay()
+            else:
+                step(rounds[i], n_acc_round[i], stream)
         ev1.record(stream)
         torch.cuda.synchronize()
     prof_ms, launches = fmb.fm_profile_read(ctx.ctx, reset=True)
     fmb.fm_profile(ctx.ctx, 0)
+    if not graphs:
+        launches_per_step = sum(launches) / args.steps
+        timed_steps = args.steps
+    else:
+        timed_steps = R   # each graph's event pairs hold its last replay
     barrier()
     ms = max_over_ranks(ev0.elapsed_time(ev1))
-    n_sum = int(n_acc_all[args.warmup:].sum().item())
+    n_round = n_acc_round.sum(dim=1).cpu().numpy()
+    n_sum = int(sum(n_round[(args.warmup + k) % R] for k in range(args.steps)))
     verified = n_sum + args.steps * B           # accepted + one target token per sequence
     if dist is not None:
         t = torch.tensor([float(verified)], dtype=torch.float64, device="cuda")
@@ -274,11 +299,11 @@ def run_fm(args, w, rank, world, local_rank):
     for c in prof_classes:
         i = fmb.FM_PROF[c]
         n_launch = launches[i]
-        if prof_ms[i] > 0 and n_launch > 0:
-            avg = prof_ms[i] / (args.steps * (len(w.t_grid) - 1))
+        if prof_ms[i] > 0:
+            avg = prof_ms[i] / (timed_steps * (len(w.t_grid) - 1))
             per_class[c] = {"ms_per_launch": avg, "bytes_per_launch": ab[f"{c}_per_launch"],
                             "gbs": ab[f"{c}_per_launch"] / (avg / 1e3) / 1e9,
-                            "share_of_step": prof_ms[i] / ms}
+                            "share_of_step": prof_ms[i] / timed_steps / (ms / args.steps)}
     dom = max(per_class, key=lambda c: per_class[c]["share_of_step"]) if per_class else None
     roof = None
     if dom:
@@ -302,7 +327,8 @@ def run_fm(args, w, rank, world, local_rank):
         "step_hbm_gbs": round(step_bytes / (ms / args.steps / 1e3) / 1e9, 1),
         "step_hbm_frac": round(step_bytes / (ms / args.steps / 1e3) / 1e9 / pk["hbm_gbs"], 4),
         "roofline": roof, "kernels": per_class,
-        "gpu_launches": int(sum(launches)),
+        "gpu_launches": int(round(launches_per_step * args.steps)),
+        "cuda_graphs": bool(graphs),
         "clocks": clk.summary(), "setup_s": round(setup_s, 1),
     }
 
@@ -315,10 +341,19 @@ def run_fm(args, w, rank, world, local_rank):
             rd = rounds[i]
             pin.append({k: (v.cpu().pin_memory() if v is not None else None) for k, v in rd.items()})
         dev_in = {k: (torch.empty_like(v) if v is not None else None) for k, v in rounds[0].items()}
+        n_stage = torch.zeros(B, dtype=torch.int32, device="cuda")
         host_n = torch.empty((args.steps, B), dtype=torch.int32).pin_memory()
         host_tok = torch.empty((args.steps, B, K + 1), dtype=torch.int32).pin_memory()
         h2d = sum(v.numel() * v.element_size() for v in pin[0].values() if v is not None)
         d2h = B * 4 + B * (K + 1) * 4
+        gstage = None
+        if graphs:
+            for key, v in pin[0].items():
+                if v is not None:
+                    dev_in[key].copy_(v)
+            gstage = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gstage):
+                step(dev_in, n_stage, torch.cuda.current_stream())
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
@@ -327,8 +362,11 @@ def run_fm(args, w, rank, world, local_rank):
             for key, v in src.items():
                 if v is not None:
                     dev_in[key].copy_(v, non_blocking=True)
-            step(dev_in, k, n_acc_all[args.warmup + k])
-            host_n[k].copy_(n_acc_all[args.warmup + k], non_blocking=True)
+            if gstage is not None:
+                gstage.replay()
+            else:
+                step(dev_in, n_stage, stream)
+            host_n[k].copy_(n_stage, non_blocking=True)
             host_tok[k].copy_(out_tok, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()

@@ -312,7 +312,7 @@ fm_status load_impl(fm_ctx* c, cudaStream_t st) {
   FM_TRY(dalloc_t(c, &c->tile_cnt, c->tile_cnt_n));
   FM_CUDA(cudaMemsetAsync(c->tile_cnt, 0, c->tile_cnt_n * sizeof(unsigned), st));
   c->attn_pairs_max = call_seqs * g.n_heads;
-  c->attn_part_elems = (size_t)(2 * c->sms + 2 * c->attn_pairs_max) * g.max_noise * 16 * (fm::AM_DH + 2);
+  c->attn_part_elems = (size_t)(2 * c->sms + 2 * c->attn_pairs_max) * g.max_noise * 16 * fm::AM_PSTRIDE;
   FM_TRY(dalloc_t(c, &c->attn_part, c->attn_part_elems));
   FM_TRY(dalloc_t(c, &c->attn_cnt, (size_t)c->attn_pairs_max));
   FM_CUDA(cudaMemsetAsync(c->attn_cnt, 0, c->attn_pairs_max * sizeof(unsigned), st));
@@ -388,7 +388,7 @@ template <int N>
 fm_status attn_mma_launch(fm_ctx* c, const fm::AttnMmaArgs& am, dim3 grid, const bf16* qkv,
                           const bf16* Kc, const bf16* Vc, bf16* o, cudaStream_t st) {
   constexpr int smem = fm::attn_mma_smem<N>();
-  FM_CUDA(cudaFuncSetAttribute(fm::k_attn_mma<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  FM_CUDA(fm::set_smem_once(fm::k_attn_mma<N>, smem));
   FM_KERNEL(c, FM_PROF_ATTN, fm::k_attn_mma<N><<<grid, fm::AM_THREADS, smem, st>>>(qkv, Kc, Vc, o, am));
   return FM_OK;
 }
@@ -402,7 +402,7 @@ fm_status attn_mma(fm_ctx* c, int n_noise, fm::AttnMmaArgs am, const bf16* qkv, 
   s_ctx = std::min(s_ctx, (max_len + fm::AM_CHUNK - 1) / fm::AM_CHUNK);
   s_ctx = std::max(s_ctx, 1);
   while (s_ctx > 1 &&
-         (size_t)pairs * (s_ctx + 1) * n_noise * 16 * (fm::AM_DH + 2) > c->attn_part_elems)
+         (size_t)pairs * (s_ctx + 1) * n_noise * 16 * fm::AM_PSTRIDE > c->attn_part_elems)
     --s_ctx;
   am.n_ctx_splits = s_ctx;
   dim3 grid(pairs, s_ctx + 1);

@@ -23,11 +23,12 @@ constexpr int AM_DH = 128;            // head width
 constexpr int AM_CHUNK = 64;          // context rows per smem stage
 constexpr int AM_LD = AM_DH + 8;      // padded smem row (272 bytes): conflict-free ldmatrix
 constexpr int AM_THREADS = 128;
+constexpr int AM_PSTRIDE = AM_DH + 4;  // floats per partial row: O[128], m, l, pad (16-byte rows)
 
 struct AttnMmaArgs {
   int n_seqs, n_noise, K, d, n_heads, max_ctx, n_ctx_splits;
   float scale_log2;    // log2(e) / sqrt(dh)
-  float* part;         // [pairs][n_ctx_splits + 1][N*16][AM_DH + 2]
+  float* part;         // [pairs][n_ctx_splits + 1][N*16][AM_PSTRIDE]
   unsigned* cnt;       // [pairs], zero between launches
   int slot[256];
   int len[256];
@@ -278,7 +279,7 @@ k_attn_mma(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc, const bf16
     wo[(g + 8) * (AM_DH + 2) + AM_DH + 1] = l_tot[1];
   }
   __syncthreads();
-  float* part = a.part + ((size_t)pair * S_all + split) * NQ * (AM_DH + 2);
+  float* part = a.part + ((size_t)pair * S_all + split) * NQ * AM_PSTRIDE;
   for (int e = threadIdx.x; e < NQ * AM_DH; e += blockDim.x) {
     const int q = e / AM_DH, c = e % AM_DH;
     const int tile = q / 16, rr = q % 16;
@@ -291,10 +292,10 @@ k_attn_mma(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc, const bf16
       o += f * w[c];
       l += f * w[AM_DH + 1];
     }
-    part[q * (AM_DH + 2) + c] = o;
+    part[q * AM_PSTRIDE + c] = o;
     if (c == 0) {
-      part[q * (AM_DH + 2) + AM_DH] = M;
-      part[q * (AM_DH + 2) + AM_DH + 1] = l;
+      part[q * AM_PSTRIDE + AM_DH] = M;
+      part[q * AM_PSTRIDE + AM_DH + 1] = l;
     }
   }
   __threadfence();
@@ -303,22 +304,35 @@ k_attn_mma(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc, const bf16
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // ---- last CTA of this (sequence, head): merge the splits in order
-  const float* pp = a.part + (size_t)pair * S_all * NQ * (AM_DH + 2);
-  for (int e = threadIdx.x; e < NQ * AM_DH; e += blockDim.x) {
-    const int q = e / AM_DH, c = e % AM_DH;
-    float M = -INFINITY;
-    for (int s2 = 0; s2 < S_all; ++s2) M = fmaxf(M, __ldcg(pp + ((size_t)s2 * NQ + q) * (AM_DH + 2) + AM_DH));
-    float o = 0.f, l = 0.f;
+  // ---- last CTA of this (sequence, head): merge the splits in split order,
+  // one warp per query row, four columns per lane, loads of several splits
+  // in flight
+  const float* pp = a.part + (size_t)pair * S_all * NQ * AM_PSTRIDE;
+  for (int q = warp; q < NQ; q += AM_THREADS / 32) {
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    float l = 0.f, M = -INFINITY;
+#pragma unroll 4
     for (int s2 = 0; s2 < S_all; ++s2) {
-      const float* w = pp + ((size_t)s2 * NQ + q) * (AM_DH + 2);
-      const float ms = __ldcg(w + AM_DH);
-      const float f = (ms == -INFINITY) ? 0.f : exp2f(ms - M);
-      o += f * __ldcg(w + c);
-      l += f * __ldcg(w + AM_DH + 1);
+      const float* w = pp + ((size_t)s2 * NQ + q) * AM_PSTRIDE;
+      const float2 ml = __ldcg((const float2*)(w + AM_DH));
+      const float4 os = __ldcg((const float4*)(w + 4 * lane));
+      if (ml.x == -INFINITY) continue;
+      if (ml.x > M) {
+        const float f = (M == -INFINITY) ? 0.f : exp2f(M - ml.x);
+        o.x *= f; o.y *= f; o.z *= f; o.w *= f;
+        l *= f;
+        M = ml.x;
+      }
+      const float f = exp2f(ml.x - M);
+      o.x += f * os.x; o.y += f * os.y; o.z += f * os.z; o.w += f * os.w;
+      l += f * ml.y;
     }
+    const float inv = 1.f / l;
     const int j = q / 16, i = q % 16;
-    out[(size_t)(row0 + j * a.K + i) * a.d + h * AM_DH + c] = __float2bfloat16_rn(o / l);
+    __nv_bfloat162* dst =
+        (__nv_bfloat162*)(out + (size_t)(row0 + j * a.K + i) * a.d + h * AM_DH + 4 * lane);
+    dst[0] = __floats2bfloat162_rn(o.x * inv, o.y * inv);
+    dst[1] = __floats2bfloat162_rn(o.z * inv, o.w * inv);
   }
   if (threadIdx.x == 0) a.cnt[pair] = 0u;
 }

@@ -5,6 +5,9 @@
 #include <stdint.h>
 #include <math.h>
 
+#include <mutex>
+#include <unordered_map>
+
 namespace fm {
 
 typedef __nv_bfloat16 bf16;
@@ -92,6 +95,27 @@ __device__ __forceinline__ ArgMax block_argmax(ArgMax a, float* shv, int* shi) {
   if (lane < nw) { a.v = shv[lane]; a.i = shi[lane]; } else { a.v = -INFINITY; a.i = 0x7fffffff; }
   a = warp_argmax(a);
   return a;
+}
+
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device):
+// the call is host-side only and would otherwise cost host time per launch.
+inline cudaError_t set_smem_once_ptr(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::unordered_map<const void*, unsigned long long> done;  // bit per device id < 64
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = 1ull << (dev & 63);
+  std::lock_guard<std::mutex> lock(mu);
+  unsigned long long& m = done[kernel];
+  if (m & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) m |= bit;
+  return e;
+}
+template <typename F>
+inline cudaError_t set_smem_once(F* kernel, int bytes) {
+  return set_smem_once_ptr((const void*)kernel, bytes);
 }
 
 __device__ __forceinline__ float gelu_tanh(float u) {

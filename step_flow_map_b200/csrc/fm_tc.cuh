@@ -368,16 +368,28 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUte
         const int last = *s_last;
         if (last) {
           __threadfence();
+          const size_t zstride = (size_t)tiles * TC_BM * BN;
+          const float* p0 = a.partial + ((size_t)tile * TC_BM + r) * BN;
           for (int j0 = 0; j0 < BN; j0 += 16) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] = 0.f;
-            for (int zz = 0; zz < a.splits; ++zz) {
-              const float* p = a.partial + (((size_t)zz * tiles + tile) * TC_BM + r) * BN + j0;
+            // four splits' loads in flight at a time; sums stay in split order
+            for (int zz = 0; zz < a.splits; zz += 4) {
+              float4 t[4][4];
 #pragma unroll
-              for (int j = 0; j < 16; j += 4) {
-                float4 t = __ldcg((const float4*)(p + j));
-                v[j] += t.x; v[j + 1] += t.y; v[j + 2] += t.z; v[j + 3] += t.w;
-              }
+              for (int u2 = 0; u2 < 4; ++u2)
+                if (zz + u2 < a.splits)
+#pragma unroll
+                  for (int j = 0; j < 4; ++j)
+                    t[u2][j] = __ldcg((const float4*)(p0 + (zz + u2) * zstride + j0 + 4 * j));
+#pragma unroll
+              for (int u2 = 0; u2 < 4; ++u2)
+                if (zz + u2 < a.splits)
+#pragma unroll
+                  for (int j = 0; j < 4; ++j) {
+                    v[4 * j] += t[u2][j].x; v[4 * j + 1] += t[u2][j].y;
+                    v[4 * j + 2] += t[u2][j].z; v[4 * j + 3] += t[u2][j].w;
+                  }
             }
             tc_finish_chunk<BN>(epi, a, n0, m0, r, j0, v, red_v, red_i, q);
           }
@@ -539,8 +551,7 @@ fm_status tc_launch(const TcMap& wm, const bf16* A, int lda, int M, Epi epi, flo
   CUtensorMap mapA;
   if (!tc_encode(&mapA, A, wm.Kd, M, lda, BN, err, errlen)) return FM_ERR_CUDA;
   {
-    cudaError_t e = cudaFuncSetAttribute(k_tc_gemm<BN, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM);
+    cudaError_t e = set_smem_once(k_tc_gemm<BN, Epi>, C::SMEM);
     if (e != cudaSuccess) {
       snprintf(err, errlen, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
       return FM_ERR_CUDA;
