@@ -50,6 +50,7 @@ def parse():
     ap.add_argument("--rounds", type=int, default=0, help="distinct seeded rounds cycled (0: auto)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of CUDA graphs")
+    ap.add_argument("--profile-all", action="store_true", help="log per-class kernel times")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     return ap.parse_args()
@@ -239,6 +240,19 @@ def run_fm(args, w, rank, world, local_rank):
     log(f"{R} rounds prepared in {setup_s:.1f} s; timing")
     for k in range(args.warmup):
         step(rounds[k % R], n_acc_round[k % R], stream)
+    if args.profile_all:
+        # diagnostic: every kernel class timed with events, eager launches
+        # (the event pairs serialise neighbouring kernels)
+        fmb.fm_profile(ctx.ctx, (1 << fmb.FM_PROF_N) - 1)
+        fmb.fm_profile_read(ctx.ctx, reset=True)
+        for k in range(20):
+            step(rounds[k % R], n_acc_round[k % R], stream)
+        torch.cuda.synchronize()
+        pm, pl = fmb.fm_profile_read(ctx.ctx, reset=True)
+        fmb.fm_profile(ctx.ctx, 0)
+        for name, i in sorted(fmb.FM_PROF.items(), key=lambda x: x[1]):
+            if pl[i]:
+                log(f"profile {name:9s}: {pm[i] / 20 * 1e3:8.1f} us/step, {pl[i] / 20:.0f} launches/step")
     ab = algorithmic_bytes(w)
     prof_classes = ["embed", "lm_head"]
     mask = sum(1 << fmb.FM_PROF[c] for c in prof_classes)

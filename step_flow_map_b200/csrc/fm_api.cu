@@ -136,19 +136,24 @@ struct Prof {
     if (((c->prof_mask >> cls) & 1) && c->ev_used < c->ev_a.size()) {
       slot = (long)c->ev_used++;
       c->ev_cls[slot] = cls;
-      cudaEventRecord(c->ev_a[slot], st);
+      // "external" records also become real timing records inside a CUDA graph
+      cudaEventRecordWithFlags(c->ev_a[slot], st, cudaEventRecordExternal);
     }
   }
   ~Prof() {
-    if (slot >= 0) cudaEventRecord(c->ev_b[slot], st);
+    if (slot >= 0) cudaEventRecordWithFlags(c->ev_b[slot], st, cudaEventRecordExternal);
   }
 };
 
-#define FM_KERNEL(c, cls, ...)   \
-  do {                           \
-    __VA_ARGS__;                 \
-    (c)->launches[cls]++;        \
-    FM_LAUNCHED();               \
+// Every kernel goes out with programmatic stream serialization (see
+// fm::pdl_wait): it may start while its predecessor drains.
+#define FM_LAUNCH(c, cls, kernel, grid, block, smem, st, ...)                               \
+  do {                                                                                   \
+    cudaError_t e_ = fm::launch_pdl(kernel, dim3(grid), dim3(block), smem, st, __VA_ARGS__); \
+    (c)->launches[cls]++;                                                                \
+    if (e_ != cudaSuccess)                                                               \
+      return set_err(FM_ERR_CUDA, "launch of %s failed: %s (%s:%d)", #kernel,            \
+                     cudaGetErrorString(e_), __FILE__, __LINE__);                        \
   } while (0)
 
 int grid_1d(size_t n, int threads, int cap = 148 * 16) {
@@ -181,14 +186,14 @@ fm_status gemm_simt(fm_ctx* c, int cls, const TA* A, int lda, const TW* W, int l
   }
   grid.z = splits;
   if (wk)
-    FM_KERNEL(c, cls, fm::k_gemm_simt<TA, TW, true, Epi><<<grid, 256, 0, st>>>(
-                          A, lda, W, ldw, M, N, Kd, k_split, c->splitk, epi));
+    FM_LAUNCH(c, cls, (fm::k_gemm_simt<TA, TW, true, Epi>), grid, 256, 0, st,
+              A, lda, W, ldw, M, N, Kd, k_split, c->splitk, epi);
   else
-    FM_KERNEL(c, cls, fm::k_gemm_simt<TA, TW, false, Epi><<<grid, 256, 0, st>>>(
-                          A, lda, W, ldw, M, N, Kd, k_split, c->splitk, epi));
+    FM_LAUNCH(c, cls, (fm::k_gemm_simt<TA, TW, false, Epi>), grid, 256, 0, st,
+              A, lda, W, ldw, M, N, Kd, k_split, c->splitk, epi);
   if (splits > 1)
-    FM_KERNEL(c, cls, fm::k_splitk_apply<Epi><<<grid_1d((size_t)M * N, 256), 256, 0, st>>>(
-                          c->splitk, splits, M, N, epi));
+    FM_LAUNCH(c, cls, (fm::k_splitk_apply<Epi>), grid_1d((size_t)M * N, 256), 256, 0, st,
+              c->splitk, splits, M, N, epi);
   return FM_OK;
 }
 
@@ -219,16 +224,18 @@ fm_status compute_mods(fm_ctx* c, float s, float t, float* out, cudaStream_t st)
   auto gemv = [&](const void* W, int n_out, int n_in, const float* x, float* y, const float* add,
                   int act) -> fm_status {
     int threads = 256, blocks = (n_out * 32 + threads - 1) / threads;
-    FM_KERNEL(c, FM_PROF_OTHER,
-              fm::k_gemv<T><<<blocks, threads, 0, st>>>((const T*)W, n_out, n_in, x, y, add, act));
+    FM_LAUNCH(c, FM_PROF_OTHER, (fm::k_gemv<T>), blocks, threads, 0, st,
+              (const T*)W, n_out, n_in, x, y, add, act);
     return FM_OK;
   };
-  FM_KERNEL(c, FM_PROF_OTHER, fm::k_time_features<<<1, 256, 0, st>>>((double)s, (double)t, c->phi));
+  FM_LAUNCH(c, FM_PROF_OTHER, (fm::k_time_features), 1, 256, 0, st,
+              (double)s, (double)t, c->phi);
   FM_TRY(gemv(c->w.W_ts1, d, 256, c->phi, tv, nullptr, 1));                // SiLU(W1 phi(s))
   FM_TRY(gemv(c->w.W_ts2, d, d, tv, tv + d, nullptr, 0));                 // TE_s(s)
   FM_TRY(gemv(c->w.W_tt1, d, 256, c->phi + 256, tv + 2 * d, nullptr, 1)); // SiLU(W1 phi(t))
   FM_TRY(gemv(c->w.W_tt2, d, d, tv + 2 * d, tv + 3 * d, tv + d, 0));      // c = TE_s + TE_t
-  FM_KERNEL(c, FM_PROF_OTHER, fm::k_silu_vec<<<(d + 255) / 256, 256, 0, st>>>(tv + 3 * d, tv + 4 * d, d));
+  FM_LAUNCH(c, FM_PROF_OTHER, (fm::k_silu_vec), (d + 255) / 256, 256, 0, st,
+              tv + 3 * d, tv + 4 * d, d);
   for (int l = 0; l < nb; ++l)
     FM_TRY(gemv(c->wada[l], 6 * d, d, tv + 4 * d, out + (size_t)l * 6 * d, nullptr, 0));
   FM_TRY(gemv(c->w.W_ada_f, 2 * d, d, tv + 4 * d, out + (size_t)nb * 6 * d, nullptr, 0));
@@ -266,7 +273,8 @@ fm_status load_impl(fm_ctx* c, cudaStream_t st) {
   FM_TRY(dalloc(c, &c->Et, (size_t)g.V * d * sizeof(T)));
   {
     dim3 grid((d + 31) / 32, (g.V + 31) / 32), block(32, 8);
-    FM_KERNEL(c, FM_PROF_OTHER, fm::k_transpose<T><<<grid, block, 0, st>>>((const T*)c->w.E, (T*)c->Et, g.V, d));
+    FM_LAUNCH(c, FM_PROF_OTHER, (fm::k_transpose<T>), grid, block, 0, st,
+              (const T*)c->w.E, (T*)c->Et, g.V, d);
   }
   c->Kc.resize(g.n_blocks);
   c->Vc.resize(g.n_blocks);
@@ -360,8 +368,8 @@ fm_status project_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void
                    fm::EpiStoreF32{c->c_raw, d}, st, &c->tc.fc));
   {
     Prof prof(c, FM_PROF_CONTEXT, st);
-    FM_KERNEL(c, FM_PROF_CONTEXT, fm::k_adaln<float, T><<<R, 256, 0, st>>>(
-                                      c->c_raw, d, nullptr, nullptr, (T*)c->c_norm));
+    FM_LAUNCH(c, FM_PROF_CONTEXT, (fm::k_adaln<float, T>), R, 256, 0, st,
+              c->c_raw, d, nullptr, nullptr, (T*)c->c_norm);
   }
   fm::EpiCtxKV<T> epi;
   epi.d = d;
@@ -389,7 +397,8 @@ fm_status attn_mma_launch(fm_ctx* c, const fm::AttnMmaArgs& am, dim3 grid, const
                           const bf16* Kc, const bf16* Vc, bf16* o, cudaStream_t st) {
   constexpr int smem = fm::attn_mma_smem<N>();
   FM_CUDA(fm::set_smem_once(fm::k_attn_mma<N>, smem));
-  FM_KERNEL(c, FM_PROF_ATTN, fm::k_attn_mma<N><<<grid, fm::AM_THREADS, smem, st>>>(qkv, Kc, Vc, o, am));
+  FM_LAUNCH(c, FM_PROF_ATTN, (fm::k_attn_mma<N>), grid, fm::AM_THREADS, smem, st,
+              qkv, Kc, Vc, o, am);
   return FM_OK;
 }
 
@@ -398,8 +407,10 @@ fm_status attn_mma_launch(fm_ctx* c, const fm::AttnMmaArgs& am, dim3 grid, const
 fm_status attn_mma(fm_ctx* c, int n_noise, fm::AttnMmaArgs am, const bf16* qkv, const bf16* Kc,
                    const bf16* Vc, bf16* o, int n_seqs, int max_len, cudaStream_t st) {
   const int pairs = n_seqs * am.n_heads;
+  // at most about two CTAs per SM, and at least four 64-row chunks per split:
+  // every extra split adds a partial to the final merge
   int s_ctx = (2 * c->sms + pairs - 1) / pairs - 1;
-  s_ctx = std::min(s_ctx, (max_len + fm::AM_CHUNK - 1) / fm::AM_CHUNK);
+  s_ctx = std::min(s_ctx, (max_len + 4 * fm::AM_CHUNK - 1) / (4 * fm::AM_CHUNK));
   s_ctx = std::max(s_ctx, 1);
   while (s_ctx > 1 &&
          (size_t)pairs * (s_ctx + 1) * n_noise * 16 * fm::AM_PSTRIDE > c->attn_part_elems)
@@ -493,7 +504,8 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
       const float* ml = mods + (size_t)l * 6 * d;
       {
         Prof prof(c, FM_PROF_NORM, st);
-        FM_KERNEL(c, FM_PROF_NORM, fm::k_adaln<float, T><<<M, 256, 0, st>>>(c->x, d, ml, ml + d, h));
+        FM_LAUNCH(c, FM_PROF_NORM, (fm::k_adaln<float, T>), M, 256, 0, st,
+              c->x, d, ml, ml + d, h);
       }
       FM_TRY(gemm_w<T>(c, FM_PROF_DIT_GEMM, h, d, (const T*)c->wqkv[l], M, 3 * d, d,
                        fm::EpiStore<T>{qkv, 3 * d}, st, &c->tc.qkv[l]));
@@ -504,16 +516,17 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
                           (const bf16*)c->Vc[l], (bf16*)o, n_seqs, max_len, st));
         } else {
           dim3 grid(n_seqs, g.n_heads, n_noise);
-          FM_KERNEL(c, FM_PROF_ATTN, fm::k_attn_simt<T><<<grid, 128, 0, st>>>(
-                                         qkv, (const T*)c->Kc[l], (const T*)c->Vc[l], o, aa));
+          FM_LAUNCH(c, FM_PROF_ATTN, (fm::k_attn_simt<T>), grid, 128, 0, st,
+              qkv, (const T*)c->Kc[l], (const T*)c->Vc[l], o, aa);
         }
       }
       FM_TRY(gemm_w<T>(c, FM_PROF_DIT_GEMM, o, d, (const T*)c->wo[l], M, d, d,
                        fm::EpiResidual{c->x, ml + 2 * d, d}, st, &c->tc.o[l]));
       {
         Prof prof(c, FM_PROF_NORM, st);
-        FM_KERNEL(c, FM_PROF_NORM, fm::k_adaln<float, T><<<M, 256, 0, st>>>(c->x, d, ml + 3 * d,
-                                                                            ml + 4 * d, h));
+        FM_LAUNCH(c, FM_PROF_NORM, (fm::k_adaln<float, T>), M, 256, 0, st,
+              c->x, d, ml + 3 * d,
+                                                                            ml + 4 * d, h);
       }
       FM_TRY(gemm_w<T>(c, FM_PROF_DIT_GEMM, h, d, (const T*)c->wup[l], M, F, d,
                        fm::EpiGelu<T>{u, F}, st, &c->tc.up[l]));
@@ -523,7 +536,8 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
     const float* mf = mods + (size_t)nb * 6 * d;
     {
       Prof prof(c, FM_PROF_NORM, st);
-      FM_KERNEL(c, FM_PROF_NORM, fm::k_adaln<float, T><<<M, 256, 0, st>>>(c->x, d, mf, mf + d, h));
+      FM_LAUNCH(c, FM_PROF_NORM, (fm::k_adaln<float, T>), M, 256, 0, st,
+              c->x, d, mf, mf + d, h);
     }
     // LM head: greedy-only final steps keep the logits on chip when possible
     const bool need_logits = !last || any_sample || draft_logits != nullptr;
@@ -541,12 +555,12 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
     }
     Prof prof(c, FM_PROF_NORM, st);
     if (!last) {
-      FM_KERNEL(c, FM_PROF_NORM, fm::k_softmax_rows<T><<<M, 1024, 0, st>>>(logits, V, (T*)c->D));
+      FM_LAUNCH(c, FM_PROF_NORM, (fm::k_softmax_rows<T>), M, 1024, 0, st,
+              logits, V, (T*)c->D);
     } else {
-      FM_KERNEL(c, FM_PROF_NORM,
-                fm::k_select_tokens<<<M, 1024, 0, st>>>(
-                    have_partials ? nullptr : logits, V, have_partials ? c->part_v : nullptr,
-                    have_partials ? c->part_i : nullptr, c->n_part, u_draft, ta, tokens));
+      FM_LAUNCH(c, FM_PROF_NORM, (fm::k_select_tokens), M, 1024, 0, st,
+              have_partials ? nullptr : logits, V, have_partials ? c->part_v : nullptr,
+                    have_partials ? c->part_i : nullptr, c->n_part, u_draft, ta, tokens);
     }
   }
   return FM_OK;
@@ -702,9 +716,9 @@ extern "C" fm_status fm_verify_greedy(fm_ctx* c, const float* target_logits, con
   const long rows = (long)B * N * (K + 1);
   const int ch = verify_chunks(c, rows, V);
   Prof prof(c, FM_PROF_VERIFY, st);
-  FM_KERNEL(c, FM_PROF_VERIFY, fm::k_verify_greedy<<<(unsigned)(rows * ch), fm::VG_THREADS, 0, st>>>(
-      target_logits, draft, B, N, K, V, ch, c->vg_pv, c->vg_pi, c->vg_cnt, n_acc, branch,
-      out_tokens));
+  FM_LAUNCH(c, FM_PROF_VERIFY, (fm::k_verify_greedy), (unsigned)(rows * ch), fm::VG_THREADS, 0, st,
+              target_logits, draft, B, N, K, V, ch, c->vg_pv, c->vg_pi, c->vg_cnt, n_acc, branch,
+      out_tokens);
   return FM_OK;
 }
 
@@ -721,11 +735,11 @@ extern "C" fm_status fm_verify_sample(fm_ctx* c, const float* target_logits,
   const int n_rows = n_tgt + (draft_logits ? B * N * K : 0);
   const int ch = verify_chunks(c, n_rows, V);
   Prof prof(c, FM_PROF_VERIFY, st);
-  FM_KERNEL(c, FM_PROF_VERIFY, fm::k_row_stats<<<(unsigned)((long)n_rows * ch), fm::VS_THREADS, 0, st>>>(
-      target_logits, draft_logits, n_tgt, n_rows, V, ch, temperature, c->vs_pm, c->vs_ps));
-  FM_KERNEL(c, FM_PROF_VERIFY, fm::k_verify_sample_decide<<<B, fm::VS_DECIDE_THREADS, 0, st>>>(
-      target_logits, draft_logits, draft, B, N, K, V, temperature, u_accept, u_res, c->vs_pm,
-      c->vs_ps, ch, c->vs_resid, n_acc, branch, out_tokens));
+  FM_LAUNCH(c, FM_PROF_VERIFY, (fm::k_row_stats), (unsigned)((long)n_rows * ch), fm::VS_THREADS, 0, st,
+              target_logits, draft_logits, n_tgt, n_rows, V, ch, temperature, c->vs_pm, c->vs_ps);
+  FM_LAUNCH(c, FM_PROF_VERIFY, (fm::k_verify_sample_decide), B, fm::VS_DECIDE_THREADS, 0, st,
+              target_logits, draft_logits, draft, B, N, K, V, temperature, u_accept, u_res, c->vs_pm,
+      c->vs_ps, ch, c->vs_resid, n_acc, branch, out_tokens);
   return FM_OK;
 }
 

@@ -165,6 +165,8 @@ template <int N>
 __global__ void __launch_bounds__(AM_THREADS)
 k_attn_mma(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc, const bf16* __restrict__ Vc,
            bf16* __restrict__ out, AttnMmaArgs a) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(16) uint8_t smem_raw[];
   bf16* sQ = (bf16*)smem_raw;                       // [N*16][AM_LD]
   bf16* sK = sQ + N * 16 * AM_LD;                   // [2][AM_CHUNK][AM_LD]
@@ -311,21 +313,33 @@ k_attn_mma(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc, const bf16
   for (int q = warp; q < NQ; q += AM_THREADS / 32) {
     float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
     float l = 0.f, M = -INFINITY;
-#pragma unroll 4
-    for (int s2 = 0; s2 < S_all; ++s2) {
-      const float* w = pp + ((size_t)s2 * NQ + q) * AM_PSTRIDE;
-      const float2 ml = __ldcg((const float2*)(w + AM_DH));
-      const float4 os = __ldcg((const float4*)(w + 4 * lane));
-      if (ml.x == -INFINITY) continue;
-      if (ml.x > M) {
-        const float f = (M == -INFINITY) ? 0.f : exp2f(M - ml.x);
-        o.x *= f; o.y *= f; o.z *= f; o.w *= f;
-        l *= f;
-        M = ml.x;
+    for (int s0 = 0; s0 < S_all; s0 += 8) {
+      float2 ml[8];
+      float4 os[8];
+#pragma unroll
+      for (int u2 = 0; u2 < 8; ++u2) {   // all loads of the batch in flight
+        if (s0 + u2 < S_all) {
+          const float* w = pp + ((size_t)(s0 + u2) * NQ + q) * AM_PSTRIDE;
+          ml[u2] = __ldcg((const float2*)(w + AM_DH));
+          os[u2] = __ldcg((const float4*)(w + 4 * lane));
+        } else {
+          ml[u2] = make_float2(-INFINITY, 0.f);
+          os[u2] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
       }
-      const float f = exp2f(ml.x - M);
-      o.x += f * os.x; o.y += f * os.y; o.z += f * os.z; o.w += f * os.w;
-      l += f * ml.y;
+#pragma unroll
+      for (int u2 = 0; u2 < 8; ++u2) {
+        if (ml[u2].x == -INFINITY) continue;
+        if (ml[u2].x > M) {
+          const float f = (M == -INFINITY) ? 0.f : exp2f(M - ml[u2].x);
+          o.x *= f; o.y *= f; o.z *= f; o.w *= f;
+          l *= f;
+          M = ml[u2].x;
+        }
+        const float f = exp2f(ml[u2].x - M);
+        o.x += f * os[u2].x; o.y += f * os[u2].y; o.z += f * os[u2].z; o.w += f * os[u2].w;
+        l += f * ml[u2].y;
+      }
     }
     const float inv = 1.f / l;
     const int j = q / 16, i = q % 16;

@@ -7,6 +7,7 @@
 
 #include <mutex>
 #include <unordered_map>
+#include <utility>
 
 namespace fm {
 
@@ -95,6 +96,35 @@ __device__ __forceinline__ ArgMax block_argmax(ArgMax a, float* shv, int* shi) {
   if (lane < nw) { a.v = shv[lane]; a.i = shi[lane]; } else { a.v = -INFINITY; a.i = 0x7fffffff; }
   a = warp_argmax(a);
   return a;
+}
+
+// Programmatic dependent launch.  A kernel launched with the programmatic
+// stream-serialization attribute may start while the previous kernel on the
+// stream is still running: pdl_wait() blocks until that kernel has finished
+// and its memory is visible; pdl_trigger() lets the next kernel launch once
+// every CTA of this one has started.  Both are no-ops without the attribute.
+// Every kernel here calls pdl_wait() before its first global write and
+// before reading anything an earlier kernel produced.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launch with the programmatic stream-serialization attribute.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // Raises a kernel's dynamic shared-memory limit once per (kernel, device):

@@ -9,6 +9,8 @@ namespace fm {
 // 256-wide time features of s and t: [cos(1000 tau f_j), sin(1000 tau f_j)],
 // f_j = 10000^(-j/128), evaluated in fp64.
 __global__ void k_time_features(double s, double t, float* __restrict__ phi) {
+  pdl_wait();
+  pdl_trigger();
   int e = threadIdx.x;  // 0..255
   int j = e & 127;
   double f = exp(-log(10000.0) * (double)j / 128.0);
@@ -23,6 +25,8 @@ __global__ void k_time_features(double s, double t, float* __restrict__ phi) {
 template <typename T>
 __global__ void k_gemv(const T* __restrict__ W, int n_out, int n_in, const float* __restrict__ x,
                        float* __restrict__ y, const float* __restrict__ add, int act) {
+  pdl_wait();
+  pdl_trigger();
   int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= n_out) return;
   const T* row = W + (size_t)warp * n_in;
@@ -37,6 +41,8 @@ __global__ void k_gemv(const T* __restrict__ W, int n_out, int n_in, const float
 }
 
 __global__ void k_silu_vec(const float* __restrict__ x, float* __restrict__ y, int n) {
+  pdl_wait();
+  pdl_trigger();
   int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) y[i] = silu(x[i]);
 }
@@ -49,6 +55,8 @@ template <typename TI, typename TO>
 __global__ void __launch_bounds__(256)
 k_adaln(const TI* __restrict__ x, int d, const float* __restrict__ shift,
         const float* __restrict__ scale, TO* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float sh[32];
   const int m = blockIdx.x;
   const TI* row = x + (size_t)m * d;
@@ -75,6 +83,8 @@ k_adaln(const TI* __restrict__ x, int d, const float* __restrict__ shift,
 template <typename TO>
 __global__ void __launch_bounds__(1024)
 k_softmax_rows(const float* __restrict__ logits, int V, TO* __restrict__ D) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float sh[32];
   const float* row = logits + (size_t)blockIdx.x * V;
   float mx = -INFINITY;
@@ -172,6 +182,8 @@ __global__ void __launch_bounds__(1024)
 k_select_tokens(const float* __restrict__ logits, int V, const float* __restrict__ part_v,
                 const int* __restrict__ part_i, int n_part, const double* __restrict__ u,
                 TempArgs ta, int* __restrict__ tokens) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float shv[32];
   __shared__ int shi[32];
   __shared__ double shd[32];
@@ -212,6 +224,8 @@ k_select_tokens(const float* __restrict__ logits, int V, const float* __restrict
 // out[c][r] = in[r][c] for in [R][C]; 32 x 32 tiles.
 template <typename T>
 __global__ void k_transpose(const T* __restrict__ in, T* __restrict__ out, int R, int C) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ T tile[32][33];
   int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
   for (int i = threadIdx.y; i < 32; i += 8) {

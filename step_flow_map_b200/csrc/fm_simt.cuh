@@ -98,6 +98,8 @@ template <typename TA, typename TW, bool WK, class Epi>
 __global__ void __launch_bounds__(256)
 k_gemm_simt(const TA* __restrict__ A, int lda, const TW* __restrict__ W, int ldw,
             int M, int N, int Kd, int k_split, float* __restrict__ partial, Epi epi) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float As[SG_BK][SG_BM];
   __shared__ float Ws[SG_BK][SG_BN + 1];
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
@@ -155,6 +157,8 @@ k_gemm_simt(const TA* __restrict__ A, int lda, const TW* __restrict__ W, int ldw
 
 template <class Epi>
 __global__ void k_splitk_apply(const float* __restrict__ partial, int splits, int M, int N, Epi epi) {
+  pdl_wait();
+  pdl_trigger();
   size_t total = (size_t)M * N;
   for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total;
        e += (size_t)gridDim.x * blockDim.x) {
@@ -183,6 +187,8 @@ template <typename T>
 __global__ void __launch_bounds__(128)
 k_attn_simt(const T* __restrict__ qkv, const T* __restrict__ Kc, const T* __restrict__ Vc,
             T* __restrict__ out, AttnArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.x, h = blockIdx.y, j = blockIdx.z;
   const int dh = a.d / a.n_heads, K = a.K, d3 = 3 * a.d;
   const int L = a.len[b];

@@ -184,12 +184,24 @@ struct TcArgs {
   int* err;
 };
 
+// Ring depth: "deep" (about 200 KB, one CTA per SM) for long weight streams
+// per CTA; "shallow" (about 100 KB) for short ones, so that two CTAs -- the
+// running GEMM's and the next GEMM's, launched early -- share an SM and the
+// next weight stream starts while the current one drains.
 template <int BN>
+__host__ __device__ constexpr int tc_stages(bool deep) {
+  return deep ? ((200 * 1024) / (TC_BM * TC_BK * 2 + BN * TC_BK * 2) > 12
+                     ? 12
+                     : (200 * 1024) / (TC_BM * TC_BK * 2 + BN * TC_BK * 2))
+              : (100 * 1024) / (TC_BM * TC_BK * 2 + BN * TC_BK * 2);
+}
+
+template <int BN, int STAGES_>
 struct TcCfg {
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;  // 16 KB
   static constexpr int B_BYTES = BN * TC_BK * 2;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (200 * 1024) / STAGE > 12 ? 12 : (200 * 1024) / STAGE;
+  static constexpr int STAGES = STAGES_;
   static constexpr int TMEM_COLS = (2 * BN) < 32 ? 32 : 2 * BN;
   static constexpr int SMEM = STAGES * STAGE + 1024 /*align*/ + 256 /*barriers*/ + 8 * BN * 4;
 };
@@ -220,11 +232,12 @@ __device__ __forceinline__ void tc_finish_chunk(const Epi& epi, const TcArgs& a,
   }
 }
 
-template <int BN, class Epi>
+template <int BN, int STAGES, class Epi>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 k_tc_gemm(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUtensorMap mapA,
           TcArgs a, Epi epi) {
-  using C = TcCfg<BN>;
+  using C = TcCfg<BN, STAGES>;
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sA = base;
@@ -271,10 +284,32 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUte
       asm volatile("prefetch.tensormap [%0];" ::"l"((unsigned long long)&mapA) : "memory");
       int stage = 0;
       uint32_t phase = 0;
-      for (int u = blockIdx.x; u < a.units && !*abort; u += gridDim.x) {
+      // Weights do not depend on earlier kernels: the first unit's weight
+      // tiles go out before the dependency wait, the activation tiles after.
+      int npre = 0;
+      {
+        const int u = blockIdx.x;
         const int mt = u % a.m_tiles, rest = u / a.m_tiles;
         const int z = rest % a.splits, nt = rest / a.splits;
         const int kb0 = (int)((long)z * a.k_blocks / a.splits);
+        const int kb1 = (int)((long)(z + 1) * a.k_blocks / a.splits);
+        npre = min(C::STAGES, kb1 - kb0);
+        for (int i = 0; i < npre; ++i) {
+          const uint32_t fb = smem_u32(&full[i]);
+          mbar_expect_tx(fb, C::STAGE);
+          tma_load_2d(smem_u32(sA + i * C::A_BYTES), &mapW, (kb0 + i) * TC_BK, nt * TC_BM, fb);
+        }
+        pdl_wait();
+        for (int i = 0; i < npre; ++i)
+          tma_load_2d(smem_u32(sB + i * C::B_BYTES), &mapA, (kb0 + i) * TC_BK, mt * BN,
+                      smem_u32(&full[i]));
+        stage = npre % C::STAGES;
+        phase = (npre == C::STAGES) ? 1u : 0u;
+      }
+      for (int u = blockIdx.x; u < a.units && !*abort; u += gridDim.x) {
+        const int mt = u % a.m_tiles, rest = u / a.m_tiles;
+        const int z = rest % a.splits, nt = rest / a.splits;
+        const int kb0 = (int)((long)z * a.k_blocks / a.splits) + (u == (int)blockIdx.x ? npre : 0);
         const int kb1 = (int)((long)(z + 1) * a.k_blocks / a.splits);
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort)) break;
@@ -323,6 +358,7 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUte
     const int q = warp & 3;
     const int r = q * 32 + lane;          // feature row within the tile
     const int et = threadIdx.x - 64;      // 0..127
+    pdl_wait();                           // epilogues read and write earlier kernels' data
     int acc = 0;
     uint32_t acc_phase = 0;
     int it = 0;
@@ -523,11 +559,26 @@ inline int tc_pick_bn(int M) {
   return 256;
 }
 
+template <int BN, int STAGES, class Epi>
+fm_status tc_launch_cfg(const TcMap& wm, const CUtensorMap& mapA, const TcArgs& a, int grid, Epi epi,
+                        cudaStream_t st, char* err, size_t errlen, int* n_launch) {
+  using C = TcCfg<BN, STAGES>;
+  cudaError_t e = set_smem_once(k_tc_gemm<BN, STAGES, Epi>, C::SMEM);
+  if (e == cudaSuccess)
+    e = launch_pdl(k_tc_gemm<BN, STAGES, Epi>, dim3(grid), dim3(TC_THREADS), C::SMEM, st, wm.map,
+                   mapA, a, epi);
+  if (e != cudaSuccess) {
+    snprintf(err, errlen, "tensor-core GEMM launch: %s", cudaGetErrorString(e));
+    return FM_ERR_CUDA;
+  }
+  if (n_launch) ++*n_launch;
+  return FM_OK;
+}
+
 template <int BN, class Epi>
 fm_status tc_launch(const TcMap& wm, const bf16* A, int lda, int M, Epi epi, float* partial,
                     size_t partial_elems, unsigned* tile_cnt, int tile_cnt_n, int sms, int* err_word,
                     cudaStream_t st, char* err, size_t errlen, int* n_launch) {
-  using C = TcCfg<BN>;
   TcArgs a;
   a.M = M;
   a.N = wm.N;
@@ -550,22 +601,14 @@ fm_status tc_launch(const TcMap& wm, const bf16* A, int lda, int M, Epi epi, flo
   a.err = err_word;
   CUtensorMap mapA;
   if (!tc_encode(&mapA, A, wm.Kd, M, lda, BN, err, errlen)) return FM_ERR_CUDA;
-  {
-    cudaError_t e = set_smem_once(k_tc_gemm<BN, Epi>, C::SMEM);
-    if (e != cudaSuccess) {
-      snprintf(err, errlen, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-      return FM_ERR_CUDA;
-    }
-  }
   const int grid = a.units < sms ? a.units : sms;
-  k_tc_gemm<BN, Epi><<<grid, TC_THREADS, C::SMEM, st>>>(wm.map, mapA, a, epi);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) {
-    snprintf(err, errlen, "tensor-core GEMM launch: %s", cudaGetErrorString(e));
-    return FM_ERR_CUDA;
+  // k-blocks one CTA streams: deep ring for long streams, shallow otherwise
+  const long per_cta = (long)((a.units + grid - 1) / grid) * ((a.k_blocks + a.splits - 1) / a.splits);
+  if constexpr (BN <= 64) {
+    if (per_cta < 24)
+      return tc_launch_cfg<BN, tc_stages<BN>(false)>(wm, mapA, a, grid, epi, st, err, errlen, n_launch);
   }
-  if (n_launch) ++*n_launch;
-  return FM_OK;
+  return tc_launch_cfg<BN, tc_stages<BN>(true)>(wm, mapA, a, grid, epi, st, err, errlen, n_launch);
 }
 
 template <class Epi>

@@ -24,6 +24,8 @@ k_verify_greedy(const float* __restrict__ tgt, const int* __restrict__ draft, in
                 int K, int V, int chunks, float* __restrict__ pv, int* __restrict__ pi,
                 unsigned* __restrict__ counter, int* __restrict__ n_acc,
                 int* __restrict__ branch, int* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float shv[32];
   __shared__ int shi[32];
   __shared__ int amax[VG_MAX_ROWS];
@@ -90,6 +92,8 @@ __global__ void __launch_bounds__(VS_THREADS)
 k_row_stats(const float* __restrict__ tgt, const float* __restrict__ dlog, int n_tgt_rows,
             int n_rows, int V, int chunks, float T, float* __restrict__ pm,
             double* __restrict__ ps) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float shf[32];
   __shared__ double shd[32];
   const int row = blockIdx.x / chunks, c = blockIdx.x - row * chunks;
@@ -137,6 +141,8 @@ k_verify_sample_decide(const float* __restrict__ tgt, const float* __restrict__ 
                        const float* __restrict__ pm, const double* __restrict__ ps, int chunks,
                        double* __restrict__ resid, int* __restrict__ n_acc,
                        int* __restrict__ branch, int* __restrict__ out) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ double shd[32];
   __shared__ int s_accept, s_mode, s_buf;
   __shared__ double s_mp, s_Sp, s_mq, s_Sq;
