@@ -199,3 +199,4 @@ def fm_profile_read(ctx, reset: bool = False):
 def fm_device_status(ctx, stream=None) -> None:
     """Raise FlashmapError(FM_ERR_TIMEOUT) if a kernel's bounded wait gave up."""
     _check(load_library().fm_device_status(ctx, _stream(stream)))
+

@@ -136,12 +136,21 @@ struct Prof {
     if (((c->prof_mask >> cls) & 1) && c->ev_used < c->ev_a.size()) {
       slot = (long)c->ev_used++;
       c->ev_cls[slot] = cls;
-      // "external" records also become real timing records inside a CUDA graph
-      cudaEventRecordWithFlags(c->ev_a[slot], st, cudaEventRecordExternal);
+      record(c->ev_a[slot]);
     }
   }
   ~Prof() {
-    if (slot >= 0) cudaEventRecordWithFlags(c->ev_b[slot], st, cudaEventRecordExternal);
+    if (slot >= 0) record(c->ev_b[slot]);
+  }
+  // inside a stream capture only "external" records become timing records
+  // of the graph; outside a capture the plain record is the valid one
+  void record(cudaEvent_t e) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(st, &cs);
+    if (cs == cudaStreamCaptureStatusActive)
+      cudaEventRecordWithFlags(e, st, cudaEventRecordExternal);
+    else
+      cudaEventRecord(e, st);
   }
 };
 
