@@ -185,6 +185,25 @@ fm_status fm_verify_sample(fm_ctx *ctx, const float *target_logits, const float 
                            int32_t *n_acc, int32_t *branch, int32_t *out_tokens,
                            fm_stream stream);
 
+/* Greedy verify that allocates nothing and needs no context: same inputs,
+ * outputs and bit-exact results as fm_verify_greedy (the pages have no
+ * counterpart; this is a deployment variant).  It is for callers that
+ * cannot allocate device memory -- servers whose arena owns the whole
+ * device, or verify-only users without a drafter context.  Its scratch is a
+ * fixed device array inside the library (about 260 KB on every GPU that
+ * loads it, kept until exit), so: B <= 1024, N*(K+1) <= 1024 and
+ * B*N*(K+1) <= 32768, else FM_ERR_UNSUPPORTED.  The first call on a device
+ * looks the array up (cudaGetSymbolAddress) and should come before any
+ * stream capture.  Each call clears the scratch counters it uses; all calls
+ * share the one array, so calls that overlap on the same GPU (issued on
+ * different streams or from different host threads) race and must be
+ * serialised by the caller.  No cudaMalloc, cudaFree or allocating library
+ * call is made. */
+fm_status fm_verify_greedy_noalloc(const float *target_logits, const int32_t *draft,
+                                   int B, int N, int K, int V,
+                                   int32_t *n_acc, int32_t *branch, int32_t *out_tokens,
+                                   fm_stream stream);
+
 /* Reads and clears the context's device error word: FM_OK, or
  * FM_ERR_TIMEOUT when a bounded wait inside a kernel gave up (the kernel
  * then stopped early and its outputs are invalid).  Waits for the work

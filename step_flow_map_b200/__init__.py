@@ -25,6 +25,7 @@ FM_MAX_STEPS = 8
 EXPORTS = (
     "fm_load_weights", "fm_free", "fm_last_error", "fm_project_context",
     "fm_draft", "fm_verify_greedy", "fm_verify_sample", "fm_profile", "fm_profile_read", "fm_device_status",
+    "fm_verify_greedy_noalloc",
 )
 FM_PROF = {"embed": 0, "dit_gemm": 1, "attn": 2, "norm": 3, "lm_head": 4, "context": 5,
            "verify": 6, "other": 7}
@@ -83,6 +84,8 @@ def load_library(path: str = LIB_PATH):
     lib.fm_verify_greedy.argtypes = [p, p, p, i, i, i, i, p, p, p, st]
     lib.fm_verify_sample.restype = i
     lib.fm_verify_sample.argtypes = [p, p, p, p, i, i, i, i, f, p, p, p, p, p, st]
+    lib.fm_verify_greedy_noalloc.restype = i
+    lib.fm_verify_greedy_noalloc.argtypes = [p, p, i, i, i, i, p, p, p, st]
     lib.fm_device_status.restype = i
     lib.fm_device_status.argtypes = [p, st]
     lib.fm_profile.restype = i
@@ -200,3 +203,10 @@ def fm_device_status(ctx, stream=None) -> None:
     """Raise FlashmapError(FM_ERR_TIMEOUT) if a kernel's bounded wait gave up."""
     _check(load_library().fm_device_status(ctx, _stream(stream)))
 
+
+def fm_verify_greedy_noalloc(target_logits, draft, B, N, K, V, n_acc, branch, out_tokens,
+                             stream=None) -> None:
+    """Greedy verify without a context or any device allocation (see the header)."""
+    _check(load_library().fm_verify_greedy_noalloc(_ptr(target_logits), _ptr(draft), B, N, K, V,
+                                                   _ptr(n_acc), _ptr(branch), _ptr(out_tokens),
+                                                   _stream(stream)))

@@ -802,3 +802,85 @@ extern "C" fm_status fm_device_status(fm_ctx* c, fm_stream stream) {
   }
   return FM_OK;
 }
+
+// ------------------------------------------------------------------ greedy verify without allocation
+// Some callers cannot allocate device memory at call time: inference servers
+// that reserve the whole device in their own arena and forbid further
+// cudaMalloc, and verify-only users who bring their own drafter and do not
+// want a drafter context (fm_load_weights allocates the weight copy, caches
+// and workspaces).  fm_verify_greedy_noalloc serves them: it runs the same
+// greedy-verify kernel as fm_verify_greedy, with its scratch (per-chunk
+// partial maxima and per-sequence arrival counters) in the file-scope device
+// array below instead of a context's workspace.  Every GPU that loads the
+// library holds this array (about 260 KB) until the process exits.
+#define FM_NOALLOC_PARTIALS 32768  /* (row, vocabulary chunk) partials */
+#define FM_NOALLOC_SEQS 1024       /* sequences per call */
+
+namespace {
+struct NoallocScratch {
+  float pv[FM_NOALLOC_PARTIALS];
+  int pi[FM_NOALLOC_PARTIALS];
+  unsigned cnt[FM_NOALLOC_SEQS];
+};
+}  // namespace
+
+static __device__ __align__(256) NoallocScratch g_noalloc_scratch;
+
+// Device address of the scratch for the current device, looked up once per
+// device (the name is only a host-side stand-in for the device symbol).
+static fm_status noalloc_scratch(NoallocScratch** out, int* sms) {
+  static std::mutex mu;
+  static NoallocScratch* addr[64] = {};
+  static int sm_count[64] = {};
+  int dev = 0;
+  FM_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return set_err(FM_ERR_UNSUPPORTED, "device id %d >= 64", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return set_err(FM_ERR_CUDA, "cudaGetSymbolAddress(scratch) failed: %s", cudaGetErrorString(e));
+    FM_CUDA(cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev));
+    addr[dev] = (NoallocScratch*)p;
+  }
+  *out = addr[dev];
+  *sms = sm_count[dev];
+  return FM_OK;
+}
+
+extern "C" fm_status fm_verify_greedy_noalloc(const float* target_logits, const int32_t* draft,
+                                              int B, int N, int K, int V, int32_t* n_acc,
+                                              int32_t* branch, int32_t* out_tokens,
+                                              fm_stream stream) {
+  if (!target_logits || !draft || !n_acc || !branch || !out_tokens)
+    return set_err(FM_ERR_ARG, "NULL argument");
+  if (B < 1 || N < 1 || K < 1 || V < 1) return set_err(FM_ERR_ARG, "sizes must be positive");
+  if (B > FM_NOALLOC_SEQS)
+    return set_err(FM_ERR_UNSUPPORTED, "B=%d exceeds the no-allocation limit of %d sequences", B,
+                   FM_NOALLOC_SEQS);
+  if (N * (K + 1) > fm::VG_MAX_ROWS)
+    return set_err(FM_ERR_UNSUPPORTED, "N*(K+1)=%d exceeds %d rows per sequence", N * (K + 1),
+                   fm::VG_MAX_ROWS);
+  const long rows = (long)B * N * (K + 1);
+  if (rows > FM_NOALLOC_PARTIALS)
+    return set_err(FM_ERR_UNSUPPORTED, "B*N*(K+1)=%ld exceeds the no-allocation limit of %d rows",
+                   rows, FM_NOALLOC_PARTIALS);
+  NoallocScratch* s = nullptr;
+  int sms = 148;
+  FM_TRY(noalloc_scratch(&s, &sms));
+  long want = (2L * sms + rows - 1) / rows;
+  int ch = (int)std::min<long>(want, 64);
+  ch = std::min(ch, std::max(1, V / 1024));
+  ch = (int)std::min<long>(ch, FM_NOALLOC_PARTIALS / rows);
+  ch = std::max(ch, 1);
+  cudaStream_t st = (cudaStream_t)stream;
+  // the counters start at zero (the kernel also returns them to zero)
+  FM_CUDA(cudaMemsetAsync(s->cnt, 0, (size_t)B * sizeof(unsigned), st));
+  cudaError_t e = fm::launch_pdl(fm::k_verify_greedy, dim3((unsigned)(rows * ch)),
+                                 dim3(fm::VG_THREADS), 0, st, target_logits, draft, B, N, K, V, ch,
+                                 s->pv, s->pi, s->cnt, n_acc, branch, out_tokens);
+  if (e != cudaSuccess)
+    return set_err(FM_ERR_CUDA, "greedy verify launch failed: %s", cudaGetErrorString(e));
+  return FM_OK;
+}
