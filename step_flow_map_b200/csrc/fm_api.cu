@@ -225,6 +225,26 @@ fm_status gemm_w(fm_ctx* c, int cls, const T* A, int lda, const T* W, int M, int
   return gemm_simt<T, T, Epi>(c, cls, A, lda, W, Kd, true, M, N, Kd, epi, st);
 }
 
+// GEMM whose input is the modulated LayerNorm of the residual stream,
+// LN0(x)(1 + scale) + shift, computed inside the tensor-core kernel.  Sets
+// *done = false (and launches nothing) when the shape needs the separate
+// LayerNorm kernel instead.
+template <class Epi>
+fm_status gemm_ln(fm_ctx* c, int cls, const float* x, const float* shift, const float* scale,
+                  int M, Epi epi, cudaStream_t st, const fm::TcMap* map, bool* done) {
+  *done = false;
+  if (!c->use_tc || !map || !map->valid || M > 32) return FM_OK;
+  Prof prof(c, cls, st);
+  int n_launch = 0;
+  fm_status s = fm::tc_gemm_ln(c->tc, *map, x, shift, scale, M, epi, c->splitk, c->splitk_elems,
+                               c->tile_cnt, c->tile_cnt_n, c->sms, st, g_err, sizeof(g_err),
+                               &n_launch);
+  c->launches[cls] += n_launch;
+  if (s == FM_ERR_UNSUPPORTED) return FM_OK;
+  if (s == FM_OK) *done = true;
+  return s;
+}
+
 // ------------------------------------------------------------------ conditioning
 template <typename T>
 fm_status compute_mods(fm_ctx* c, float s, float t, float* out, cudaStream_t st) {
@@ -511,13 +531,18 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
     }
     for (int l = 0; l < nb; ++l) {
       const float* ml = mods + (size_t)l * 6 * d;
-      {
-        Prof prof(c, FM_PROF_NORM, st);
-        FM_LAUNCH(c, FM_PROF_NORM, (fm::k_adaln<float, T>), M, 256, 0, st,
-              c->x, d, ml, ml + d, h);
+      bool fused = false;
+      FM_TRY(gemm_ln(c, FM_PROF_DIT_GEMM, c->x, ml, ml + d, M, fm::EpiStore<T>{qkv, 3 * d}, st,
+                     &c->tc.qkv[l], &fused));
+      if (!fused) {
+        {
+          Prof prof(c, FM_PROF_NORM, st);
+          FM_LAUNCH(c, FM_PROF_NORM, (fm::k_adaln<float, T>), M, 256, 0, st,
+                c->x, d, ml, ml + d, h);
+        }
+        FM_TRY(gemm_w<T>(c, FM_PROF_DIT_GEMM, h, d, (const T*)c->wqkv[l], M, 3 * d, d,
+                         fm::EpiStore<T>{qkv, 3 * d}, st, &c->tc.qkv[l]));
       }
-      FM_TRY(gemm_w<T>(c, FM_PROF_DIT_GEMM, h, d, (const T*)c->wqkv[l], M, 3 * d, d,
-                       fm::EpiStore<T>{qkv, 3 * d}, st, &c->tc.qkv[l]));
       {
         Prof prof(c, FM_PROF_ATTN, st);
         if (use_mma_attn) {
@@ -531,36 +556,48 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
       }
       FM_TRY(gemm_w<T>(c, FM_PROF_DIT_GEMM, o, d, (const T*)c->wo[l], M, d, d,
                        fm::EpiResidual{c->x, ml + 2 * d, d}, st, &c->tc.o[l]));
-      {
-        Prof prof(c, FM_PROF_NORM, st);
-        FM_LAUNCH(c, FM_PROF_NORM, (fm::k_adaln<float, T>), M, 256, 0, st,
-              c->x, d, ml + 3 * d,
-                                                                            ml + 4 * d, h);
+      FM_TRY(gemm_ln(c, FM_PROF_DIT_GEMM, c->x, ml + 3 * d, ml + 4 * d, M, fm::EpiGelu<T>{u, F}, st,
+                     &c->tc.up[l], &fused));
+      if (!fused) {
+        {
+          Prof prof(c, FM_PROF_NORM, st);
+          FM_LAUNCH(c, FM_PROF_NORM, (fm::k_adaln<float, T>), M, 256, 0, st,
+                c->x, d, ml + 3 * d, ml + 4 * d, h);
+        }
+        FM_TRY(gemm_w<T>(c, FM_PROF_DIT_GEMM, h, d, (const T*)c->wup[l], M, F, d,
+                         fm::EpiGelu<T>{u, F}, st, &c->tc.up[l]));
       }
-      FM_TRY(gemm_w<T>(c, FM_PROF_DIT_GEMM, h, d, (const T*)c->wup[l], M, F, d,
-                       fm::EpiGelu<T>{u, F}, st, &c->tc.up[l]));
       FM_TRY(gemm_w<T>(c, FM_PROF_DIT_GEMM, u, F, (const T*)c->wdown[l], M, d, F,
                        fm::EpiResidual{c->x, ml + 5 * d, d}, st, &c->tc.down[l]));
     }
     const float* mf = mods + (size_t)nb * 6 * d;
-    {
-      Prof prof(c, FM_PROF_NORM, st);
-      FM_LAUNCH(c, FM_PROF_NORM, (fm::k_adaln<float, T>), M, 256, 0, st,
-              c->x, d, mf, mf + d, h);
-    }
     // LM head: greedy-only final steps keep the logits on chip when possible
     const bool need_logits = !last || any_sample || draft_logits != nullptr;
-    bool have_partials = false;
-    if (c->use_tc && c->tc.lm.valid && !need_logits) {
-      Prof prof(c, FM_PROF_LM_HEAD, st);
-      int n_launch = 0;
-      FM_TRY(fm::tc_lm_head_argmax(c->tc, (const bf16*)h, d, M, V, c->part_v, c->part_i,
-                                   c->n_part, c->sms, st, g_err, sizeof(g_err), &n_launch));
-      c->launches[FM_PROF_LM_HEAD] += n_launch;
-      have_partials = true;
+    bool have_partials = false, fused = false;
+    if (need_logits) {
+      FM_TRY(gemm_ln(c, FM_PROF_LM_HEAD, c->x, mf, mf + d, M, fm::EpiStoreF32{logits, V}, st,
+                     &c->tc.lm, &fused));
     } else {
-      FM_TRY(gemm_w<T>(c, FM_PROF_LM_HEAD, h, d, (const T*)c->w.W_lm, M, V, d,
-                       fm::EpiStoreF32{logits, V}, st, &c->tc.lm));
+      FM_TRY(gemm_ln(c, FM_PROF_LM_HEAD, c->x, mf, mf + d, M,
+                     fm::EpiArgmax{c->part_v, c->part_i, c->n_part}, st, &c->tc.lm, &fused));
+      have_partials = fused;
+    }
+    if (!fused) {
+      {
+        Prof prof(c, FM_PROF_NORM, st);
+        FM_LAUNCH(c, FM_PROF_NORM, (fm::k_adaln<float, T>), M, 256, 0, st, c->x, d, mf, mf + d, h);
+      }
+      if (c->use_tc && c->tc.lm.valid && !need_logits) {
+        Prof prof(c, FM_PROF_LM_HEAD, st);
+        int n_launch = 0;
+        FM_TRY(fm::tc_lm_head_argmax(c->tc, (const bf16*)h, d, M, V, c->part_v, c->part_i,
+                                     c->n_part, c->sms, st, g_err, sizeof(g_err), &n_launch));
+        c->launches[FM_PROF_LM_HEAD] += n_launch;
+        have_partials = true;
+      } else {
+        FM_TRY(gemm_w<T>(c, FM_PROF_LM_HEAD, h, d, (const T*)c->w.W_lm, M, V, d,
+                         fm::EpiStoreF32{logits, V}, st, &c->tc.lm));
+      }
     }
     Prof prof(c, FM_PROF_NORM, st);
     if (!last) {

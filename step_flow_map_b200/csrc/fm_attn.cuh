@@ -21,6 +21,7 @@ namespace fm {
 
 constexpr int AM_DH = 128;            // head width
 constexpr int AM_CHUNK = 64;          // context rows per smem stage
+constexpr int AM_STAGES = 3;          // context chunks in flight per CTA
 constexpr int AM_LD = AM_DH + 8;      // padded smem row (272 bytes): conflict-free ldmatrix
 constexpr int AM_THREADS = 128;
 constexpr int AM_PSTRIDE = AM_DH + 4;  // floats per partial row: O[128], m, l, pad (16-byte rows)
@@ -169,8 +170,8 @@ k_attn_mma(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc, const bf16
   pdl_trigger();
   extern __shared__ __align__(16) uint8_t smem_raw[];
   bf16* sQ = (bf16*)smem_raw;                       // [N*16][AM_LD]
-  bf16* sK = sQ + N * 16 * AM_LD;                   // [2][AM_CHUNK][AM_LD]
-  bf16* sV = sK + 2 * AM_CHUNK * AM_LD;             // [2][AM_CHUNK][AM_LD]
+  bf16* sK = sQ + N * 16 * AM_LD;                   // [AM_STAGES][AM_CHUNK][AM_LD]
+  bf16* sV = sK + AM_STAGES * AM_CHUNK * AM_LD;     // [AM_STAGES][AM_CHUNK][AM_LD]
   __shared__ int s_last;
   constexpr int WPM = 4 / N;                        // warps sharing one 16-query tile
   const int pair = blockIdx.x, split = blockIdx.y;
@@ -192,9 +193,7 @@ k_attn_mma(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc, const bf16
   st.l[0] = st.l[1] = 0.f;
 
   uint32_t qa[8][4];
-  auto load_q = [&]() {
-    cp_wait<0>();
-    __syncthreads();
+  auto q_fragments = [&]() {
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
       const int r = mt * 16 + (lane & 15), c = kk * 16 + (lane >> 4) * 8;
@@ -209,23 +208,28 @@ k_attn_mma(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc, const bf16
     const int k1 = (int)((long)(split + 1) * L / a.n_ctx_splits);
     const size_t base = (size_t)a.slot[b] * a.max_ctx * a.d + h * AM_DH;
     const int n_chunks = (k1 - k0 + AM_CHUNK - 1) / AM_CHUNK;
-    if (n_chunks > 0) {
-      const int nr = min(AM_CHUNK, k1 - k0);
-      load_rows(sK, Kc + base + (size_t)k0 * a.d, a.d, nr, AM_CHUNK);
-      load_rows(sV, Vc + base + (size_t)k0 * a.d, a.d, nr, AM_CHUNK);
-    }
-    cp_commit();
-    load_q();
-    for (int c = 0; c < n_chunks; ++c) {
-      const int buf = c & 1;
-      if (c + 1 < n_chunks) {
-        const int r0 = k0 + (c + 1) * AM_CHUNK, nr = min(AM_CHUNK, k1 - r0);
-        load_rows(sK + (buf ^ 1) * AM_CHUNK * AM_LD, Kc + base + (size_t)r0 * a.d, a.d, nr, AM_CHUNK);
-        load_rows(sV + (buf ^ 1) * AM_CHUNK * AM_LD, Vc + base + (size_t)r0 * a.d, a.d, nr, AM_CHUNK);
-      }
+    auto load_chunk = [&](int c) {
+      const int r0 = k0 + c * AM_CHUNK, nr = min(AM_CHUNK, k1 - r0);
+      const int buf = c % AM_STAGES;
+      load_rows(sK + buf * AM_CHUNK * AM_LD, Kc + base + (size_t)r0 * a.d, a.d, nr, AM_CHUNK);
+      load_rows(sV + buf * AM_CHUNK * AM_LD, Vc + base + (size_t)r0 * a.d, a.d, nr, AM_CHUNK);
+    };
+    // one commit group per chunk (empty past the end) keeps the group count
+    // fixed: AM_STAGES - 1 chunks are always in flight ahead of the one used
+#pragma unroll
+    for (int c = 0; c < AM_STAGES - 1; ++c) {
+      if (c < n_chunks) load_chunk(c);
       cp_commit();
-      cp_wait<1>();
+    }
+    cp_wait<AM_STAGES - 1>();   // the query group
+    __syncthreads();
+    q_fragments();
+    for (int c = 0; c < n_chunks; ++c) {
+      if (c + AM_STAGES - 1 < n_chunks) load_chunk(c + AM_STAGES - 1);
+      cp_commit();
+      cp_wait<AM_STAGES - 1>();
       __syncthreads();
+      const int buf = c % AM_STAGES;
       const int nk_chunk = min(AM_CHUNK, k1 - (k0 + c * AM_CHUNK));
       constexpr int KW = AM_CHUNK / WPM;            // keys of this warp within the chunk
       const int kw0 = sub * KW;
@@ -250,7 +254,9 @@ k_attn_mma(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc, const bf16
       }
     }
     cp_commit();
-    load_q();
+    cp_wait<0>();
+    __syncthreads();
+    q_fragments();
     if (sub == 0) attn_block<2>(st, qa, sK + mt * 16 * AM_LD, sV + mt * 16 * AM_LD, 16, a.scale_log2);
     __syncthreads();
   }
@@ -353,7 +359,7 @@ k_attn_mma(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc, const bf16
 
 template <int N>
 constexpr int attn_mma_smem() {
-  return (N * 16 + 4 * AM_CHUNK) * AM_LD * 2;
+  return (N * 16 + 2 * AM_STAGES * AM_CHUNK) * AM_LD * 2;
 }
 
 }  // namespace fm

@@ -148,6 +148,11 @@ inline cudaError_t set_smem_once(F* kernel, int bytes) {
   return set_smem_once_ptr((const void*)kernel, bytes);
 }
 
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *(uint32_t*)&v;
+}
+
 __device__ __forceinline__ float gelu_tanh(float u) {
   const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
   return 0.5f * u * (1.f + tanhf(k0 * (u + 0.044715f * u * u * u)));

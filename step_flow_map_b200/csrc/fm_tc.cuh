@@ -182,6 +182,11 @@ struct TcArgs {
   float* partial;       // [splits][tiles][128][BN] fp32 (splits > 1)
   unsigned* tile_cnt;   // [tiles], zero between launches
   int* err;
+  // B operand computed in the kernel as LN0(x) (1 + scale) + shift (bf16)
+  const float* ln_x;    // [M][Kd] fp32
+  const float* ln_shift;
+  const float* ln_scale;
+  int b_kb;             // k-blocks of the shared-memory-resident B operand
 };
 
 // Ring depth: "deep" (about 200 KB, one CTA per SM) for long weight streams
@@ -232,7 +237,67 @@ __device__ __forceinline__ void tc_finish_chunk(const Epi& epi, const TcArgs& a,
   }
 }
 
-template <int BN, int STAGES, class Epi>
+// Modulated LayerNorm of the activation rows, written straight into the
+// shared-memory B operand (128-byte swizzle, K-major, one BN x 64 tile per
+// k-block) by the 128 epilogue threads before any accumulator is ready.
+// Rows past M are zero.  Row statistics in fp32, two passes.
+template <int BN>
+__device__ __forceinline__ void tc_ln_fill(uint8_t* sB, const TcArgs& a, int kb0, int nkb, int et,
+                                           float* s_stat) {
+  constexpr int TPR = 128 / BN;  // threads per row, consecutive lanes
+  const int Kd = a.Kd;
+  {
+    const int row = et / TPR, part = et % TPR;
+    const bool valid = row < a.M;
+    const float* xr = a.ln_x + (size_t)row * Kd;
+    float s = 0.f;
+    if (valid)
+      for (int c = part * 4; c < Kd; c += TPR * 4) {
+        const float4 v = *(const float4*)(xr + c);
+        s += (v.x + v.y) + (v.z + v.w);
+      }
+#pragma unroll
+    for (int o = 1; o < TPR; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float mean = s / (float)Kd;
+    float q = 0.f;
+    if (valid)
+      for (int c = part * 4; c < Kd; c += TPR * 4) {
+        const float4 v = *(const float4*)(xr + c);
+        const float a0 = v.x - mean, a1 = v.y - mean, a2 = v.z - mean, a3 = v.w - mean;
+        q += (a0 * a0 + a1 * a1) + (a2 * a2 + a3 * a3);
+      }
+#pragma unroll
+    for (int o = 1; o < TPR; o <<= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+    if (part == 0) {
+      s_stat[row] = mean;
+      s_stat[BN + row] = rsqrtf(q / (float)Kd + 1e-6f);
+    }
+  }
+  named_sync(1, 128);
+  constexpr int B_BYTES = BN * TC_BK * 2;
+  for (int idx = et; idx < nkb * BN * 8; idx += 128) {
+    const int kbi = idx / (BN * 8), rem = idx - kbi * (BN * 8);
+    const int row = rem >> 3, ch = rem & 7;
+    const int col = (kb0 + kbi) * TC_BK + ch * 8;
+    uint4 packed = make_uint4(0, 0, 0, 0);
+    if (row < a.M && col < Kd) {
+      const float mean = s_stat[row], rstd = s_stat[BN + row];
+      const float* xr = a.ln_x + (size_t)row * Kd + col;
+      const float4 x0 = *(const float4*)xr, x1 = *(const float4*)(xr + 4);
+      const float4 c0 = *(const float4*)(a.ln_scale + col), c1 = *(const float4*)(a.ln_scale + col + 4);
+      const float4 h0 = *(const float4*)(a.ln_shift + col), h1 = *(const float4*)(a.ln_shift + col + 4);
+      packed.x = pack_bf16x2((x0.x - mean) * rstd * (1.f + c0.x) + h0.x, (x0.y - mean) * rstd * (1.f + c0.y) + h0.y);
+      packed.y = pack_bf16x2((x0.z - mean) * rstd * (1.f + c0.z) + h0.z, (x0.w - mean) * rstd * (1.f + c0.w) + h0.w);
+      packed.z = pack_bf16x2((x1.x - mean) * rstd * (1.f + c1.x) + h1.x, (x1.y - mean) * rstd * (1.f + c1.y) + h1.y);
+      packed.w = pack_bf16x2((x1.z - mean) * rstd * (1.f + c1.z) + h1.z, (x1.w - mean) * rstd * (1.f + c1.w) + h1.w);
+    }
+    *(uint4*)(sB + kbi * B_BYTES + row * 128 + ((ch ^ (row & 7)) << 4)) = packed;
+  }
+  // generic-proxy writes must be visible to the tensor core's async proxy
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+template <int BN, int STAGES, bool LNB, class Epi>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 k_tc_gemm(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUtensorMap mapA,
           TcArgs a, Epi epi) {
@@ -240,18 +305,22 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUte
   pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  // ring of A (weight) tiles, then B: a ring of activation tiles, or with
+  // LNB one resident tile per k-block computed in the kernel
   uint8_t* sA = base;
   uint8_t* sB = base + C::STAGES * C::A_BYTES;
-  uint64_t* bars = (uint64_t*)(base + C::STAGES * C::STAGE);
+  const int data_bytes = LNB ? C::STAGES * C::A_BYTES + a.b_kb * C::B_BYTES : C::STAGES * C::STAGE;
+  uint64_t* bars = (uint64_t*)(base + data_bytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + C::STAGES;
   uint64_t* tfull = bars + 2 * C::STAGES;
   uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_slot = (uint32_t*)(tempty + 2);
+  uint64_t* bready = tempty + 2;
+  uint32_t* tmem_slot = (uint32_t*)(bready + 1);
   volatile int* abort = (volatile int*)(tmem_slot + 1);
   int* s_last = (int*)(tmem_slot + 2);
   volatile int* s_ok = (volatile int*)(tmem_slot + 3);  // two slots
-  float* red_v = (float*)(base + C::STAGES * C::STAGE + 256);
+  float* red_v = (float*)(base + data_bytes + 256);
   int* red_i = (int*)(red_v + 4 * BN);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -264,6 +333,7 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUte
       mbar_init(smem_u32(&tfull[i]), 1);
       mbar_init(smem_u32(&tempty[i]), 128);
     }
+    mbar_init(smem_u32(bready), 128);
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -296,13 +366,14 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUte
         npre = min(C::STAGES, kb1 - kb0);
         for (int i = 0; i < npre; ++i) {
           const uint32_t fb = smem_u32(&full[i]);
-          mbar_expect_tx(fb, C::STAGE);
+          mbar_expect_tx(fb, LNB ? C::A_BYTES : C::STAGE);
           tma_load_2d(smem_u32(sA + i * C::A_BYTES), &mapW, (kb0 + i) * TC_BK, nt * TC_BM, fb);
         }
         pdl_wait();
-        for (int i = 0; i < npre; ++i)
-          tma_load_2d(smem_u32(sB + i * C::B_BYTES), &mapA, (kb0 + i) * TC_BK, mt * BN,
-                      smem_u32(&full[i]));
+        if (!LNB)
+          for (int i = 0; i < npre; ++i)
+            tma_load_2d(smem_u32(sB + i * C::B_BYTES), &mapA, (kb0 + i) * TC_BK, mt * BN,
+                        smem_u32(&full[i]));
         stage = npre % C::STAGES;
         phase = (npre == C::STAGES) ? 1u : 0u;
       }
@@ -314,9 +385,9 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUte
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort)) break;
           const uint32_t fb = smem_u32(&full[stage]);
-          mbar_expect_tx(fb, C::STAGE);
+          mbar_expect_tx(fb, LNB ? C::A_BYTES : C::STAGE);
           tma_load_2d(smem_u32(sA + stage * C::A_BYTES), &mapW, kb * TC_BK, nt * TC_BM, fb);
-          tma_load_2d(smem_u32(sB + stage * C::B_BYTES), &mapA, kb * TC_BK, mt * BN, fb);
+          if (!LNB) tma_load_2d(smem_u32(sB + stage * C::B_BYTES), &mapA, kb * TC_BK, mt * BN, fb);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -329,7 +400,12 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUte
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      for (int u = blockIdx.x; u < a.units && !*abort; u += gridDim.x) {
+      // resident B starts at the first unit's k-block (every unit of a CTA
+      // shares it: one unit per CTA, or no split of K)
+      const int kb_res0 = (int)((long)((blockIdx.x / a.m_tiles) % a.splits) * a.k_blocks / a.splits);
+      bool b_ok = true;
+      if (LNB) b_ok = mbar_wait(smem_u32(bready), 0, abort);
+      for (int u = blockIdx.x; b_ok && u < a.units && !*abort; u += gridDim.x) {
         const int z = (u / a.m_tiles) % a.splits;
         const int kb0 = (int)((long)z * a.k_blocks / a.splits);
         const int kb1 = (int)((long)(z + 1) * a.k_blocks / a.splits);
@@ -341,7 +417,8 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUte
           if (!mbar_wait(smem_u32(&full[stage]), phase, abort)) { ok = false; break; }
           tc_fence_after();
           const uint64_t ad = desc_sw128(smem_u32(sA + stage * C::A_BYTES));
-          const uint64_t bd = desc_sw128(smem_u32(sB + stage * C::B_BYTES));
+          const uint64_t bd =
+              desc_sw128(smem_u32(sB + (LNB ? kb - kb_res0 : stage) * C::B_BYTES));
 #pragma unroll
           for (int k = 0; k < TC_BK / 16; ++k)
             tc_mma(d_tmem, ad + 2 * k, bd + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
@@ -359,6 +436,13 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUte
     const int r = q * 32 + lane;          // feature row within the tile
     const int et = threadIdx.x - 64;      // 0..127
     pdl_wait();                           // epilogues read and write earlier kernels' data
+    if constexpr (LNB) {
+      const int u = blockIdx.x;
+      const int z = (u / a.m_tiles) % a.splits;
+      const int kb0 = (int)((long)z * a.k_blocks / a.splits);
+      tc_ln_fill<BN>(sB, a, kb0, a.b_kb, et, red_v);
+      mbar_arrive(smem_u32(bready));
+    }
     int acc = 0;
     uint32_t acc_phase = 0;
     int it = 0;
@@ -559,13 +643,15 @@ inline int tc_pick_bn(int M) {
   return 256;
 }
 
-template <int BN, int STAGES, class Epi>
+template <int BN, int STAGES, class Epi, bool LNB = false>
 fm_status tc_launch_cfg(const TcMap& wm, const CUtensorMap& mapA, const TcArgs& a, int grid, Epi epi,
                         cudaStream_t st, char* err, size_t errlen, int* n_launch) {
   using C = TcCfg<BN, STAGES>;
-  cudaError_t e = set_smem_once(k_tc_gemm<BN, STAGES, Epi>, C::SMEM);
+  const int smem = LNB ? C::STAGES * C::A_BYTES + a.b_kb * C::B_BYTES + 1024 + 256 + 8 * BN * 4
+                       : C::SMEM;
+  cudaError_t e = set_smem_once(k_tc_gemm<BN, STAGES, LNB, Epi>, LNB ? 227 * 1024 : C::SMEM);
   if (e == cudaSuccess)
-    e = launch_pdl(k_tc_gemm<BN, STAGES, Epi>, dim3(grid), dim3(TC_THREADS), C::SMEM, st, wm.map,
+    e = launch_pdl(k_tc_gemm<BN, STAGES, LNB, Epi>, dim3(grid), dim3(TC_THREADS), smem, st, wm.map,
                    mapA, a, epi);
   if (e != cudaSuccess) {
     snprintf(err, errlen, "tensor-core GEMM launch: %s", cudaGetErrorString(e));
@@ -599,6 +685,8 @@ fm_status tc_launch(const TcMap& wm, const bf16* A, int lda, int M, Epi epi, flo
   a.partial = partial;
   a.tile_cnt = tile_cnt;
   a.err = err_word;
+  a.ln_x = a.ln_shift = a.ln_scale = nullptr;
+  a.b_kb = 0;
   CUtensorMap mapA;
   if (!tc_encode(&mapA, A, wm.Kd, M, lda, BN, err, errlen)) return FM_ERR_CUDA;
   const int grid = a.units < sms ? a.units : sms;
@@ -627,6 +715,65 @@ fm_status tc_gemm(const TcMaps& maps, const TcMap& wm, const bf16* A, int lda, i
     case 128: return tc_launch<128>(wm, A, lda, M, epi, partial, partial_elems, tile_cnt, tile_cnt_n, sms, maps.err, st, err, errlen, n_launch);
     default: return tc_launch<256>(wm, A, lda, M, epi, partial, partial_elems, tile_cnt, tile_cnt_n, sms, maps.err, st, err, errlen, n_launch);
   }
+}
+
+// y = (LN0(x) (1 + scale) + shift) . W^T with the normalisation done inside
+// the GEMM (no separate LayerNorm kernel, no bf16 activation round trip).
+// Needs M <= 32 (one activation tile) and every CTA's units sharing one
+// k-range; returns FM_ERR_UNSUPPORTED otherwise so the caller can fall back.
+template <int BN, class Epi>
+fm_status tc_launch_ln(const TcMap& wm, const float* x, const float* shift, const float* scale,
+                       int M, Epi epi, float* partial, size_t partial_elems, unsigned* tile_cnt,
+                       int tile_cnt_n, int sms, int* err_word, cudaStream_t st, char* err,
+                       size_t errlen, int* n_launch) {
+  TcArgs a;
+  a.M = M;
+  a.N = wm.N;
+  a.Kd = wm.Kd;
+  a.n_tiles = (wm.N + TC_BM - 1) / TC_BM;
+  a.m_tiles = 1;
+  a.k_blocks = (wm.Kd + TC_BK - 1) / TC_BK;
+  const int tiles = a.n_tiles;
+  int splits = 1;
+  if (tiles < sms) {
+    splits = sms / tiles;
+    splits = splits > a.k_blocks ? a.k_blocks : splits;
+    while (splits > 1 && (size_t)splits * tiles * TC_BM * BN > partial_elems) --splits;
+  }
+  if (splits > 1 && tiles > tile_cnt_n) splits = 1;
+  a.splits = splits < 1 ? 1 : splits;
+  a.units = tiles * a.splits;
+  a.partial = partial;
+  a.tile_cnt = tile_cnt;
+  a.err = err_word;
+  a.ln_x = x;
+  a.ln_shift = shift;
+  a.ln_scale = scale;
+  const int grid = a.units < sms ? a.units : sms;
+  if (a.units > grid && a.splits > 1) return FM_ERR_UNSUPPORTED;
+  a.b_kb = (a.units <= grid) ? (a.k_blocks + a.splits - 1) / a.splits : a.k_blocks;
+  const long per_cta = (long)((a.units + grid - 1) / grid) * ((a.k_blocks + a.splits - 1) / a.splits);
+  const bool deep = per_cta >= 24;
+  using CS = TcCfg<BN, 5>;
+  using CD = TcCfg<BN, 8>;
+  if ((deep ? 8 * CD::A_BYTES : 5 * CS::A_BYTES) + a.b_kb * CS::B_BYTES + 1280 + 8 * BN * 4 >
+      227 * 1024)
+    return FM_ERR_UNSUPPORTED;
+  if (deep)
+    return tc_launch_cfg<BN, 8, Epi, true>(wm, wm.map, a, grid, epi, st, err, errlen, n_launch);
+  return tc_launch_cfg<BN, 5, Epi, true>(wm, wm.map, a, grid, epi, st, err, errlen, n_launch);
+}
+
+template <class Epi>
+fm_status tc_gemm_ln(const TcMaps& maps, const TcMap& wm, const float* x, const float* shift,
+                     const float* scale, int M, Epi epi, float* partial, size_t partial_elems,
+                     unsigned* tile_cnt, int tile_cnt_n, int sms, cudaStream_t st, char* err,
+                     size_t errlen, int* n_launch) {
+  if (M <= 16)
+    return tc_launch_ln<16>(wm, x, shift, scale, M, epi, partial, partial_elems, tile_cnt, tile_cnt_n, sms, maps.err, st, err, errlen, n_launch);
+  if (M <= 32)
+    return tc_launch_ln<32>(wm, x, shift, scale, M, epi, partial, partial_elems, tile_cnt, tile_cnt_n, sms, maps.err, st, err, errlen, n_launch);
+  return FM_ERR_UNSUPPORTED;
 }
 
 inline fm_status tc_lm_head_argmax(const TcMaps& maps, const bf16* h, int lda, int M, int V,
