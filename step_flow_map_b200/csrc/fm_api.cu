@@ -83,6 +83,11 @@ struct fm_ctx {
   int tile_cnt_n = 0;
   float* c_raw = nullptr;
   void* c_norm = nullptr;
+  // context rows projected by fc + LN but whose keys/values are not yet in
+  // the cache: the next draft computes them inside its QKV GEMMs (same
+  // W_k, W_v), or they are flushed by separate GEMMs
+  int pending_rows = 0;
+  fm::RowMap pending_map;
   int v_chunks = 1;
   float* vg_pv = nullptr;
   int* vg_pi = nullptr;
@@ -95,6 +100,9 @@ struct fm_ctx {
   double* vs_ps = nullptr;
   double* vs_resid = nullptr;
   bool use_tc = false;
+  // LayerNorm inside the consuming GEMM (measured slower than a LayerNorm
+  // kernel followed by the GEMM at 16 rows; kept off)
+  bool ln_in_gemm = false;
   fm::TcMaps tc;  // tensor maps of the weight operands (tensor-core path)
   // launch counts and optional device timing per kernel class
   long long launches[FM_PROF_N] = {};
@@ -231,14 +239,15 @@ fm_status gemm_w(fm_ctx* c, int cls, const T* A, int lda, const T* W, int M, int
 // LayerNorm kernel instead.
 template <class Epi>
 fm_status gemm_ln(fm_ctx* c, int cls, const float* x, const float* shift, const float* scale,
-                  int M, Epi epi, cudaStream_t st, const fm::TcMap* map, bool* done) {
+                  int M, Epi epi, cudaStream_t st, const fm::TcMap* map, bool* done,
+                  const bf16* extra = nullptr, int n_extra = 0) {
   *done = false;
-  if (!c->use_tc || !map || !map->valid || M > 32) return FM_OK;
+  if (!c->use_tc || !map || !map->valid || M > 32 || !c->ln_in_gemm) return FM_OK;
   Prof prof(c, cls, st);
   int n_launch = 0;
-  fm_status s = fm::tc_gemm_ln(c->tc, *map, x, shift, scale, M, epi, c->splitk, c->splitk_elems,
-                               c->tile_cnt, c->tile_cnt_n, c->sms, st, g_err, sizeof(g_err),
-                               &n_launch);
+  fm_status s = fm::tc_gemm_ln(c->tc, *map, x, shift, scale, M, extra, M + n_extra, epi, c->splitk,
+                               c->splitk_elems, c->tile_cnt, c->tile_cnt_n, c->sms, st, g_err,
+                               sizeof(g_err), &n_launch);
   c->launches[cls] += n_launch;
   if (s == FM_ERR_UNSUPPORTED) return FM_OK;
   if (s == FM_OK) *done = true;
@@ -389,26 +398,14 @@ fm_status load_impl(fm_ctx* c, cudaStream_t st) {
 
 // ------------------------------------------------------------------ context projection
 template <typename T>
-fm_status project_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* hidden,
-                       int n_new, const int32_t* pos0, cudaStream_t st) {
+fm_status flush_pending(fm_ctx* c, cudaStream_t st) {
+  if (c->pending_rows == 0) return FM_OK;
   const fm_config& g = c->cfg;
-  const int d = g.d, R = n_seqs * n_new, in = g.n_taps * g.target_hidden;
-  FM_TRY(gemm_w<T>(c, FM_PROF_CONTEXT, (const T*)hidden, in, (const T*)c->w.W_fc, R, d, in,
-                   fm::EpiStoreF32{c->c_raw, d}, st, &c->tc.fc));
-  {
-    Prof prof(c, FM_PROF_CONTEXT, st);
-    FM_LAUNCH(c, FM_PROF_CONTEXT, (fm::k_adaln<float, T>), R, 256, 0, st,
-              c->c_raw, d, nullptr, nullptr, (T*)c->c_norm);
-  }
+  const int d = g.d, R = c->pending_rows;
   fm::EpiCtxKV<T> epi;
   epi.d = d;
   epi.max_ctx = g.max_ctx;
-  epi.map.n_seqs = n_seqs;
-  epi.map.n_new = n_new;
-  for (int q = 0; q < n_seqs; ++q) {
-    epi.map.slot[q] = seq_ids[q];
-    epi.map.pos0[q] = pos0[q];
-  }
+  epi.map = c->pending_map;
   for (int l = 0; l < g.n_blocks; ++l) {
     epi.Kc = (T*)c->Kc[l];
     epi.Vc = (T*)c->Vc[l];
@@ -416,6 +413,37 @@ fm_status project_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void
     FM_TRY(gemm_w<T>(c, FM_PROF_CONTEXT, (const T*)c->c_norm, d, Wkv, R, 2 * d, d, epi, st,
                      &c->tc.kv[l]));
   }
+  c->pending_rows = 0;
+  return FM_OK;
+}
+
+// Rows that a following one-step draft of at most this many block rows can
+// absorb into its QKV GEMMs (one 64-row activation tile).
+constexpr int FUSED_CTX_ROWS = 64;
+
+template <typename T>
+fm_status project_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* hidden,
+                       int n_new, const int32_t* pos0, cudaStream_t st) {
+  const fm_config& g = c->cfg;
+  const int d = g.d, R = n_seqs * n_new, in = g.n_taps * g.target_hidden;
+  FM_TRY(flush_pending<T>(c, st));   // c_norm is about to be overwritten
+  FM_TRY(gemm_w<T>(c, FM_PROF_CONTEXT, (const T*)hidden, in, (const T*)c->w.W_fc, R, d, in,
+                   fm::EpiStoreF32{c->c_raw, d}, st, &c->tc.fc));
+  {
+    Prof prof(c, FM_PROF_CONTEXT, st);
+    FM_LAUNCH(c, FM_PROF_CONTEXT, (fm::k_adaln<float, T>), R, 256, 0, st,
+              c->c_raw, d, nullptr, nullptr, (T*)c->c_norm);
+  }
+  c->pending_map.n_seqs = n_seqs;
+  c->pending_map.n_new = n_new;
+  for (int q = 0; q < n_seqs; ++q) {
+    c->pending_map.slot[q] = seq_ids[q];
+    c->pending_map.pos0[q] = pos0[q];
+  }
+  c->pending_rows = R;
+  // keys/values now unless a small draft can take them over
+  if (!(sizeof(T) == 2 && c->use_tc && c->ln_in_gemm && R < FUSED_CTX_ROWS))
+    FM_TRY(flush_pending<T>(c, st));
   for (int q = 0; q < n_seqs; ++q) c->ctx_len[seq_ids[q]] = pos0[q] + n_new;
   return FM_OK;
 }
@@ -508,6 +536,16 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
     any_sample |= temps[q] > 0.f;
   }
   float* logits = draft_logits ? draft_logits : c->logits;
+  // context rows whose keys/values are still pending: the first step's QKV
+  // GEMMs compute them when the rows fit one activation tile, else now
+  bool fuse_ctx = false;
+  if (c->pending_rows > 0) {
+    if (sizeof(T) == 2 && c->use_tc && c->ln_in_gemm && M <= 32 &&
+        M + c->pending_rows <= FUSED_CTX_ROWS)
+      fuse_ctx = true;
+    else
+      FM_TRY(flush_pending<T>(c, st));
+  }
   for (int k = 0; k < num_steps; ++k) {
     const float s = t_grid[k], t = t_grid[k + 1];
     const bool last = (k == num_steps - 1);
@@ -532,8 +570,31 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
     for (int l = 0; l < nb; ++l) {
       const float* ml = mods + (size_t)l * 6 * d;
       bool fused = false;
-      FM_TRY(gemm_ln(c, FM_PROF_DIT_GEMM, c->x, ml, ml + d, M, fm::EpiStore<T>{qkv, 3 * d}, st,
-                     &c->tc.qkv[l], &fused));
+      if constexpr (sizeof(T) == 2) {
+        if (fuse_ctx) {
+          // this step's QKV GEMM also projects the pending context rows
+          fm::EpiQkvCtx<T> e;
+          e.qkv = qkv;
+          e.ld = 3 * d;
+          e.M_draft = M;
+          e.d = d;
+          e.kv.Kc = (T*)c->Kc[l];
+          e.kv.Vc = (T*)c->Vc[l];
+          e.kv.d = d;
+          e.kv.max_ctx = g.max_ctx;
+          e.kv.map = c->pending_map;
+          FM_TRY(gemm_ln(c, FM_PROF_DIT_GEMM, c->x, ml, ml + d, M, e, st, &c->tc.qkv[l], &fused,
+                         (const bf16*)c->c_norm, c->pending_rows));
+          if (!fused) {
+            if (l > 0) return set_err(FM_ERR_CUDA, "fused context projection stopped at block %d", l);
+            fuse_ctx = false;
+            FM_TRY(flush_pending<T>(c, st));
+          }
+        }
+      }
+      if (!fused)
+        FM_TRY(gemm_ln(c, FM_PROF_DIT_GEMM, c->x, ml, ml + d, M, fm::EpiStore<T>{qkv, 3 * d}, st,
+                       &c->tc.qkv[l], &fused));
       if (!fused) {
         {
           Prof prof(c, FM_PROF_NORM, st);
@@ -569,6 +630,10 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
       }
       FM_TRY(gemm_w<T>(c, FM_PROF_DIT_GEMM, u, F, (const T*)c->wdown[l], M, d, F,
                        fm::EpiResidual{c->x, ml + 5 * d, d}, st, &c->tc.down[l]));
+    }
+    if (fuse_ctx) {
+      c->pending_rows = 0;
+      fuse_ctx = false;
     }
     const float* mf = mods + (size_t)nb * 6 * d;
     // LM head: greedy-only final steps keep the logits on chip when possible

@@ -87,6 +87,20 @@ struct EpiCtxKV {
   }
 };
 
+// QKV of the block rows plus, in the same GEMM, the keys and values of
+// context rows appended after them (rows >= M_draft; their query columns
+// are not needed and are dropped).
+template <typename TO>
+struct EpiQkvCtx {
+  TO* qkv;
+  int ld, M_draft, d;
+  EpiCtxKV<TO> kv;
+  __device__ __forceinline__ void operator()(int m, int n, float v) const {
+    if (m < M_draft) qkv[(size_t)m * ld + n] = from_f<TO>(v);
+    else if (n >= d) kv(m - M_draft, n - d, v);
+  }
+};
+
 // ------------------------------------------------------------------ SIMT GEMM
 // Y[m][n] = sum_k A[m][k] * W(n,k), W(n,k) = W[n*ldw+k] (WK) or W[k*ldw+n].
 // Tile 32 x 64 x 16, 256 threads, 2 x 4 outputs per thread.  With

@@ -183,9 +183,11 @@ struct TcArgs {
   unsigned* tile_cnt;   // [tiles], zero between launches
   int* err;
   // B operand computed in the kernel as LN0(x) (1 + scale) + shift (bf16)
-  const float* ln_x;    // [M][Kd] fp32
+  const float* ln_x;    // [M_ln][Kd] fp32
   const float* ln_shift;
   const float* ln_scale;
+  int M_ln;             // rows [0, M_ln) come from x; rows [M_ln, M) are copied from ln_extra
+  const bf16* ln_extra; // [M - M_ln][Kd] bf16, already normalised
   int b_kb;             // k-blocks of the shared-memory-resident B operand
 };
 
@@ -240,35 +242,37 @@ __device__ __forceinline__ void tc_finish_chunk(const Epi& epi, const TcArgs& a,
 // Modulated LayerNorm of the activation rows, written straight into the
 // shared-memory B operand (128-byte swizzle, K-major, one BN x 64 tile per
 // k-block) by the 128 epilogue threads before any accumulator is ready.
-// Rows past M are zero.  Row statistics in fp32, two passes.
+// Rows [0, M_ln) are LN0(x)(1 + scale) + shift with fp32 statistics (two
+// passes, eight threads per row); rows [M_ln, M) are copied from ln_extra;
+// rows past M are zero.
 template <int BN>
 __device__ __forceinline__ void tc_ln_fill(uint8_t* sB, const TcArgs& a, int kb0, int nkb, int et,
                                            float* s_stat) {
-  constexpr int TPR = 128 / BN;  // threads per row, consecutive lanes
   const int Kd = a.Kd;
-  {
-    const int row = et / TPR, part = et % TPR;
-    const bool valid = row < a.M;
+  const int part = et & 7;
+  for (int r0 = 0; r0 < a.M_ln; r0 += 16) {
+    const int row = r0 + (et >> 3);
+    const bool valid = row < a.M_ln;
     const float* xr = a.ln_x + (size_t)row * Kd;
     float s = 0.f;
     if (valid)
-      for (int c = part * 4; c < Kd; c += TPR * 4) {
+      for (int c = part * 4; c < Kd; c += 32) {
         const float4 v = *(const float4*)(xr + c);
         s += (v.x + v.y) + (v.z + v.w);
       }
 #pragma unroll
-    for (int o = 1; o < TPR; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    for (int o = 1; o < 8; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     const float mean = s / (float)Kd;
     float q = 0.f;
     if (valid)
-      for (int c = part * 4; c < Kd; c += TPR * 4) {
+      for (int c = part * 4; c < Kd; c += 32) {
         const float4 v = *(const float4*)(xr + c);
         const float a0 = v.x - mean, a1 = v.y - mean, a2 = v.z - mean, a3 = v.w - mean;
         q += (a0 * a0 + a1 * a1) + (a2 * a2 + a3 * a3);
       }
 #pragma unroll
-    for (int o = 1; o < TPR; o <<= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
-    if (part == 0) {
+    for (int o = 1; o < 8; o <<= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+    if (part == 0 && valid) {
       s_stat[row] = mean;
       s_stat[BN + row] = rsqrtf(q / (float)Kd + 1e-6f);
     }
@@ -280,16 +284,20 @@ __device__ __forceinline__ void tc_ln_fill(uint8_t* sB, const TcArgs& a, int kb0
     const int row = rem >> 3, ch = rem & 7;
     const int col = (kb0 + kbi) * TC_BK + ch * 8;
     uint4 packed = make_uint4(0, 0, 0, 0);
-    if (row < a.M && col < Kd) {
-      const float mean = s_stat[row], rstd = s_stat[BN + row];
-      const float* xr = a.ln_x + (size_t)row * Kd + col;
-      const float4 x0 = *(const float4*)xr, x1 = *(const float4*)(xr + 4);
-      const float4 c0 = *(const float4*)(a.ln_scale + col), c1 = *(const float4*)(a.ln_scale + col + 4);
-      const float4 h0 = *(const float4*)(a.ln_shift + col), h1 = *(const float4*)(a.ln_shift + col + 4);
-      packed.x = pack_bf16x2((x0.x - mean) * rstd * (1.f + c0.x) + h0.x, (x0.y - mean) * rstd * (1.f + c0.y) + h0.y);
-      packed.y = pack_bf16x2((x0.z - mean) * rstd * (1.f + c0.z) + h0.z, (x0.w - mean) * rstd * (1.f + c0.w) + h0.w);
-      packed.z = pack_bf16x2((x1.x - mean) * rstd * (1.f + c1.x) + h1.x, (x1.y - mean) * rstd * (1.f + c1.y) + h1.y);
-      packed.w = pack_bf16x2((x1.z - mean) * rstd * (1.f + c1.z) + h1.z, (x1.w - mean) * rstd * (1.f + c1.w) + h1.w);
+    if (col < Kd) {
+      if (row < a.M_ln) {
+        const float mean = s_stat[row], rstd = s_stat[BN + row];
+        const float* xr = a.ln_x + (size_t)row * Kd + col;
+        const float4 x0 = *(const float4*)xr, x1 = *(const float4*)(xr + 4);
+        const float4 c0 = *(const float4*)(a.ln_scale + col), c1 = *(const float4*)(a.ln_scale + col + 4);
+        const float4 h0 = *(const float4*)(a.ln_shift + col), h1 = *(const float4*)(a.ln_shift + col + 4);
+        packed.x = pack_bf16x2((x0.x - mean) * rstd * (1.f + c0.x) + h0.x, (x0.y - mean) * rstd * (1.f + c0.y) + h0.y);
+        packed.y = pack_bf16x2((x0.z - mean) * rstd * (1.f + c0.z) + h0.z, (x0.w - mean) * rstd * (1.f + c0.w) + h0.w);
+        packed.z = pack_bf16x2((x1.x - mean) * rstd * (1.f + c1.x) + h1.x, (x1.y - mean) * rstd * (1.f + c1.y) + h1.y);
+        packed.w = pack_bf16x2((x1.z - mean) * rstd * (1.f + c1.z) + h1.z, (x1.w - mean) * rstd * (1.f + c1.w) + h1.w);
+      } else if (row < a.M) {
+        packed = *(const uint4*)(a.ln_extra + (size_t)(row - a.M_ln) * Kd + col);
+      }
     }
     *(uint4*)(sB + kbi * B_BYTES + row * 128 + ((ch ^ (row & 7)) << 4)) = packed;
   }
@@ -686,6 +694,8 @@ fm_status tc_launch(const TcMap& wm, const bf16* A, int lda, int M, Epi epi, flo
   a.tile_cnt = tile_cnt;
   a.err = err_word;
   a.ln_x = a.ln_shift = a.ln_scale = nullptr;
+  a.M_ln = 0;
+  a.ln_extra = nullptr;
   a.b_kb = 0;
   CUtensorMap mapA;
   if (!tc_encode(&mapA, A, wm.Kd, M, lda, BN, err, errlen)) return FM_ERR_CUDA;
@@ -723,11 +733,13 @@ fm_status tc_gemm(const TcMaps& maps, const TcMap& wm, const bf16* A, int lda, i
 // k-range; returns FM_ERR_UNSUPPORTED otherwise so the caller can fall back.
 template <int BN, class Epi>
 fm_status tc_launch_ln(const TcMap& wm, const float* x, const float* shift, const float* scale,
-                       int M, Epi epi, float* partial, size_t partial_elems, unsigned* tile_cnt,
-                       int tile_cnt_n, int sms, int* err_word, cudaStream_t st, char* err,
-                       size_t errlen, int* n_launch) {
+                       int M_ln, const bf16* extra, int M, Epi epi, float* partial,
+                       size_t partial_elems, unsigned* tile_cnt, int tile_cnt_n, int sms,
+                       int* err_word, cudaStream_t st, char* err, size_t errlen, int* n_launch) {
   TcArgs a;
   a.M = M;
+  a.M_ln = M_ln;
+  a.ln_extra = extra;
   a.N = wm.N;
   a.Kd = wm.Kd;
   a.n_tiles = (wm.N + TC_BM - 1) / TC_BM;
@@ -764,15 +776,20 @@ fm_status tc_launch_ln(const TcMap& wm, const float* x, const float* shift, cons
   return tc_launch_cfg<BN, 5, Epi, true>(wm, wm.map, a, grid, epi, st, err, errlen, n_launch);
 }
 
+// Rows [0, M_ln) are LN(x) rows; rows [M_ln, M) come from `extra` (bf16,
+// normalised context rows riding along in the same GEMM).
 template <class Epi>
 fm_status tc_gemm_ln(const TcMaps& maps, const TcMap& wm, const float* x, const float* shift,
-                     const float* scale, int M, Epi epi, float* partial, size_t partial_elems,
-                     unsigned* tile_cnt, int tile_cnt_n, int sms, cudaStream_t st, char* err,
-                     size_t errlen, int* n_launch) {
+                     const float* scale, int M_ln, const bf16* extra, int M, Epi epi,
+                     float* partial, size_t partial_elems, unsigned* tile_cnt, int tile_cnt_n,
+                     int sms, cudaStream_t st, char* err, size_t errlen, int* n_launch) {
+  if (M_ln > 32 || M < M_ln || (M > M_ln && !extra)) return FM_ERR_UNSUPPORTED;
   if (M <= 16)
-    return tc_launch_ln<16>(wm, x, shift, scale, M, epi, partial, partial_elems, tile_cnt, tile_cnt_n, sms, maps.err, st, err, errlen, n_launch);
+    return tc_launch_ln<16>(wm, x, shift, scale, M_ln, extra, M, epi, partial, partial_elems, tile_cnt, tile_cnt_n, sms, maps.err, st, err, errlen, n_launch);
   if (M <= 32)
-    return tc_launch_ln<32>(wm, x, shift, scale, M, epi, partial, partial_elems, tile_cnt, tile_cnt_n, sms, maps.err, st, err, errlen, n_launch);
+    return tc_launch_ln<32>(wm, x, shift, scale, M_ln, extra, M, epi, partial, partial_elems, tile_cnt, tile_cnt_n, sms, maps.err, st, err, errlen, n_launch);
+  if (M <= 64)
+    return tc_launch_ln<64>(wm, x, shift, scale, M_ln, extra, M, epi, partial, partial_elems, tile_cnt, tile_cnt_n, sms, maps.err, st, err, errlen, n_launch);
   return FM_ERR_UNSUPPORTED;
 }
 
