@@ -14,6 +14,7 @@
 #include "fm_verify.cuh"
 #include "fm_tc.cuh"
 #include "fm_attn.cuh"
+#include "fm_dit.cuh"
 
 using fm::bf16;
 
@@ -92,6 +93,11 @@ struct fm_ctx {
   float* vg_pv = nullptr;
   int* vg_pi = nullptr;
   unsigned* vg_cnt = nullptr;
+  unsigned* dit_bar = nullptr;   // persistent DiT pass: grid barrier counter, abort flag,
+  int* dit_abort = nullptr;      //   LayerNorm tile statistics, final LayerNorm output
+  float* dit_stats = nullptr;
+  void* dit_hf = nullptr;
+  bool dit_ok = false;           // the persistent pass fits this configuration and device
   float* attn_part = nullptr;   // split-KV attention partials
   unsigned* attn_cnt = nullptr;
   size_t attn_part_elems = 0;
@@ -362,6 +368,10 @@ fm_status load_impl(fm_ctx* c, cudaStream_t st) {
   FM_TRY(dalloc_t(c, &c->attn_part, c->attn_part_elems));
   FM_TRY(dalloc_t(c, &c->attn_cnt, (size_t)c->attn_pairs_max));
   FM_CUDA(cudaMemsetAsync(c->attn_cnt, 0, c->attn_pairs_max * sizeof(unsigned), st));
+  FM_TRY(dalloc_t(c, &c->dit_bar, 1));
+  FM_TRY(dalloc_t(c, &c->dit_abort, 1));
+  FM_TRY(dalloc_t(c, &c->dit_stats, (size_t)(d / 128 + 1) * fm::DIT_M * 2));
+  FM_TRY(dalloc(c, &c->dit_hf, (size_t)fm::DIT_M * d * sizeof(T)));
   FM_TRY(dalloc_t(c, &c->c_raw, (size_t)c->R_max * d));
   FM_TRY(dalloc(c, &c->c_norm, (size_t)c->R_max * d * sizeof(T)));
   // verify workspaces: rows = B*N*(K+1) target + B*N*K draft rows
@@ -384,6 +394,21 @@ fm_status load_impl(fm_ctx* c, cudaStream_t st) {
                             c->wup.data(), c->wdown.data(), g.n_blocks, g.d, g.mlp, g.V,
                             g.n_taps * g.target_hidden, g_err, sizeof(g_err)))
         return FM_ERR_CUDA;
+    }
+  }
+  if constexpr (sizeof(T) == 2) {
+    int coop = 0;
+    cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, c->dev);
+    const char* off = getenv("FM_DISABLE_PERSISTENT");  // diagnostic: per-kernel DiT path
+    c->dit_ok = c->use_tc && coop && !(off && *off == '1') && g.n_blocks <= fm::DIT_MAX_BLOCKS &&
+                d / g.n_heads == fm::AM_DH && g.K == fm::DIT_M && d % 128 == 0 && g.mlp % 128 == 0 &&
+                d / 128 <= c->sms;
+    if (c->dit_ok) {
+      FM_CUDA(fm::set_smem_once(fm::k_dit_persistent, fm::DIT_SMEM));
+      int per_sm = 0;
+      FM_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fm::k_dit_persistent,
+                                                            fm::TC_THREADS, fm::DIT_SMEM));
+      c->dit_ok = per_sm >= 1;
     }
   }
   // the grids every draft uses
@@ -481,6 +506,100 @@ fm_status attn_mma(fm_ctx* c, int n_noise, fm::AttnMmaArgs am, const bf16* qkv, 
   }
 }
 
+// ------------------------------------------------------------------ persistent DiT pass
+// One cooperative launch for all blocks of one 16-row draft (one sequence,
+// one noise draft); leaves the final modulated LayerNorm in c->dit_hf.
+// Returns FM_ERR_UNSUPPORTED (nothing launched) when a limit does not hold.
+fm_status dit_persistent(fm_ctx* c, const float* mods, int slot, int ctx_len, bool with_ctx,
+                         cudaStream_t st) {
+  const fm_config& g = c->cfg;
+  const int d = g.d, G = c->sms;
+  fm::DitParams P;
+  memset(&P, 0, sizeof(P));
+  for (int l = 0; l < g.n_blocks; ++l) {
+    P.w[l][0] = c->tc.qkv[l].map;
+    P.w[l][1] = c->tc.o[l].map;
+    P.w[l][2] = c->tc.up[l].map;
+    P.w[l][3] = c->tc.down[l].map;
+    P.Kc[l] = (bf16*)c->Kc[l];
+    P.Vc[l] = (bf16*)c->Vc[l];
+  }
+  P.n_blocks = g.n_blocks;
+  P.d = d;
+  P.F = g.mlp;
+  P.M = fm::DIT_M;
+  // K splits per GEMM kind: about one unit per SM
+  const int tiles[5] = {3 * d / 128, 0, d / 128, g.mlp / 128, d / 128};
+  const int kbs[5] = {d / 64, 0, d / 64, d / 64, g.mlp / 64};
+  for (int k : {fm::DIT_QKV, fm::DIT_O, fm::DIT_UP, fm::DIT_DOWN}) {
+    if (tiles[k] > G) return FM_ERR_UNSUPPORTED;
+    P.splits[k] = std::max(1, std::min(G / tiles[k], kbs[k]));
+  }
+  P.x = c->x;
+  P.stats = c->dit_stats;
+  P.partial = c->splitk;
+  P.tile_cnt = c->tile_cnt;
+  P.bar = c->dit_bar;
+  P.err = c->tc.err;
+  P.abort_g = c->dit_abort;
+  P.qkv = (bf16*)c->qkv;
+  P.o = (bf16*)c->o;
+  P.u = (bf16*)c->u;
+  P.hf = (bf16*)c->dit_hf;
+  P.mods = mods;
+  P.max_ctx = g.max_ctx;
+  P.n_ctx = 0;
+  if (with_ctx && c->pending_rows > 0) {
+    P.n_ctx = c->pending_rows;
+    P.ctx_rows = (const bf16*)c->c_norm;
+    P.ctx_map = c->pending_map;
+  }
+  if (fm::DIT_M + P.n_ctx > fm::DIT_BROWS_MAX) return FM_ERR_UNSUPPORTED;
+  // shared-memory and workspace limits of every phase
+  for (int k : {fm::DIT_QKV, fm::DIT_O, fm::DIT_UP, fm::DIT_DOWN}) {
+    const int brows = (k == fm::DIT_QKV && P.n_ctx) ? (fm::DIT_M + P.n_ctx + 15) / 16 * 16 : 16;
+    const int nkb = (kbs[k] + P.splits[k] - 1) / P.splits[k];
+    if ((size_t)nkb * brows * 128 > (size_t)fm::DIT_UNION) return FM_ERR_UNSUPPORTED;
+    if ((size_t)P.splits[k] * tiles[k] * 128 * brows > c->splitk_elems) return FM_ERR_UNSUPPORTED;
+  }
+  fm::AttnMmaArgs& am = P.attn;
+  am.n_seqs = 1;
+  am.n_noise = 1;
+  am.K = g.K;
+  am.d = d;
+  am.n_heads = g.n_heads;
+  am.max_ctx = g.max_ctx;
+  am.scale_log2 = (float)(1.4426950408889634 / sqrt((double)fm::AM_DH));
+  am.part = c->attn_part;
+  am.cnt = c->attn_cnt;
+  am.slot[0] = slot;
+  am.len[0] = ctx_len;
+  int s_ctx = G / g.n_heads - 1;
+  s_ctx = std::min(s_ctx, (ctx_len + fm::AM_CHUNK - 1) / fm::AM_CHUNK);
+  s_ctx = std::max(s_ctx, 1);
+  if (g.n_heads * (s_ctx + 1) > G) return FM_ERR_UNSUPPORTED;
+  if ((size_t)g.n_heads * (s_ctx + 1) * 16 * fm::AM_PSTRIDE > c->attn_part_elems)
+    return FM_ERR_UNSUPPORTED;
+  am.n_ctx_splits = s_ctx;
+  P.splits[fm::DIT_ATTN] = s_ctx;
+  FM_CUDA(cudaMemsetAsync(c->dit_bar, 0, sizeof(unsigned), st));
+  FM_CUDA(cudaMemsetAsync(c->dit_abort, 0, sizeof(int), st));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(G);
+  cfg.blockDim = dim3(fm::TC_THREADS);
+  cfg.dynamicSmemBytes = fm::DIT_SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  FM_CUDA(cudaLaunchKernelEx(&cfg, fm::k_dit_persistent, P));
+  c->launches[FM_PROF_DIT_GEMM]++;
+  if (P.n_ctx) c->pending_rows = 0;
+  return FM_OK;
+}
+
 // ------------------------------------------------------------------ draft
 template <typename T>
 fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* noise,
@@ -539,11 +658,12 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
   // context rows whose keys/values are still pending: the first step's QKV
   // GEMMs compute them when the rows fit one activation tile, else now
   bool fuse_ctx = false;
+  const bool will_persist = sizeof(T) == 2 && c->dit_ok && M == fm::DIT_M && n_seqs == 1;
   if (c->pending_rows > 0) {
     if (sizeof(T) == 2 && c->use_tc && c->ln_in_gemm && M <= 32 &&
         M + c->pending_rows <= FUSED_CTX_ROWS)
       fuse_ctx = true;
-    else
+    else if (!will_persist)   // the persistent pass takes them over
       FM_TRY(flush_pending<T>(c, st));
   }
   for (int k = 0; k < num_steps; ++k) {
@@ -567,7 +687,17 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
       FM_TRY((gemm_simt<T, T, fm::EpiEmbed>(c, FM_PROF_EMBED, A, V, (const T*)c->w.E, d, false, M,
                                              d, V, emb, st)));
     }
-    for (int l = 0; l < nb; ++l) {
+    bool persistent = false;
+    if constexpr (sizeof(T) == 2) {
+      if (will_persist) {
+        Prof prof(c, FM_PROF_DIT_GEMM, st);
+        fm_status ps = dit_persistent(c, mods, seq_ids[0], c->ctx_len[seq_ids[0]], k == 0, st);
+        if (ps == FM_OK) persistent = true;
+        else if (ps != FM_ERR_UNSUPPORTED) return ps;
+      }
+    }
+    if (!persistent && c->pending_rows > 0 && !fuse_ctx) FM_TRY(flush_pending<T>(c, st));
+    for (int l = 0; l < nb && !persistent; ++l) {
       const float* ml = mods + (size_t)l * 6 * d;
       bool fused = false;
       if constexpr (sizeof(T) == 2) {
@@ -639,7 +769,20 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
     // LM head: greedy-only final steps keep the logits on chip when possible
     const bool need_logits = !last || any_sample || draft_logits != nullptr;
     bool have_partials = false, fused = false;
-    if (need_logits) {
+    if (persistent) {
+      fused = true;
+      if (need_logits) {
+        FM_TRY(gemm_w<T>(c, FM_PROF_LM_HEAD, (const T*)c->dit_hf, d, (const T*)c->w.W_lm, M, V, d,
+                         fm::EpiStoreF32{logits, V}, st, &c->tc.lm));
+      } else {
+        Prof prof(c, FM_PROF_LM_HEAD, st);
+        int n_launch = 0;
+        FM_TRY(fm::tc_lm_head_argmax(c->tc, (const bf16*)c->dit_hf, d, M, V, c->part_v, c->part_i,
+                                     c->n_part, c->sms, st, g_err, sizeof(g_err), &n_launch));
+        c->launches[FM_PROF_LM_HEAD] += n_launch;
+        have_partials = true;
+      }
+    } else if (need_logits) {
       FM_TRY(gemm_ln(c, FM_PROF_LM_HEAD, c->x, mf, mf + d, M, fm::EpiStoreF32{logits, V}, st,
                      &c->tc.lm, &fused));
     } else {

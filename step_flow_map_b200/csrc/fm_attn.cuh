@@ -152,9 +152,11 @@ __device__ __forceinline__ void attn_block(AttnState& st, const uint32_t (&qa)[8
 }
 
 // Loads rows [r0, r0+nr) of a [rows][ld] bf16 matrix (dh columns from col0)
-// into smem [nr][AM_LD]; rows past nr up to `pad_to` are zero-filled.
-__device__ __forceinline__ void load_rows(bf16* dst, const bf16* src, size_t ld, int nr, int pad_to) {
-  for (int e = threadIdx.x; e < pad_to * (AM_DH / 8); e += blockDim.x) {
+// into smem [nr][AM_LD]; rows past nr up to `pad_to` are zero-filled.  Run by
+// the AM_THREADS threads of an attention work item (tid 0..AM_THREADS-1).
+__device__ __forceinline__ void load_rows(bf16* dst, const bf16* src, size_t ld, int nr, int pad_to,
+                                          int tid) {
+  for (int e = tid; e < pad_to * (AM_DH / 8); e += AM_THREADS) {
     const int r = e / (AM_DH / 8), c8 = (e % (AM_DH / 8)) * 8;
     bf16* dp = dst + r * AM_LD + c8;
     if (r < nr) cp_async16((uint32_t)__cvta_generic_to_shared(dp), src + (size_t)r * ld + c8);
@@ -162,28 +164,29 @@ __device__ __forceinline__ void load_rows(bf16* dst, const bf16* src, size_t ld,
   }
 }
 
-template <int N>
-__global__ void __launch_bounds__(AM_THREADS)
-k_attn_mma(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc, const bf16* __restrict__ Vc,
-           bf16* __restrict__ out, AttnMmaArgs a) {
-  pdl_wait();
-  pdl_trigger();
-  extern __shared__ __align__(16) uint8_t smem_raw[];
+// One work item -- (sequence, head) pair `pair`, split `split` -- run by
+// AM_THREADS threads (tid 0..AM_THREADS-1, four whole warps) that
+// synchronise with `sync()`.  `smem_raw` holds attn_mma_smem<N>() bytes;
+// `s_last` is one shared int.
+template <int N, class Sync>
+__device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc,
+                                          const bf16* __restrict__ Vc, bf16* __restrict__ out,
+                                          const AttnMmaArgs& a, int pair, int split,
+                                          uint8_t* smem_raw, int* s_last_p, int tid, Sync sync) {
   bf16* sQ = (bf16*)smem_raw;                       // [N*16][AM_LD]
   bf16* sK = sQ + N * 16 * AM_LD;                   // [AM_STAGES][AM_CHUNK][AM_LD]
   bf16* sV = sK + AM_STAGES * AM_CHUNK * AM_LD;     // [AM_STAGES][AM_CHUNK][AM_LD]
-  __shared__ int s_last;
+  int& s_last = *s_last_p;
   constexpr int WPM = 4 / N;                        // warps sharing one 16-query tile
-  const int pair = blockIdx.x, split = blockIdx.y;
   const int b = pair / a.n_heads, h = pair - b * a.n_heads;
-  const int d3 = 3 * a.d, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int d3 = 3 * a.d, warp = tid >> 5, lane = tid & 31;
   const int mt = warp % N, sub = warp / N;          // query tile, key sub-slice
   const int row0 = b * a.n_noise * a.K;             // first block row of the sequence
   const int S_all = a.n_ctx_splits + 1;
   const int NQ = N * 16;
 
   // queries of all drafts of the sequence
-  load_rows(sQ, qkv + (size_t)row0 * d3 + h * AM_DH, d3, NQ, NQ);
+  load_rows(sQ, qkv + (size_t)row0 * d3 + h * AM_DH, d3, NQ, NQ, tid);
   cp_commit();
 
   AttnState st;
@@ -211,8 +214,8 @@ k_attn_mma(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc, const bf16
     auto load_chunk = [&](int c) {
       const int r0 = k0 + c * AM_CHUNK, nr = min(AM_CHUNK, k1 - r0);
       const int buf = c % AM_STAGES;
-      load_rows(sK + buf * AM_CHUNK * AM_LD, Kc + base + (size_t)r0 * a.d, a.d, nr, AM_CHUNK);
-      load_rows(sV + buf * AM_CHUNK * AM_LD, Vc + base + (size_t)r0 * a.d, a.d, nr, AM_CHUNK);
+      load_rows(sK + buf * AM_CHUNK * AM_LD, Kc + base + (size_t)r0 * a.d, a.d, nr, AM_CHUNK, tid);
+      load_rows(sV + buf * AM_CHUNK * AM_LD, Vc + base + (size_t)r0 * a.d, a.d, nr, AM_CHUNK, tid);
     };
     // one commit group per chunk (empty past the end) keeps the group count
     // fixed: AM_STAGES - 1 chunks are always in flight ahead of the one used
@@ -222,13 +225,13 @@ k_attn_mma(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc, const bf16
       cp_commit();
     }
     cp_wait<AM_STAGES - 1>();   // the query group
-    __syncthreads();
+    sync();
     q_fragments();
     for (int c = 0; c < n_chunks; ++c) {
       if (c + AM_STAGES - 1 < n_chunks) load_chunk(c + AM_STAGES - 1);
       cp_commit();
       cp_wait<AM_STAGES - 1>();
-      __syncthreads();
+      sync();
       const int buf = c % AM_STAGES;
       const int nk_chunk = min(AM_CHUNK, k1 - (k0 + c * AM_CHUNK));
       constexpr int KW = AM_CHUNK / WPM;            // keys of this warp within the chunk
@@ -237,7 +240,7 @@ k_attn_mma(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc, const bf16
       const bf16* ks = sK + buf * AM_CHUNK * AM_LD + kw0 * AM_LD;
       const bf16* vs = sV + buf * AM_CHUNK * AM_LD + kw0 * AM_LD;
       if (nk > 0) attn_block<KW / 8>(st, qa, ks, vs, nk, a.scale_log2);
-      __syncthreads();
+      sync();
     }
   } else {
     // each draft's own block rows: keys/values of rows row0 + mt*16 .. +16
@@ -255,10 +258,10 @@ k_attn_mma(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc, const bf16
     }
     cp_commit();
     cp_wait<0>();
-    __syncthreads();
+    sync();
     q_fragments();
     if (sub == 0) attn_block<2>(st, qa, sK + mt * 16 * AM_LD, sV + mt * 16 * AM_LD, 16, a.scale_log2);
-    __syncthreads();
+    sync();
   }
 
   // ---- merge the warps of each query tile in smem, write this split's partial
@@ -286,9 +289,9 @@ k_attn_mma(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc, const bf16
     wo[(g + 8) * (AM_DH + 2) + AM_DH] = st.m[1];
     wo[(g + 8) * (AM_DH + 2) + AM_DH + 1] = l_tot[1];
   }
-  __syncthreads();
+  sync();
   float* part = a.part + ((size_t)pair * S_all + split) * NQ * AM_PSTRIDE;
-  for (int e = threadIdx.x; e < NQ * AM_DH; e += blockDim.x) {
+  for (int e = tid; e < NQ * AM_DH; e += AM_THREADS) {
     const int q = e / AM_DH, c = e % AM_DH;
     const int tile = q / 16, rr = q % 16;
     float M = -INFINITY;
@@ -307,9 +310,9 @@ k_attn_mma(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc, const bf16
     }
   }
   __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) s_last = (atomicAdd(&a.cnt[pair], 1u) == (unsigned)(S_all - 1));
-  __syncthreads();
+  sync();
+  if (tid == 0) s_last = (atomicAdd(&a.cnt[pair], 1u) == (unsigned)(S_all - 1));
+  sync();
   if (!s_last) return;
   __threadfence();
   // ---- last CTA of this (sequence, head): merge the splits in split order,
@@ -354,7 +357,19 @@ k_attn_mma(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc, const bf16
     dst[0] = __floats2bfloat162_rn(o.x * inv, o.y * inv);
     dst[1] = __floats2bfloat162_rn(o.z * inv, o.w * inv);
   }
-  if (threadIdx.x == 0) a.cnt[pair] = 0u;
+  if (tid == 0) a.cnt[pair] = 0u;
+}
+
+template <int N>
+__global__ void __launch_bounds__(AM_THREADS)
+k_attn_mma(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc, const bf16* __restrict__ Vc,
+           bf16* __restrict__ out, AttnMmaArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  __shared__ int s_last;
+  attn_item<N>(qkv, Kc, Vc, out, a, blockIdx.x, blockIdx.y, smem_raw, &s_last, threadIdx.x,
+               [] __device__() { __syncthreads(); });
 }
 
 template <int N>

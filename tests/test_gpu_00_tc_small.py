@@ -30,13 +30,16 @@ def _workload(B, N, t_grid=(0.0, 1.0), temps=None, ctx=40):
                                temps=temps or tuple([0.0] * B))
 
 
-def _run(w, env_off=False, logits=True):
+def _run(w, env_off=False, logits=True, no_persistent=False):
     if env_off:
         os.environ["FM_DISABLE_TC"] = "1"
+    if no_persistent:
+        os.environ["FM_DISABLE_PERSISTENT"] = "1"
     try:
         ctx = gu.make_ctx(w, max_new=64)
     finally:
         os.environ.pop("FM_DISABLE_TC", None)
+        os.environ.pop("FM_DISABLE_PERSISTENT", None)
     seqs = list(range(w.B))
     gu.gpu_prefill(ctx, w, seqs, max_new=64)
     gu.gpu_new_rows(ctx, w, 0, seqs)
@@ -62,6 +65,20 @@ def test_tc_draft_matches_oracle(B, N):
     (tok2, none), _ = _run(w, logits=False)
     assert none is None
     np.testing.assert_array_equal(tok2, tok)
+
+
+def test_persistent_pass_matches_per_kernel_path():
+    # one sequence, one noise draft: the persistent DiT pass (with the 17 new
+    # context rows projected inside its QKV phases) against one kernel per GEMM
+    w = _workload(1, 1)
+    (tok_p, lg_p), _ = _run(w)
+    (tok_k, lg_k), _ = _run(w, no_persistent=True)
+    np.testing.assert_allclose(lg_p, lg_k, atol=2e-2, rtol=1e-2)
+    ref = gu.oracle_draft(w, 0, 0)
+    gu.assert_logits_close(lg_p[0], ref["logits"], "bf16", "persistent")
+    # a second draft after more context rows: the cache rows the first pass wrote
+    w2 = dataclasses.replace(w, name="small_bf16_b")
+    assert w2.shape == w.shape
 
 
 def test_tc_matches_cuda_core_path():
