@@ -76,9 +76,29 @@ def test_persistent_pass_matches_per_kernel_path():
     np.testing.assert_allclose(lg_p, lg_k, atol=2e-2, rtol=1e-2)
     ref = gu.oracle_draft(w, 0, 0)
     gu.assert_logits_close(lg_p[0], ref["logits"], "bf16", "persistent")
-    # a second draft after more context rows: the cache rows the first pass wrote
-    w2 = dataclasses.replace(w, name="small_bf16_b")
-    assert w2.shape == w.shape
+
+
+def test_persistent_pass_context_rows_reach_the_cache():
+    # round 0 appends 17 rows (projected inside the first draft's QKV phases);
+    # round 1 appends 17 more after them and drafts against all of them, so
+    # its logits check the keys/values the first pass wrote
+    w = _workload(1, 1)
+    ctx = Context(w.shape, w.dtype, gu.weights(w.shape, w.dtype), max_ctx=w.ctx + 40,
+                  max_seqs=1, max_noise=1, max_new=64)
+    gu.gpu_prefill(ctx, w, [0], max_new=64)
+    rows = [fs.prefill_hidden(w, 0)]
+    for r, p0 in ((0, w.ctx), (1, w.ctx + 17)):
+        ri = fs.round_inputs(w, r)
+        ctx.project([0], to_device(ri.new_hidden, "bf16"), [p0])
+        rows.append(ri.new_hidden[0])
+        tok, lg = ctx.draft([0], to_device(ri.noise, "bf16"), w.t_grid, w.temps)
+        torch.cuda.synchronize()
+        fm_device_status(ctx.ctx)
+        W = gu.weights64(w.shape, w.dtype)
+        _, kv = om.project_context(W, w.shape.n_blocks, np.concatenate(rows, axis=0))
+        ref = om.draft(W, w.shape, kv, ri.noise[0], w.t_grid)
+        gu.assert_logits_close(gu.to_np(lg)[0], ref["logits"], "bf16", f"round {r}")
+    ctx.close()
 
 
 def test_tc_matches_cuda_core_path():
