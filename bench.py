@@ -268,7 +268,7 @@ def run_fm(args, w, rank, world, local_rank):
             with torch.cuda.graph(gr):
                 step(rounds[i], n_acc_round[i], torch.cuda.current_stream())
             graphs.append(gr)
-        _, cap_launches = fmb.fm_profile_read(ctx.ctx)
+        _, cap_launches = fmb.fm_profile_read(ctx.ctx, times=False)
         launches_per_step = sum(cap_launches) / R
         for gr in graphs:          # one untimed replay each
             gr.replay()

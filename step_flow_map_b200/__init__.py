@@ -191,12 +191,17 @@ def fm_profile(ctx, mask: int) -> None:
     _check(load_library().fm_profile(ctx, int(mask)))
 
 
-def fm_profile_read(ctx, reset: bool = False):
-    """(ms per class, launches per class), each a list of FM_PROF_N numbers."""
-    ms = (ctypes.c_double * FM_PROF_N)()
+def fm_profile_read(ctx, reset: bool = False, times: bool = True):
+    """(ms per class, launches per class), each a list of FM_PROF_N numbers.
+
+    ``times=False`` reads the launch counts only (ms comes back as None); use
+    it while the recorded events have not run yet, e.g. right after a CUDA
+    graph capture.
+    """
+    ms = (ctypes.c_double * FM_PROF_N)() if times else None
     n = (ctypes.c_int64 * FM_PROF_N)()
     _check(load_library().fm_profile_read(ctx, ms, n, int(bool(reset))))
-    return list(ms), list(n)
+    return (list(ms) if times else None), list(n)
 
 
 def fm_device_status(ctx, stream=None) -> None:

@@ -98,6 +98,7 @@ struct fm_ctx {
   float* dit_stats = nullptr;
   void* dit_hf = nullptr;
   bool dit_ok = false;           // the persistent pass fits this configuration and device
+  int dit_l2_ahead = 0;          // weight k-blocks the persistent pass prefetches into L2 (measured: no gain)
   float* attn_part = nullptr;   // split-KV attention partials
   unsigned* attn_cnt = nullptr;
   size_t attn_part_elems = 0;
@@ -410,6 +411,9 @@ fm_status load_impl(fm_ctx* c, cudaStream_t st) {
                                                             fm::TC_THREADS, fm::DIT_SMEM));
       c->dit_ok = per_sm >= 1;
     }
+    // diagnostic: L2 prefetch depth of the persistent pass (k-blocks, 0 = off)
+    const char* ahead = getenv("FM_DIT_L2_AHEAD");
+    if (ahead) c->dit_l2_ahead = std::max(0, std::min(256, atoi(ahead)));
   }
   // the grids every draft uses
   const float grids[3][2] = {{0.f, 1.f}, {0.f, 0.5f}, {0.5f, 1.f}};
@@ -467,8 +471,12 @@ fm_status project_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void
   }
   c->pending_rows = R;
   // keys/values now unless a small draft can take them over
-  if (!(sizeof(T) == 2 && c->use_tc && c->ln_in_gemm && R < FUSED_CTX_ROWS))
-    FM_TRY(flush_pending<T>(c, st));
+  // keys/values now unless a following draft can take them over: the
+  // persistent pass (one 16-row draft) or an in-GEMM LayerNorm path
+  const bool absorb = sizeof(T) == 2 && c->use_tc &&
+                      ((c->ln_in_gemm && R < FUSED_CTX_ROWS) ||
+                       (c->dit_ok && fm::DIT_M + R <= fm::DIT_BROWS_MAX));
+  if (!absorb) FM_TRY(flush_pending<T>(c, st));
   for (int q = 0; q < n_seqs; ++q) c->ctx_len[seq_ids[q]] = pos0[q] + n_new;
   return FM_OK;
 }
@@ -528,6 +536,7 @@ fm_status dit_persistent(fm_ctx* c, const float* mods, int slot, int ctx_len, bo
   P.d = d;
   P.F = g.mlp;
   P.M = fm::DIT_M;
+  P.l2_ahead = c->dit_l2_ahead;
   // K splits per GEMM kind: about one unit per SM
   const int tiles[5] = {3 * d / 128, 0, d / 128, g.mlp / 128, d / 128};
   const int kbs[5] = {d / 64, 0, d / 64, d / 64, g.mlp / 64};
@@ -560,6 +569,8 @@ fm_status dit_persistent(fm_ctx* c, const float* mods, int slot, int ctx_len, bo
     const int brows = (k == fm::DIT_QKV && P.n_ctx) ? (fm::DIT_M + P.n_ctx + 15) / 16 * 16 : 16;
     const int nkb = (kbs[k] + P.splits[k] - 1) / P.splits[k];
     if ((size_t)nkb * brows * 128 > (size_t)fm::DIT_UNION) return FM_ERR_UNSUPPORTED;
+    if (nkb * 64 > 1024) return FM_ERR_UNSUPPORTED;  // staged shift/scale slice
+    if ((size_t)P.splits[k] * 128 * brows * 4 > (size_t)fm::DIT_UNION) return FM_ERR_UNSUPPORTED;
     if ((size_t)P.splits[k] * tiles[k] * 128 * brows > c->splitk_elems) return FM_ERR_UNSUPPORTED;
   }
   fm::AttnMmaArgs& am = P.attn;

@@ -316,46 +316,55 @@ __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf
   if (!s_last) return;
   __threadfence();
   // ---- last CTA of this (sequence, head): merge the splits in split order,
-  // one warp per query row, four columns per lane, loads of several splits
-  // in flight
+  // eight threads per query row (sixteen columns each), four splits' partials
+  // in flight per thread
   const float* pp = a.part + (size_t)pair * S_all * NQ * AM_PSTRIDE;
-  for (int q = warp; q < NQ; q += AM_THREADS / 32) {
-    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-    float l = 0.f, M = -INFINITY;
-    for (int s0 = 0; s0 < S_all; s0 += 8) {
-      float2 ml[8];
-      float4 os[8];
+  const int cg = (tid & 7) * 16;
+  for (int q = tid >> 3; q < NQ; q += AM_THREADS / 8) {
+    float o[16];
 #pragma unroll
-      for (int u2 = 0; u2 < 8; ++u2) {   // all loads of the batch in flight
+    for (int i = 0; i < 16; ++i) o[i] = 0.f;
+    float l = 0.f, M = -INFINITY;
+    for (int s0 = 0; s0 < S_all; s0 += 4) {
+      float2 ml[4];
+      float4 os[4][4];
+#pragma unroll
+      for (int u2 = 0; u2 < 4; ++u2) {
         if (s0 + u2 < S_all) {
           const float* w = pp + ((size_t)(s0 + u2) * NQ + q) * AM_PSTRIDE;
           ml[u2] = __ldcg((const float2*)(w + AM_DH));
-          os[u2] = __ldcg((const float4*)(w + 4 * lane));
+#pragma unroll
+          for (int i = 0; i < 4; ++i) os[u2][i] = __ldcg((const float4*)(w + cg + 4 * i));
         } else {
           ml[u2] = make_float2(-INFINITY, 0.f);
-          os[u2] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
 #pragma unroll
-      for (int u2 = 0; u2 < 8; ++u2) {
+      for (int u2 = 0; u2 < 4; ++u2) {
         if (ml[u2].x == -INFINITY) continue;
         if (ml[u2].x > M) {
           const float f = (M == -INFINITY) ? 0.f : exp2f(M - ml[u2].x);
-          o.x *= f; o.y *= f; o.z *= f; o.w *= f;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) o[i] *= f;
           l *= f;
           M = ml[u2].x;
         }
         const float f = exp2f(ml[u2].x - M);
-        o.x += f * os[u2].x; o.y += f * os[u2].y; o.z += f * os[u2].z; o.w += f * os[u2].w;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          o[4 * i] += f * os[u2][i].x; o[4 * i + 1] += f * os[u2][i].y;
+          o[4 * i + 2] += f * os[u2][i].z; o[4 * i + 3] += f * os[u2][i].w;
+        }
         l += f * ml[u2].y;
       }
     }
     const float inv = 1.f / l;
     const int j = q / 16, i = q % 16;
-    __nv_bfloat162* dst =
-        (__nv_bfloat162*)(out + (size_t)(row0 + j * a.K + i) * a.d + h * AM_DH + 4 * lane);
-    dst[0] = __floats2bfloat162_rn(o.x * inv, o.y * inv);
-    dst[1] = __floats2bfloat162_rn(o.z * inv, o.w * inv);
+    uint4* dst = (uint4*)(out + (size_t)(row0 + j * a.K + i) * a.d + h * AM_DH + cg);
+    dst[0] = make_uint4(pack_bf16x2(o[0] * inv, o[1] * inv), pack_bf16x2(o[2] * inv, o[3] * inv),
+                        pack_bf16x2(o[4] * inv, o[5] * inv), pack_bf16x2(o[6] * inv, o[7] * inv));
+    dst[1] = make_uint4(pack_bf16x2(o[8] * inv, o[9] * inv), pack_bf16x2(o[10] * inv, o[11] * inv),
+                        pack_bf16x2(o[12] * inv, o[13] * inv), pack_bf16x2(o[14] * inv, o[15] * inv));
   }
   if (tid == 0) a.cnt[pair] = 0u;
 }

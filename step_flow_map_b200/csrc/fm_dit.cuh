@@ -35,7 +35,7 @@ constexpr int DIT_RING = 6;                            // weight stages of 16 KB
 constexpr int DIT_M = 16;                              // block rows
 constexpr int DIT_BROWS_MAX = 64;                      // block rows + context rows
 constexpr int DIT_UNION = 109568;                      // B tiles or attention scratch
-constexpr int DIT_SMEM = 1024 + DIT_RING * 16384 + DIT_UNION + 4096;
+constexpr int DIT_SMEM = 1024 + DIT_RING * 16384 + DIT_UNION + 12288;
 
 enum { DIT_QKV = 0, DIT_ATTN = 1, DIT_O = 2, DIT_UP = 3, DIT_DOWN = 4 };
 
@@ -43,6 +43,7 @@ struct DitParams {
   CUtensorMap w[DIT_MAX_BLOCKS][4];   // W_qkv, W_o, W_up, W_down (K-major, box 64 x 128)
   int n_blocks, d, F, M;              // M <= 16 block rows
   int splits[5];                      // per GEMM kind (index by DIT_*; [1] = attention splits)
+  int l2_ahead;                       // weight k-blocks prefetched into L2 beyond the ring
   float* x;                           // residual stream [M][d] fp32
   float* stats;                       // [d/128 tiles][M][2]: tile mean, tile sum of squared deviations
   float* partial;                     // split-K partials
@@ -65,10 +66,11 @@ struct DitParams {
 };
 
 struct DitShared {                    // after the ring and the union region
-  uint64_t full[DIT_RING], empty[DIT_RING], tfull[2], tempty[2], bready;
+  uint64_t full[DIT_RING], empty[DIT_RING], tfull[2], tempty[2], bready, rbar;
   uint32_t tmem;
   int abort, last, ok[2], attn_last;
   float stat[2 * DIT_BROWS_MAX];      // mean, rstd per row
+  float ss[2][1024];                  // shift, scale of this CTA's column slice
   float red[4][DIT_M][2];             // per-warp row partials
 };
 
@@ -88,6 +90,48 @@ __device__ __forceinline__ void dit_gemm_shape(const DitParams& P, int kind, int
   else if (kind == DIT_O) { *N = d; *Kd = d; }
   else if (kind == DIT_UP) { *N = P.F; *Kd = d; }
   else { *N = d; *Kd = P.F; }
+}
+
+// Position of the weight producer in this CTA's sequence of k-blocks over all
+// GEMM phases.
+struct DitCursor {
+  int p, l, kind, nt, kb, kb1;
+  bool valid;
+};
+
+// First k-block of the first phase >= p with GEMM work for this CTA.
+__device__ __forceinline__ void dit_cursor_seek(const DitParams& P, int cta, int n_phases, int p,
+                                                DitCursor& c) {
+  for (; p < n_phases - 1; ++p) {
+    int l = 0;
+    const int kind = dit_phase_kind(p, P.n_blocks, &l);
+    if (kind < 0 || kind == DIT_ATTN) continue;
+    int N, Kd;
+    dit_gemm_shape(P, kind, &N, &Kd);
+    const int S = P.splits[kind], tiles = N / TC_BM, kbs = Kd / TC_BK;
+    if (cta >= tiles * S) continue;
+    const int z = cta % S;
+    c.p = p;
+    c.l = l;
+    c.kind = kind;
+    c.nt = cta / S;
+    c.kb = z * kbs / S;
+    c.kb1 = (z + 1) * kbs / S;
+    if (c.kb >= c.kb1) continue;
+    c.valid = true;
+    return;
+  }
+  c.valid = false;
+}
+
+__device__ __forceinline__ void dit_cursor_next(const DitParams& P, int cta, int n_phases,
+                                                DitCursor& c) {
+  if (++c.kb < c.kb1) return;
+  dit_cursor_seek(P, cta, n_phases, c.p + 1, c);
+}
+
+__device__ __forceinline__ const CUtensorMap* dit_wmap(const DitParams& P, const DitCursor& c) {
+  return &P.w[c.l][c.kind == DIT_QKV ? 0 : c.kind - 1];
 }
 
 __device__ __forceinline__ int dit_brows(const DitParams& P, int kind) {
@@ -142,22 +186,37 @@ __device__ __forceinline__ void dit_tile_stats(const float* v, int M, int et, Di
   named_sync(1, 128);
 }
 
-// Row mean / rstd from the 16 tile partials (fixed order; equal tile sizes).
+// Row mean / rstd from the tile partials (fixed order; equal tile sizes):
+// eight threads per row, each loading two tiles' (mean, M2), combined over
+// the eight lanes with shuffles (Chan's update with equal counts).
 __device__ __forceinline__ void dit_row_stats(const DitParams& P, int et, DitShared* sh) {
-  if (et < P.M) {
-    const float* st = P.stats;
-    const int tiles = P.d / 128;
-    float mean = 0.f;
-    for (int t = 0; t < tiles; ++t) mean += __ldcg(st + ((size_t)t * P.M + et) * 2);
-    mean /= (float)tiles;
-    float m2 = 0.f;
-    for (int t = 0; t < tiles; ++t) {
-      const float mt = __ldcg(st + ((size_t)t * P.M + et) * 2);
-      const float dv = mt - mean;
-      m2 += __ldcg(st + ((size_t)t * P.M + et) * 2 + 1) + 128.f * dv * dv;
+  const int row = et >> 3, g = et & 7;
+  const int tiles = P.d / 128;  // <= 16
+  float mt[2] = {0.f, 0.f}, m2t[2] = {0.f, 0.f};
+  bool have[2] = {false, false};
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int t = g + 8 * i;
+    if (row < P.M && t < tiles) {
+      const float2 v = __ldcg((const float2*)(P.stats + ((size_t)t * P.M + row) * 2));
+      mt[i] = v.x;
+      m2t[i] = v.y;
+      have[i] = true;
     }
-    sh->stat[et] = mean;
-    sh->stat[DIT_BROWS_MAX + et] = rsqrtf(m2 / (float)(tiles * 128) + 1e-6f);
+  }
+  float s = (have[0] ? mt[0] : 0.f) + (have[1] ? mt[1] : 0.f);
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  const float mean = s / (float)tiles;
+  float q = 0.f;
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+    if (have[i]) q += m2t[i] + 128.f * (mt[i] - mean) * (mt[i] - mean);
+#pragma unroll
+  for (int o = 1; o < 8; o <<= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+  if (g == 0 && row < P.M) {
+    sh->stat[row] = mean;
+    sh->stat[DIT_BROWS_MAX + row] = rsqrtf(q / (float)(tiles * 128) + 1e-6f);
   }
   named_sync(1, 128);
 }
@@ -166,43 +225,88 @@ __device__ __forceinline__ void dit_row_stats(const DitParams& P, int et, DitSha
 // (128-byte swizzle).  kind QKV/UP: rows < M are the modulated LayerNorm
 // of x, QKV rows M .. M+n_ctx-1 are copied context rows; kind O/DOWN: rows
 // < M are copied from o / u.  Other rows are zero.
+// Shift and scale of a LayerNorm phase for this CTA's columns [c0, c0 + ncol)
+// into shared memory, all loads in flight at once.  The adaLN modulation is
+// fixed for the whole pass, so this runs before the phase's grid barrier.
+__device__ __forceinline__ void dit_stage_mods(const DitParams& P, int kind, int l, int c0,
+                                               int ncol, int et, DitShared* sh) {
+  const float* ml = P.mods + (size_t)l * 6 * P.d;
+  const float* shift = kind == DIT_QKV ? ml : ml + 3 * P.d;
+  const float* scale = kind == DIT_QKV ? ml + P.d : ml + 4 * P.d;
+  float hv[8], cv[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int c = et + 128 * u;
+    hv[u] = cv[u] = 0.f;
+    if (c < ncol) {
+      hv[u] = __ldg(shift + c0 + c);
+      cv[u] = __ldg(scale + c0 + c);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int c = et + 128 * u;
+    if (c < ncol) {
+      sh->ss[0][c] = hv[u];
+      sh->ss[1][c] = cv[u];
+    }
+  }
+}
+
 __device__ __forceinline__ void dit_fill_b(const DitParams& P, int kind, int l, uint8_t* sB,
                                            int kb0, int nkb, int brows, int Kd, int et,
                                            DitShared* sh) {
   const bool ln = (kind == DIT_QKV || kind == DIT_UP);
-  if (ln) dit_row_stats(P, et, sh);
-  const float* shift = nullptr;
-  const float* scale = nullptr;
-  if (ln) {
-    const float* ml = P.mods + (size_t)l * 6 * P.d;
-    shift = kind == DIT_QKV ? ml : ml + 3 * P.d;
-    scale = kind == DIT_QKV ? ml + P.d : ml + 4 * P.d;
-  }
+  if (ln) dit_row_stats(P, et, sh);   // ends with a barrier
   const bf16* src = kind == DIT_O ? P.o : P.u;
   const int tile_bytes = brows * 128;
-  for (int idx = et; idx < nkb * brows * 8; idx += 128) {
-    const int kbi = idx / (brows * 8), rem = idx - kbi * (brows * 8);
-    const int row = rem >> 3, ch = rem & 7;
-    const int col = (kb0 + kbi) * TC_BK + ch * 8;
-    uint4 packed = make_uint4(0, 0, 0, 0);
-    if (row < P.M) {
-      if (ln) {
-        const float mean = sh->stat[row], rstd = sh->stat[DIT_BROWS_MAX + row];
-        const float* xr = P.x + (size_t)row * P.d + col;
-        const float4 x0 = __ldcg((const float4*)xr), x1 = __ldcg((const float4*)(xr + 4));
-        const float4 c0 = *(const float4*)(scale + col), c1 = *(const float4*)(scale + col + 4);
-        const float4 h0 = *(const float4*)(shift + col), h1 = *(const float4*)(shift + col + 4);
-        packed.x = pack_bf16x2((x0.x - mean) * rstd * (1.f + c0.x) + h0.x, (x0.y - mean) * rstd * (1.f + c0.y) + h0.y);
-        packed.y = pack_bf16x2((x0.z - mean) * rstd * (1.f + c0.z) + h0.z, (x0.w - mean) * rstd * (1.f + c0.w) + h0.w);
-        packed.z = pack_bf16x2((x1.x - mean) * rstd * (1.f + c1.x) + h1.x, (x1.y - mean) * rstd * (1.f + c1.y) + h1.y);
-        packed.w = pack_bf16x2((x1.z - mean) * rstd * (1.f + c1.z) + h1.z, (x1.w - mean) * rstd * (1.f + c1.w) + h1.w);
-      } else {
-        packed = __ldcg((const uint4*)(src + (size_t)row * Kd + col));
+  const int items = nkb * brows * 8;
+  // eight items per thread and batch: every load of a batch is in flight
+  // before any is used
+  for (int i0 = 0; i0 < items; i0 += 128 * 8) {
+    float4 xa[8], xb[8];
+    uint4 cp[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int idx = i0 + u * 128 + et;
+      const int kbi = idx / (brows * 8), rem = idx - kbi * (brows * 8);
+      const int row = rem >> 3, ch = rem & 7;
+      const int col = (kb0 + kbi) * TC_BK + ch * 8;
+      cp[u] = make_uint4(0, 0, 0, 0);
+      xa[u] = xb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (idx < items && col < Kd) {
+        if (row < P.M) {
+          if (ln) {
+            const float* xr = P.x + (size_t)row * P.d + col;
+            xa[u] = __ldcg((const float4*)xr);
+            xb[u] = __ldcg((const float4*)(xr + 4));
+          } else {
+            cp[u] = __ldcg((const uint4*)(src + (size_t)row * Kd + col));
+          }
+        } else if (kind == DIT_QKV && row - P.M < P.n_ctx) {
+          cp[u] = __ldcg((const uint4*)(P.ctx_rows + (size_t)(row - P.M) * P.d + col));
+        }
       }
-    } else if (kind == DIT_QKV && row - P.M < P.n_ctx) {
-      packed = __ldcg((const uint4*)(P.ctx_rows + (size_t)(row - P.M) * P.d + col));
     }
-    *(uint4*)(sB + kbi * tile_bytes + row * 128 + ((ch ^ (row & 7)) << 4)) = packed;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int idx = i0 + u * 128 + et;
+      if (idx >= items) break;
+      const int kbi = idx / (brows * 8), rem = idx - kbi * (brows * 8);
+      const int row = rem >> 3, ch = rem & 7;
+      const int cc = kbi * TC_BK + ch * 8;  // column within this CTA's slice
+      uint4 packed = cp[u];
+      if (ln && row < P.M) {
+        const float mean = sh->stat[row], rstd = sh->stat[DIT_BROWS_MAX + row];
+        const float* h = sh->ss[0] + cc;
+        const float* c = sh->ss[1] + cc;
+        packed.x = pack_bf16x2((xa[u].x - mean) * rstd * (1.f + c[0]) + h[0], (xa[u].y - mean) * rstd * (1.f + c[1]) + h[1]);
+        packed.y = pack_bf16x2((xa[u].z - mean) * rstd * (1.f + c[2]) + h[2], (xa[u].w - mean) * rstd * (1.f + c[3]) + h[3]);
+        packed.z = pack_bf16x2((xb[u].x - mean) * rstd * (1.f + c[4]) + h[4], (xb[u].y - mean) * rstd * (1.f + c[5]) + h[5]);
+        packed.w = pack_bf16x2((xb[u].z - mean) * rstd * (1.f + c[6]) + h[6], (xb[u].w - mean) * rstd * (1.f + c[7]) + h[7]);
+      }
+      *(uint4*)(sB + kbi * tile_bytes + row * 128 + ((ch ^ (row & 7)) << 4)) = packed;
+    }
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -227,13 +331,20 @@ __device__ __forceinline__ void dit_epilogue_chunk(const DitParams& P, int kind,
       }
     } else if (kind == DIT_UP) {
       if (m < P.M) P.u[(size_t)m * P.F + n] = __float2bfloat16_rn(gelu_tanh(v[j]));
-    } else {  // residual: x += gate * y
-      if (m < P.M) {
-        const float* gate = P.mods + (size_t)l * 6 * d + (kind == DIT_O ? 2 : 5) * d;
-        const float xv = __ldcg(P.x + (size_t)m * d + n) + gate[n] * v[j];
-        P.x[(size_t)m * d + n] = xv;
-        xn[m] = xv;
-      }
+    }
+  }
+}
+
+// Residual epilogue of an O or down-projection tile (16 rows): x += gate * y,
+// with x and the gate loaded before the accumulator was ready.
+__device__ __forceinline__ void dit_epilogue_residual(const DitParams& P, int n, const float* v,
+                                                      const float* xo, float gate, float* xn) {
+#pragma unroll
+  for (int j = 0; j < DIT_M; ++j) {
+    if (j < P.M) {
+      const float xv = xo[j] + gate * v[j];
+      P.x[(size_t)j * P.d + n] = xv;
+      xn[j] = xv;
     }
   }
 }
@@ -259,6 +370,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
       mbar_init(smem_u32(&sh->tempty[i]), 128);
     }
     mbar_init(smem_u32(&sh->bready), 128);
+    mbar_init(smem_u32(&sh->rbar), 1);
     sh->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -272,27 +384,36 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
   const uint32_t tmem = sh->tmem;
 
   if (warp == 0) {
-    // ---------------- weight producer: all phases, never waits on a barrier
+    // ---------------- weight producer: all phases, never waits on a barrier.
+    // Loads fill the shared-memory ring; while the ring is full, L2
+    // prefetches run up to l2_ahead k-blocks further down the same sequence
+    // so HBM keeps streaming through barriers, fills and attention.
     if (lane == 0) {
+      DitCursor ld, pf;
+      dit_cursor_seek(P, cta, n_phases, 1, ld);
+      pf = ld;
+      int ahead = 0;                    // k-blocks prefetched beyond ld
       int stage = 0;
       uint32_t phase = 0;
-      for (int p = 1; p < n_phases - 1 && !*abort; ++p) {
-        int l = 0;
-        const int kind = dit_phase_kind(p, nb, &l);
-        if (kind == DIT_ATTN) continue;
-        int N, Kd;
-        dit_gemm_shape(P, kind, &N, &Kd);
-        const int S = P.splits[kind], tiles = N / TC_BM, kbs = Kd / TC_BK;
-        if (cta >= tiles * S) continue;
-        const int nt = cta / S, z = cta % S;
-        const int kb0 = z * kbs / S, kb1 = (z + 1) * kbs / S;
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(smem_u32(&sh->empty[stage]), phase ^ 1, abort)) break;
+      unsigned long long t_prog = gtimer();
+      while (ld.valid && !*abort) {
+        if (mbar_try(smem_u32(&sh->empty[stage]), phase ^ 1)) {
           const uint32_t fb = smem_u32(&sh->full[stage]);
           mbar_expect_tx(fb, 16384);
-          tma_load_2d(smem_u32(sA + stage * 16384), &P.w[l][kind == DIT_QKV ? 0 : kind - 1],
-                      kb * TC_BK, nt * TC_BM, fb);
+          tma_load_2d(smem_u32(sA + stage * 16384), dit_wmap(P, ld), ld.kb * TC_BK, ld.nt * TC_BM, fb);
           if (++stage == DIT_RING) { stage = 0; phase ^= 1; }
+          dit_cursor_next(P, cta, n_phases, ld);
+          if (ahead > 0) --ahead;
+          else pf = ld;
+          t_prog = gtimer();
+        } else if (pf.valid && ahead < P.l2_ahead) {
+          tma_prefetch_2d(dit_wmap(P, pf), pf.kb * TC_BK, pf.nt * TC_BM);
+          dit_cursor_next(P, cta, n_phases, pf);
+          ++ahead;
+          t_prog = gtimer();
+        } else if (gtimer() - t_prog > TC_TIMEOUT_NS) {
+          *abort = 1;
+          break;
         }
       }
     }
@@ -342,9 +463,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
     const int q = warp & 3;
     const int r = q * 32 + lane;          // feature row within a 128-row weight tile
     int acc = 0;
-    uint32_t acc_phase = 0;
+    uint32_t acc_phase = 0, r_phase = 0;
     int it = 0;
     for (int p = 0; p < n_phases; ++p) {
+      {
+        int l0 = 0;
+        const int k0 = dit_phase_kind(p, nb, &l0);
+        if (k0 == DIT_QKV || k0 == DIT_UP) {
+          int N, Kd;
+          dit_gemm_shape(P, k0, &N, &Kd);
+          const int S = P.splits[k0], kbs = Kd / TC_BK;
+          if (cta < (N / TC_BM) * S) {
+            const int z = cta % S;
+            const int kb0 = z * kbs / S, kb1 = (z + 1) * kbs / S;
+            dit_stage_mods(P, k0, l0, kb0 * TC_BK, (kb1 - kb0) * TC_BK, et, sh);
+          }
+        }
+      }
       if (p > 0) {
         // wait until every CTA finished phase p - 1
         if (et == 0) sh->ok[it & 1] = dit_grid_wait(P, (unsigned)(p * G)) ? 1 : 0;
@@ -391,6 +526,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
           const int brows = dit_brows(P, kind);
           dit_fill_b(P, kind, l, sU, kb0, kb1 - kb0, brows, Kd, et, sh);
           mbar_arrive(smem_u32(&sh->bready));
+          const int n = nt * TC_BM + r;
+          // residual phases: x and the gate, loaded while the MMAs run
+          const bool resid = (kind == DIT_O || kind == DIT_DOWN);
+          float xo[DIT_M];
+          float gate = 0.f;
+          if (resid) {
+            gate = __ldg(P.mods + (size_t)l * 6 * P.d + (kind == DIT_O ? 2 : 5) * P.d + n);
+#pragma unroll
+            for (int j = 0; j < DIT_M; ++j) xo[j] = j < P.M ? __ldcg(P.x + (size_t)j * P.d + n) : 0.f;
+          }
           // accumulator ready
           if (et == 0) sh->ok[it & 1] = mbar_wait(smem_u32(&sh->tfull[acc]), acc_phase, abort) ? 1 : 0;
           named_sync(1, 128);
@@ -402,7 +547,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
           ++it;
           tc_fence_after();
           const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + acc * 64;
-          const int n = nt * TC_BM + r;
           float v[16];
           float xn[DIT_M];
 #pragma unroll
@@ -410,7 +554,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
           if (S == 1) {
             for (int j0 = 0; j0 < brows; j0 += 16) {
               tmem_ld16(taddr + j0, v);
-              dit_epilogue_chunk(P, kind, l, n, j0, v, xn);
+              if (resid) dit_epilogue_residual(P, n, v, xo, gate, xn);
+              else dit_epilogue_chunk(P, kind, l, n, j0, v, xn);
             }
             tc_fence_before();
             mbar_arrive(smem_u32(&sh->tempty[acc]));
@@ -429,30 +574,44 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
             if (et == 0) sh->last = (atomicAdd(&P.tile_cnt[nt], 1u) == (unsigned)(S - 1));
             named_sync(1, 128);
             if (sh->last) {
-              __threadfence();
-              const size_t zstride = (size_t)tiles * TC_BM * brows;
-              const float* p0 = P.partial + ((size_t)nt * TC_BM + r) * brows;
+              // the S partial tiles of this output tile, one bulk copy each,
+              // into the B region (the MMAs that read it have completed)
+              const uint32_t tile_bytes = (uint32_t)(TC_BM * brows * 4);
+              const uint32_t rb = smem_u32(&sh->rbar);
+              if (et == 0) {
+                __threadfence();
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+                mbar_expect_tx(rb, tile_bytes * S);
+                for (int zz = 0; zz < S; ++zz)
+                  bulk_load(smem_u32(sU) + zz * tile_bytes,
+                            P.partial + ((size_t)zz * tiles + nt) * TC_BM * brows, tile_bytes, rb);
+              }
+              // one bounded waiter decides for all; then every thread observes
+              // the completed phase itself (it cannot advance again here)
+              if (et == 0) sh->ok[it & 1] = mbar_wait(rb, r_phase, abort) ? 1 : 0;
+              named_sync(1, 128);
+              if (!sh->ok[it & 1]) {
+                *abort = 1;
+                if (et == 0) atomicExch(P.abort_g, 1);
+                break;
+              }
+              ++it;
+              (void)mbar_wait(rb, r_phase, abort);   // returns at once
+              r_phase ^= 1;
+              const float* sp = (const float*)sU + (size_t)r * brows;
               for (int j0 = 0; j0 < brows; j0 += 16) {
 #pragma unroll
                 for (int j = 0; j < 16; ++j) v[j] = 0.f;
-                for (int zz = 0; zz < S; zz += 4) {
-                  float4 t4[4][4];
+                for (int zz = 0; zz < S; ++zz) {
+                  const float4* t4 = (const float4*)(sp + (size_t)zz * TC_BM * brows + j0);
 #pragma unroll
-                  for (int u2 = 0; u2 < 4; ++u2)
-                    if (zz + u2 < S)
-#pragma unroll
-                      for (int j = 0; j < 4; ++j)
-                        t4[u2][j] = __ldcg((const float4*)(p0 + (zz + u2) * zstride + j0 + 4 * j));
-#pragma unroll
-                  for (int u2 = 0; u2 < 4; ++u2)
-                    if (zz + u2 < S)
-#pragma unroll
-                      for (int j = 0; j < 4; ++j) {
-                        v[4 * j] += t4[u2][j].x; v[4 * j + 1] += t4[u2][j].y;
-                        v[4 * j + 2] += t4[u2][j].z; v[4 * j + 3] += t4[u2][j].w;
-                      }
+                  for (int j = 0; j < 4; ++j) {
+                    const float4 t = t4[j];
+                    v[4 * j] += t.x; v[4 * j + 1] += t.y; v[4 * j + 2] += t.z; v[4 * j + 3] += t.w;
+                  }
                 }
-                dit_epilogue_chunk(P, kind, l, n, j0, v, xn);
+                if (resid) dit_epilogue_residual(P, n, v, xo, gate, xn);
+                else dit_epilogue_chunk(P, kind, l, n, j0, v, xn);
               }
               if (et == 0) P.tile_cnt[nt] = 0u;
             }
