@@ -93,8 +93,8 @@ struct fm_ctx {
   float* vg_pv = nullptr;
   int* vg_pi = nullptr;
   unsigned* vg_cnt = nullptr;
-  unsigned* dit_bar = nullptr;   // persistent DiT pass: grid barrier counter, abort flag,
-  int* dit_abort = nullptr;      //   LayerNorm tile statistics, final LayerNorm output
+  unsigned* dit_flags = nullptr; // persistent DiT pass: abort word, completion counters and
+  size_t dit_flags_n = 0;        //   flags, LayerNorm tile statistics, final LayerNorm output
   float* dit_stats = nullptr;
   void* dit_hf = nullptr;
   bool dit_ok = false;           // the persistent pass fits this configuration and device
@@ -369,8 +369,10 @@ fm_status load_impl(fm_ctx* c, cudaStream_t st) {
   FM_TRY(dalloc_t(c, &c->attn_part, c->attn_part_elems));
   FM_TRY(dalloc_t(c, &c->attn_cnt, (size_t)c->attn_pairs_max));
   FM_CUDA(cudaMemsetAsync(c->attn_cnt, 0, c->attn_pairs_max * sizeof(unsigned), st));
-  FM_TRY(dalloc_t(c, &c->dit_bar, 1));
-  FM_TRY(dalloc_t(c, &c->dit_abort, 1));
+  // abort word, c_stats, c_o[nb], c_down[nb], f_qkv[nb][3d/128], f_head[nb][H], f_up[nb][F/128]
+  c->dit_flags_n = 2 + 2 * (size_t)g.n_blocks +
+                   (size_t)g.n_blocks * (3 * d / 128 + g.n_heads + g.mlp / 128);
+  FM_TRY(dalloc_t(c, &c->dit_flags, c->dit_flags_n));
   FM_TRY(dalloc_t(c, &c->dit_stats, (size_t)(d / 128 + 1) * fm::DIT_M * 2));
   FM_TRY(dalloc(c, &c->dit_hf, (size_t)fm::DIT_M * d * sizeof(T)));
   FM_TRY(dalloc_t(c, &c->c_raw, (size_t)c->R_max * d));
@@ -548,9 +550,18 @@ fm_status dit_persistent(fm_ctx* c, const float* mods, int slot, int ctx_len, bo
   P.stats = c->dit_stats;
   P.partial = c->splitk;
   P.tile_cnt = c->tile_cnt;
-  P.bar = c->dit_bar;
+  {
+    unsigned* f = c->dit_flags;
+    const int nb = g.n_blocks;
+    P.abort_g = (int*)f;
+    P.c_stats = f + 1;
+    P.c_o = f + 2;
+    P.c_down = P.c_o + nb;
+    P.f_qkv = P.c_down + nb;
+    P.f_head = P.f_qkv + (size_t)nb * (3 * d / 128);
+    P.f_up = P.f_head + (size_t)nb * g.n_heads;
+  }
   P.err = c->tc.err;
-  P.abort_g = c->dit_abort;
   P.qkv = (bf16*)c->qkv;
   P.o = (bf16*)c->o;
   P.u = (bf16*)c->u;
@@ -564,15 +575,20 @@ fm_status dit_persistent(fm_ctx* c, const float* mods, int slot, int ctx_len, bo
     P.ctx_map = c->pending_map;
   }
   if (fm::DIT_M + P.n_ctx > fm::DIT_BROWS_MAX) return FM_ERR_UNSUPPORTED;
-  // shared-memory and workspace limits of every phase
+  // shared-memory and workspace limits of every phase; each GEMM kind keeps
+  // its own split-K region and tile counters (consecutive phases overlap)
+  size_t part_total = 0;
   for (int k : {fm::DIT_QKV, fm::DIT_O, fm::DIT_UP, fm::DIT_DOWN}) {
     const int brows = (k == fm::DIT_QKV && P.n_ctx) ? (fm::DIT_M + P.n_ctx + 15) / 16 * 16 : 16;
     const int nkb = (kbs[k] + P.splits[k] - 1) / P.splits[k];
     if ((size_t)nkb * brows * 128 > (size_t)fm::DIT_UNION) return FM_ERR_UNSUPPORTED;
     if (nkb * 64 > 1024) return FM_ERR_UNSUPPORTED;  // staged shift/scale slice
     if ((size_t)P.splits[k] * 128 * brows * 4 > (size_t)fm::DIT_UNION) return FM_ERR_UNSUPPORTED;
-    if ((size_t)P.splits[k] * tiles[k] * 128 * brows > c->splitk_elems) return FM_ERR_UNSUPPORTED;
+    if (tiles[k] > 1024 || 4 * 1024 > c->tile_cnt_n) return FM_ERR_UNSUPPORTED;
+    P.part_off[k] = part_total;
+    part_total += (size_t)P.splits[k] * tiles[k] * 128 * brows;
   }
+  if (part_total > c->splitk_elems) return FM_ERR_UNSUPPORTED;
   fm::AttnMmaArgs& am = P.attn;
   am.n_seqs = 1;
   am.n_noise = 1;
@@ -593,8 +609,7 @@ fm_status dit_persistent(fm_ctx* c, const float* mods, int slot, int ctx_len, bo
     return FM_ERR_UNSUPPORTED;
   am.n_ctx_splits = s_ctx;
   P.splits[fm::DIT_ATTN] = s_ctx;
-  FM_CUDA(cudaMemsetAsync(c->dit_bar, 0, sizeof(unsigned), st));
-  FM_CUDA(cudaMemsetAsync(c->dit_abort, 0, sizeof(int), st));
+  FM_CUDA(cudaMemsetAsync(c->dit_flags, 0, c->dit_flags_n * sizeof(unsigned), st));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(G);
   cfg.blockDim = dim3(fm::TC_THREADS);

@@ -16,6 +16,7 @@
 // split order and writes O / l as bf16.
 #pragma once
 #include "fm_common.cuh"
+#include "fm_tc.cuh"
 
 namespace fm {
 
@@ -164,18 +165,30 @@ __device__ __forceinline__ void load_rows(bf16* dst, const bf16* src, size_t ld,
   }
 }
 
+// Merge of a head's split partials through shared memory: one bulk copy of
+// all partials, completing on `bar` (phase parity `phase`, flipped on use),
+// when they fit in `smem_bytes`; `abort` bounds the wait.  Without it the
+// merging CTA reads the partials from global memory directly.
+struct AttnBulkMerge {
+  uint64_t* bar;
+  uint32_t* phase;
+  volatile int* abort;
+  uint32_t smem_bytes;
+};
+
 // One work item -- (sequence, head) pair `pair`, split `split` -- run by
 // AM_THREADS threads (tid 0..AM_THREADS-1, four whole warps) that
-// synchronise with `sync()`.  `smem_raw` holds attn_mma_smem<N>() bytes;
-// `s_last` is one shared int.
-template <int N, class Sync>
+// synchronise with `sync()`.  ST context chunks are in flight; `smem_raw`
+// holds attn_mma_smem<N, ST>() bytes; `s_last` is one shared int.
+template <int N, int ST, class Sync>
 __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc,
                                           const bf16* __restrict__ Vc, bf16* __restrict__ out,
                                           const AttnMmaArgs& a, int pair, int split,
-                                          uint8_t* smem_raw, int* s_last_p, int tid, Sync sync) {
+                                          uint8_t* smem_raw, int* s_last_p, int tid, Sync sync,
+                                          AttnBulkMerge bm = AttnBulkMerge{nullptr, nullptr, nullptr, 0}) {
   bf16* sQ = (bf16*)smem_raw;                       // [N*16][AM_LD]
-  bf16* sK = sQ + N * 16 * AM_LD;                   // [AM_STAGES][AM_CHUNK][AM_LD]
-  bf16* sV = sK + AM_STAGES * AM_CHUNK * AM_LD;     // [AM_STAGES][AM_CHUNK][AM_LD]
+  bf16* sK = sQ + N * 16 * AM_LD;                   // [ST][AM_CHUNK][AM_LD]
+  bf16* sV = sK + ST * AM_CHUNK * AM_LD;            // [ST][AM_CHUNK][AM_LD]
   int& s_last = *s_last_p;
   constexpr int WPM = 4 / N;                        // warps sharing one 16-query tile
   const int b = pair / a.n_heads, h = pair - b * a.n_heads;
@@ -213,26 +226,26 @@ __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf
     const int n_chunks = (k1 - k0 + AM_CHUNK - 1) / AM_CHUNK;
     auto load_chunk = [&](int c) {
       const int r0 = k0 + c * AM_CHUNK, nr = min(AM_CHUNK, k1 - r0);
-      const int buf = c % AM_STAGES;
+      const int buf = c % ST;
       load_rows(sK + buf * AM_CHUNK * AM_LD, Kc + base + (size_t)r0 * a.d, a.d, nr, AM_CHUNK, tid);
       load_rows(sV + buf * AM_CHUNK * AM_LD, Vc + base + (size_t)r0 * a.d, a.d, nr, AM_CHUNK, tid);
     };
     // one commit group per chunk (empty past the end) keeps the group count
-    // fixed: AM_STAGES - 1 chunks are always in flight ahead of the one used
+    // fixed: ST - 1 chunks are always in flight ahead of the one used
 #pragma unroll
-    for (int c = 0; c < AM_STAGES - 1; ++c) {
+    for (int c = 0; c < ST - 1; ++c) {
       if (c < n_chunks) load_chunk(c);
       cp_commit();
     }
-    cp_wait<AM_STAGES - 1>();   // the query group
+    cp_wait<ST - 1>();   // the query group
     sync();
     q_fragments();
     for (int c = 0; c < n_chunks; ++c) {
-      if (c + AM_STAGES - 1 < n_chunks) load_chunk(c + AM_STAGES - 1);
+      if (c + ST - 1 < n_chunks) load_chunk(c + ST - 1);
       cp_commit();
-      cp_wait<AM_STAGES - 1>();
+      cp_wait<ST - 1>();
       sync();
-      const int buf = c % AM_STAGES;
+      const int buf = c % ST;
       const int nk_chunk = min(AM_CHUNK, k1 - (k0 + c * AM_CHUNK));
       constexpr int KW = AM_CHUNK / WPM;            // keys of this warp within the chunk
       const int kw0 = sub * KW;
@@ -316,9 +329,25 @@ __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf
   if (!s_last) return;
   __threadfence();
   // ---- last CTA of this (sequence, head): merge the splits in split order,
-  // eight threads per query row (sixteen columns each), four splits' partials
-  // in flight per thread
+  // eight threads per query row (sixteen columns each)
   const float* pp = a.part + (size_t)pair * S_all * NQ * AM_PSTRIDE;
+  const uint32_t merge_bytes = (uint32_t)((size_t)S_all * NQ * AM_PSTRIDE * 4);
+  const bool bulk = bm.bar != nullptr && merge_bytes <= bm.smem_bytes;
+  if (bulk) {
+    // all partials of the pair are contiguous: one copy into shared memory
+    const uint32_t mb = (uint32_t)__cvta_generic_to_shared(bm.bar);
+    if (tid == 0) {
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      mbar_expect_tx(mb, merge_bytes);
+      bulk_load((uint32_t)__cvta_generic_to_shared(smem_raw), pp, merge_bytes, mb);
+      if (!mbar_wait(mb, *bm.phase, bm.abort)) s_last = 0;
+    }
+    sync();
+    if (!s_last) return;   // the wait gave up (abort is set)
+    (void)mbar_wait(mb, *bm.phase, bm.abort);   // completed: returns at once
+    *bm.phase ^= 1;
+    pp = (const float*)smem_raw;
+  }
   const int cg = (tid & 7) * 16;
   for (int q = tid >> 3; q < NQ; q += AM_THREADS / 8) {
     float o[16];
@@ -332,9 +361,15 @@ __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf
       for (int u2 = 0; u2 < 4; ++u2) {
         if (s0 + u2 < S_all) {
           const float* w = pp + ((size_t)(s0 + u2) * NQ + q) * AM_PSTRIDE;
-          ml[u2] = __ldcg((const float2*)(w + AM_DH));
+          if (bulk) {
+            ml[u2] = *(const float2*)(w + AM_DH);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) os[u2][i] = __ldcg((const float4*)(w + cg + 4 * i));
+            for (int i = 0; i < 4; ++i) os[u2][i] = *(const float4*)(w + cg + 4 * i);
+          } else {
+            ml[u2] = __ldcg((const float2*)(w + AM_DH));
+#pragma unroll
+            for (int i = 0; i < 4; ++i) os[u2][i] = __ldcg((const float4*)(w + cg + 4 * i));
+          }
         } else {
           ml[u2] = make_float2(-INFINITY, 0.f);
         }
@@ -377,13 +412,13 @@ k_attn_mma(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc, const bf16
   pdl_trigger();
   extern __shared__ __align__(16) uint8_t smem_raw[];
   __shared__ int s_last;
-  attn_item<N>(qkv, Kc, Vc, out, a, blockIdx.x, blockIdx.y, smem_raw, &s_last, threadIdx.x,
+  attn_item<N, AM_STAGES>(qkv, Kc, Vc, out, a, blockIdx.x, blockIdx.y, smem_raw, &s_last, threadIdx.x,
                [] __device__() { __syncthreads(); });
 }
 
-template <int N>
+template <int N, int ST = AM_STAGES>
 constexpr int attn_mma_smem() {
-  return (N * 16 + 2 * AM_STAGES * AM_CHUNK) * AM_LD * 2;
+  return (N * 16 + 2 * ST * AM_CHUNK) * AM_LD * 2;
 }
 
 }  // namespace fm

@@ -31,11 +31,15 @@
 namespace fm {
 
 constexpr int DIT_MAX_BLOCKS = 8;
-constexpr int DIT_RING = 6;                            // weight stages of 16 KB
+constexpr int DIT_RING = 8;                            // weight stages of 16 KB
 constexpr int DIT_M = 16;                              // block rows
 constexpr int DIT_BROWS_MAX = 64;                      // block rows + context rows
-constexpr int DIT_UNION = 109568;                      // B tiles or attention scratch
+constexpr int DIT_ATTN_ST = 2;                         // context chunks in flight in attention
+// B tiles, split-K partial tiles, or attention scratch
+constexpr int DIT_UNION = 87040;
 constexpr int DIT_SMEM = 1024 + DIT_RING * 16384 + DIT_UNION + 12288;
+static_assert(attn_mma_smem<1, DIT_ATTN_ST>() <= DIT_UNION, "attention scratch");
+static_assert(DIT_SMEM <= 232448, "shared memory per CTA");
 
 enum { DIT_QKV = 0, DIT_ATTN = 1, DIT_O = 2, DIT_UP = 3, DIT_DOWN = 4 };
 
@@ -46,11 +50,19 @@ struct DitParams {
   int l2_ahead;                       // weight k-blocks prefetched into L2 beyond the ring
   float* x;                           // residual stream [M][d] fp32
   float* stats;                       // [d/128 tiles][M][2]: tile mean, tile sum of squared deviations
-  float* partial;                     // split-K partials
-  unsigned* tile_cnt;                 // per tile, zero between uses
-  unsigned* bar;                      // grid barrier counter, zeroed before the launch
+  float* partial;                     // split-K partials, one region per GEMM kind
+  size_t part_off[5];                 // float offset of each kind's region
+  unsigned* tile_cnt;                 // [kind][1024] arrivals per output tile, zero between uses
   int* err;                           // error word
   int* abort_g;                       // set when any CTA gave up; zeroed before the launch
+  // completion counters and flags, zeroed before the launch; a unit of a
+  // phase waits only for the units whose outputs it reads
+  unsigned* c_stats;                  // tiles of the embedded rows' statistics done (of d/128)
+  unsigned* c_o;                      // [n_blocks] O-projection tiles done (of d/128)
+  unsigned* c_down;                   // [n_blocks] down-projection tiles done (of d/128)
+  unsigned* f_qkv;                    // [n_blocks][3d/128] QKV output tile done
+  unsigned* f_head;                   // [n_blocks][n_heads] attention output of a head done
+  unsigned* f_up;                     // [n_blocks][F/128] up-projection tile done
   bf16* qkv;                          // [M][3d]
   bf16* o;                            // [M][d]
   bf16* u;                            // [M][F]
@@ -73,6 +85,8 @@ struct DitShared {                    // after the ring and the union region
   float ss[2][1024];                  // shift, scale of this CTA's column slice
   float red[4][DIT_M][2];             // per-warp row partials
 };
+
+static_assert(sizeof(DitShared) + 16 <= 12288, "shared bookkeeping region");
 
 __device__ __forceinline__ int dit_phase_kind(int p, int nb, int* l) {
   // p = 0: statistics of the embedded rows; p = 1 + 5 l + k: block l, kind k;
@@ -139,12 +153,12 @@ __device__ __forceinline__ int dit_brows(const DitParams& P, int kind) {
   return 16;
 }
 
-// Bounded grid barrier wait (one thread): true when `target` arrivals are in.
-__device__ __forceinline__ bool dit_grid_wait(const DitParams& P, unsigned target) {
+// Bounded wait (one thread) until the counter reaches `target`.
+__device__ __forceinline__ bool dit_wait(const DitParams& P, const unsigned* ctr, unsigned target) {
   const unsigned long long t0 = gtimer();
   while (true) {
     unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(P.bar) : "memory");
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
     if (v >= target) return true;
     if (*(volatile int*)P.abort_g) return false;
     if (gtimer() - t0 > TC_TIMEOUT_NS) {
@@ -152,6 +166,49 @@ __device__ __forceinline__ bool dit_grid_wait(const DitParams& P, unsigned targe
       return false;
     }
   }
+}
+
+// Publish one completion (thread et == 0, after the CTA's writes are ordered
+// before it by a CTA barrier).
+__device__ __forceinline__ void dit_signal(unsigned* ctr) {
+  __threadfence();
+  atomicAdd(ctr, 1u);
+}
+
+// Waits (one thread) for everything this CTA's unit of the phase reads:
+//   QKV(l)   the residual stream after the last block (all down tiles) or the
+//            embedded rows' statistics;
+//   ATTN(l)  the Q, K and V tiles of its head;
+//   O(l)     the attention outputs of the heads its k-slice covers;
+//   UP(l)    the residual stream after O(l) (all O tiles);
+//   DOWN(l)  the up-projection tiles its k-slice covers;
+//   final    the residual stream after the last block.
+// Every write-after-read hazard on the shared buffers is ordered through the
+// same chain: a unit that overwrites a buffer depends, through full-row
+// LayerNorm waits, on every unit that read the previous contents.
+__device__ bool dit_wait_deps(const DitParams& P, int kind, int l, int cta) {
+  const unsigned tiles_d = (unsigned)(P.d / TC_BM);
+  const int H = P.attn.n_heads;
+  if (kind == -1) return true;
+  if (kind == -2) return dit_wait(P, P.c_down + P.n_blocks - 1, tiles_d);
+  if (kind == DIT_QKV)
+    return l == 0 ? dit_wait(P, P.c_stats, tiles_d) : dit_wait(P, P.c_down + l - 1, tiles_d);
+  if (kind == DIT_UP) return dit_wait(P, P.c_o + l, tiles_d);
+  if (kind == DIT_ATTN) {
+    const int h = cta % H;
+    const unsigned* f = P.f_qkv + (size_t)l * 3 * H;
+    return dit_wait(P, f + h, 1) && dit_wait(P, f + H + h, 1) && dit_wait(P, f + 2 * H + h, 1);
+  }
+  int N, Kd;
+  dit_gemm_shape(P, kind, &N, &Kd);
+  const int S = P.splits[kind], kbs = Kd / TC_BK, z = cta % S;
+  const int c0 = (z * kbs / S) * TC_BK, c1 = ((z + 1) * kbs / S) * TC_BK;
+  // 128-column groups of the input this k-slice reads (a head, or an up tile)
+  const int g0 = c0 / 128, g1 = (c1 - 1) / 128;
+  const unsigned* f = kind == DIT_O ? P.f_head + (size_t)l * H : P.f_up + (size_t)l * (P.F / TC_BM);
+  for (int g = g0; g <= g1; ++g)
+    if (!dit_wait(P, f + g, 1)) return false;
+  return true;
 }
 
 // Per-row mean and sum of squared deviations over the 128 features held by
@@ -356,7 +413,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
   uint8_t* sU = base + DIT_RING * 16384;
   DitShared* sh = (DitShared*)(sU + DIT_UNION);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int G = gridDim.x, cta = blockIdx.x;
+  const int cta = blockIdx.x;
   const int nb = P.n_blocks, n_phases = 2 + 5 * nb;
   volatile int* abort = &sh->abort;
 
@@ -480,16 +537,25 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
           }
         }
       }
-      if (p > 0) {
-        // wait until every CTA finished phase p - 1
-        if (et == 0) sh->ok[it & 1] = dit_grid_wait(P, (unsigned)(p * G)) ? 1 : 0;
+      int l = 0;
+      const int kind = dit_phase_kind(p, nb, &l);
+      bool active;
+      if (kind == -1 || kind == -2) active = cta < P.d / TC_BM;
+      else if (kind == DIT_ATTN) active = cta < P.attn.n_heads * (P.attn.n_ctx_splits + 1);
+      else {
+        int N, Kd;
+        dit_gemm_shape(P, kind, &N, &Kd);
+        active = cta < (N / TC_BM) * P.splits[kind];
+      }
+      if (!active) continue;
+      if (kind != -1) {
+        // wait for the units whose outputs this one reads
+        if (et == 0) sh->ok[it & 1] = dit_wait_deps(P, kind, l, cta) ? 1 : 0;
         named_sync(1, 128);
         if (!sh->ok[it & 1]) { *abort = 1; break; }
         ++it;
         asm volatile("fence.acq_rel.gpu;" ::: "memory");
       }
-      int l = 0;
-      const int kind = dit_phase_kind(p, nb, &l);
       if (kind == -1 || kind == -2) {
         // statistics of the embedded rows (-1) or the final LayerNorm (-2):
         // CTA t < d/128 owns features [128 t, 128 t + 128)
@@ -500,6 +566,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
 #pragma unroll
             for (int j = 0; j < DIT_M; ++j) v[j] = j < P.M ? __ldcg(P.x + (size_t)j * P.d + n) : 0.f;
             dit_tile_stats(v, P.M, et, sh, P.stats + (size_t)cta * P.M * 2);
+            if (et == 0) dit_signal(P.c_stats);
           } else {
             dit_row_stats(P, et, sh);
             const float* mf = P.mods + (size_t)nb * 6 * P.d;
@@ -512,9 +579,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
       } else if (kind == DIT_ATTN) {
         const int items = P.attn.n_heads * (P.attn.n_ctx_splits + 1);
         if (cta < items) {
-          attn_item<1>(P.qkv, P.Kc[l], P.Vc[l], P.o, P.attn, cta % P.attn.n_heads,
-                       cta / P.attn.n_heads, sU, &sh->attn_last, et,
-                       [] __device__() { named_sync(1, 128); });
+          attn_item<1, DIT_ATTN_ST>(P.qkv, P.Kc[l], P.Vc[l], P.o, P.attn, cta % P.attn.n_heads,
+                                    cta / P.attn.n_heads, sU, &sh->attn_last, et,
+                                    [] __device__() { named_sync(1, 128); },
+                                    AttnBulkMerge{&sh->rbar, &r_phase, abort, (uint32_t)DIT_UNION});
+          named_sync(1, 128);
+          // the CTA that merged the head's splits publishes it
+          if (et == 0 && sh->attn_last)
+            dit_signal(P.f_head + (size_t)l * P.attn.n_heads + cta % P.attn.n_heads);
         }
       } else {
         int N, Kd;
@@ -560,7 +632,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
             tc_fence_before();
             mbar_arrive(smem_u32(&sh->tempty[acc]));
           } else {
-            float* mine = P.partial + (((size_t)z * tiles + nt) * TC_BM + r) * brows;
+            float* part = P.partial + P.part_off[kind];
+            unsigned* cnt = P.tile_cnt + kind * 1024;
+            float* mine = part + (((size_t)z * tiles + nt) * TC_BM + r) * brows;
             for (int j0 = 0; j0 < brows; j0 += 16) {
               tmem_ld16(taddr + j0, v);
 #pragma unroll
@@ -571,7 +645,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
             mbar_arrive(smem_u32(&sh->tempty[acc]));
             __threadfence();
             named_sync(1, 128);
-            if (et == 0) sh->last = (atomicAdd(&P.tile_cnt[nt], 1u) == (unsigned)(S - 1));
+            if (et == 0) sh->last = (atomicAdd(&cnt[nt], 1u) == (unsigned)(S - 1));
             named_sync(1, 128);
             if (sh->last) {
               // the S partial tiles of this output tile, one bulk copy each,
@@ -584,7 +658,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
                 mbar_expect_tx(rb, tile_bytes * S);
                 for (int zz = 0; zz < S; ++zz)
                   bulk_load(smem_u32(sU) + zz * tile_bytes,
-                            P.partial + ((size_t)zz * tiles + nt) * TC_BM * brows, tile_bytes, rb);
+                            part + ((size_t)zz * tiles + nt) * TC_BM * brows, tile_bytes, rb);
               }
               // one bounded waiter decides for all; then every thread observes
               // the completed phase itself (it cannot advance again here)
@@ -613,24 +687,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
                 if (resid) dit_epilogue_residual(P, n, v, xo, gate, xn);
                 else dit_epilogue_chunk(P, kind, l, n, j0, v, xn);
               }
-              if (et == 0) P.tile_cnt[nt] = 0u;
+              if (et == 0) cnt[nt] = 0u;
             }
           }
           const bool finished = (S == 1) || sh->last;
           if ((kind == DIT_O || kind == DIT_DOWN) && finished)
             dit_tile_stats(xn, P.M, et, sh, P.stats + (size_t)nt * P.M * 2);
           named_sync(1, 128);
+          if (finished && et == 0) {
+            if (kind == DIT_QKV) dit_signal(P.f_qkv + (size_t)l * tiles + nt);
+            else if (kind == DIT_O) dit_signal(P.c_o + l);
+            else if (kind == DIT_UP) dit_signal(P.f_up + (size_t)l * tiles + nt);
+            else dit_signal(P.c_down + l);
+          }
           if (++acc == 2) { acc = 0; acc_phase ^= 1; }
         }
       }
-      // this CTA is done with phase p
-      if (p < n_phases - 1) {
-        named_sync(1, 128);
-        if (et == 0) {
-          __threadfence();
-          atomicAdd(P.bar, 1u);
-        }
-      }
+      named_sync(1, 128);
     }
   }
 
