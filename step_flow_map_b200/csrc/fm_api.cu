@@ -608,6 +608,10 @@ fm_status dit_persistent(fm_ctx* c, const float* mods, int slot, int ctx_len, bo
   if ((size_t)g.n_heads * (s_ctx + 1) * 16 * fm::AM_PSTRIDE > c->attn_part_elems)
     return FM_ERR_UNSUPPORTED;
   am.n_ctx_splits = s_ctx;
+  // context rows this pass appends (keys/values written by its QKV phases)
+  P.attn_safe = ctx_len;
+  for (int q = 0; q < (P.n_ctx ? P.ctx_map.n_seqs : 0); ++q)
+    if (P.ctx_map.slot[q] == slot) P.attn_safe = std::min(P.attn_safe, P.ctx_map.pos0[q]);
   P.splits[fm::DIT_ATTN] = s_ctx;
   FM_CUDA(cudaMemsetAsync(c->dit_flags, 0, c->dit_flags_n * sizeof(unsigned), st));
   cudaLaunchConfig_t cfg = {};

@@ -165,6 +165,44 @@ __device__ __forceinline__ void load_rows(bf16* dst, const bf16* src, size_t ld,
   }
 }
 
+// Context rows [k0, k1) of split `split` of sequence b.
+struct AttnRange {
+  int k0, k1, n_chunks;
+  size_t base;   // element offset of (slot, row 0, head h) in the K/V caches
+};
+__device__ __forceinline__ AttnRange attn_range(const AttnMmaArgs& a, int b, int h, int split) {
+  AttnRange r;
+  const int L = a.len[b];
+  r.k0 = (int)((long)split * L / a.n_ctx_splits);
+  r.k1 = (int)((long)(split + 1) * L / a.n_ctx_splits);
+  r.n_chunks = (r.k1 - r.k0 + AM_CHUNK - 1) / AM_CHUNK;
+  r.base = (size_t)a.slot[b] * a.max_ctx * a.d + h * AM_DH;
+  return r;
+}
+
+// Issue the first ST - 1 context chunks of a split (one cp.async commit group
+// each, empty past the end) into the K/V ring.  A caller may run this before
+// the queries exist, when those rows are not written by the same pass.
+template <int N, int ST>
+__device__ __forceinline__ void attn_ctx_prologue(const bf16* __restrict__ Kc,
+                                                  const bf16* __restrict__ Vc,
+                                                  const AttnMmaArgs& a, int pair, int split,
+                                                  uint8_t* smem_raw, int tid) {
+  bf16* sK = (bf16*)smem_raw + N * 16 * AM_LD;
+  bf16* sV = sK + ST * AM_CHUNK * AM_LD;
+  const int b = pair / a.n_heads, h = pair - b * a.n_heads;
+  const AttnRange rg = attn_range(a, b, h, split);
+#pragma unroll
+  for (int c = 0; c < ST - 1; ++c) {
+    if (c < rg.n_chunks) {
+      const int r0 = rg.k0 + c * AM_CHUNK, nr = min(AM_CHUNK, rg.k1 - r0);
+      load_rows(sK + c * AM_CHUNK * AM_LD, Kc + rg.base + (size_t)r0 * a.d, a.d, nr, AM_CHUNK, tid);
+      load_rows(sV + c * AM_CHUNK * AM_LD, Vc + rg.base + (size_t)r0 * a.d, a.d, nr, AM_CHUNK, tid);
+    }
+    cp_commit();
+  }
+}
+
 // Merge of a head's split partials through shared memory: one bulk copy of
 // all partials, completing on `bar` (phase parity `phase`, flipped on use),
 // when they fit in `smem_bytes`; `abort` bounds the wait.  Without it the
@@ -185,7 +223,8 @@ __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf
                                           const bf16* __restrict__ Vc, bf16* __restrict__ out,
                                           const AttnMmaArgs& a, int pair, int split,
                                           uint8_t* smem_raw, int* s_last_p, int tid, Sync sync,
-                                          AttnBulkMerge bm = AttnBulkMerge{nullptr, nullptr, nullptr, 0}) {
+                                          AttnBulkMerge bm = AttnBulkMerge{nullptr, nullptr, nullptr, 0},
+                                          bool prologue_done = false) {
   bf16* sQ = (bf16*)smem_raw;                       // [N*16][AM_LD]
   bf16* sK = sQ + N * 16 * AM_LD;                   // [ST][AM_CHUNK][AM_LD]
   bf16* sV = sK + ST * AM_CHUNK * AM_LD;            // [ST][AM_CHUNK][AM_LD]
@@ -197,10 +236,6 @@ __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf
   const int row0 = b * a.n_noise * a.K;             // first block row of the sequence
   const int S_all = a.n_ctx_splits + 1;
   const int NQ = N * 16;
-
-  // queries of all drafts of the sequence
-  load_rows(sQ, qkv + (size_t)row0 * d3 + h * AM_DH, d3, NQ, NQ, tid);
-  cp_commit();
 
   AttnState st;
 #pragma unroll
@@ -219,11 +254,9 @@ __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf
   };
 
   if (split < a.n_ctx_splits) {
-    const int L = a.len[b];
-    const int k0 = (int)((long)split * L / a.n_ctx_splits);
-    const int k1 = (int)((long)(split + 1) * L / a.n_ctx_splits);
-    const size_t base = (size_t)a.slot[b] * a.max_ctx * a.d + h * AM_DH;
-    const int n_chunks = (k1 - k0 + AM_CHUNK - 1) / AM_CHUNK;
+    const AttnRange rg = attn_range(a, b, h, split);
+    const int k0 = rg.k0, k1 = rg.k1, n_chunks = rg.n_chunks;
+    const size_t base = rg.base;
     auto load_chunk = [&](int c) {
       const int r0 = k0 + c * AM_CHUNK, nr = min(AM_CHUNK, k1 - r0);
       const int buf = c % ST;
@@ -232,12 +265,11 @@ __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf
     };
     // one commit group per chunk (empty past the end) keeps the group count
     // fixed: ST - 1 chunks are always in flight ahead of the one used
-#pragma unroll
-    for (int c = 0; c < ST - 1; ++c) {
-      if (c < n_chunks) load_chunk(c);
-      cp_commit();
-    }
-    cp_wait<ST - 1>();   // the query group
+    if (!prologue_done) attn_ctx_prologue<N, ST>(Kc, Vc, a, pair, split, smem_raw, tid);
+    // queries of all drafts of the sequence (the newest group)
+    load_rows(sQ, qkv + (size_t)row0 * d3 + h * AM_DH, d3, NQ, NQ, tid);
+    cp_commit();
+    cp_wait<0>();
     sync();
     q_fragments();
     for (int c = 0; c < n_chunks; ++c) {
@@ -256,6 +288,7 @@ __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf
       sync();
     }
   } else {
+    load_rows(sQ, qkv + (size_t)row0 * d3 + h * AM_DH, d3, NQ, NQ, tid);
     // each draft's own block rows: keys/values of rows row0 + mt*16 .. +16
     if (sub == 0) {
       // warps sub==0 (one per draft) load their 16 rows into their own slice
@@ -322,14 +355,13 @@ __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf
       part[q * AM_PSTRIDE + AM_DH + 1] = l;
     }
   }
-  __threadfence();
   sync();
-  if (tid == 0) s_last = (atomicAdd(&a.cnt[pair], 1u) == (unsigned)(S_all - 1));
+  if (tid == 0) s_last = (atom_add_acq_rel_gpu(&a.cnt[pair], 1u) == (unsigned)(S_all - 1));
   sync();
   if (!s_last) return;
-  __threadfence();
   // ---- last CTA of this (sequence, head): merge the splits in split order,
-  // eight threads per query row (sixteen columns each)
+  // eight threads per query row, each with four float4 column groups 32
+  // columns apart (the eight lanes of a row read 128 contiguous bytes)
   const float* pp = a.part + (size_t)pair * S_all * NQ * AM_PSTRIDE;
   const uint32_t merge_bytes = (uint32_t)((size_t)S_all * NQ * AM_PSTRIDE * 4);
   const bool bulk = bm.bar != nullptr && merge_bytes <= bm.smem_bytes;
@@ -348,7 +380,7 @@ __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf
     *bm.phase ^= 1;
     pp = (const float*)smem_raw;
   }
-  const int cg = (tid & 7) * 16;
+  const int cg = (tid & 7) * 4;
   for (int q = tid >> 3; q < NQ; q += AM_THREADS / 8) {
     float o[16];
 #pragma unroll
@@ -364,11 +396,11 @@ __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf
           if (bulk) {
             ml[u2] = *(const float2*)(w + AM_DH);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) os[u2][i] = *(const float4*)(w + cg + 4 * i);
+            for (int i = 0; i < 4; ++i) os[u2][i] = *(const float4*)(w + cg + 32 * i);
           } else {
             ml[u2] = __ldcg((const float2*)(w + AM_DH));
 #pragma unroll
-            for (int i = 0; i < 4; ++i) os[u2][i] = __ldcg((const float4*)(w + cg + 4 * i));
+            for (int i = 0; i < 4; ++i) os[u2][i] = __ldcg((const float4*)(w + cg + 32 * i));
           }
         } else {
           ml[u2] = make_float2(-INFINITY, 0.f);
@@ -395,11 +427,11 @@ __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf
     }
     const float inv = 1.f / l;
     const int j = q / 16, i = q % 16;
-    uint4* dst = (uint4*)(out + (size_t)(row0 + j * a.K + i) * a.d + h * AM_DH + cg);
-    dst[0] = make_uint4(pack_bf16x2(o[0] * inv, o[1] * inv), pack_bf16x2(o[2] * inv, o[3] * inv),
-                        pack_bf16x2(o[4] * inv, o[5] * inv), pack_bf16x2(o[6] * inv, o[7] * inv));
-    dst[1] = make_uint4(pack_bf16x2(o[8] * inv, o[9] * inv), pack_bf16x2(o[10] * inv, o[11] * inv),
-                        pack_bf16x2(o[12] * inv, o[13] * inv), pack_bf16x2(o[14] * inv, o[15] * inv));
+    bf16* dst = out + (size_t)(row0 + j * a.K + i) * a.d + h * AM_DH + cg;
+#pragma unroll
+    for (int g = 0; g < 4; ++g)
+      *(uint2*)(dst + 32 * g) = make_uint2(pack_bf16x2(o[4 * g] * inv, o[4 * g + 1] * inv),
+                                           pack_bf16x2(o[4 * g + 2] * inv, o[4 * g + 3] * inv));
   }
   if (tid == 0) a.cnt[pair] = 0u;
 }

@@ -148,6 +148,19 @@ inline cudaError_t set_smem_once(F* kernel, int bytes) {
   return set_smem_once_ptr((const void*)kernel, bytes);
 }
 
+// Cross-CTA handoffs: the writing CTA orders its threads' stores with a CTA
+// barrier, then one thread publishes them with a release (cumulative over
+// what the barrier ordered before it); the reading CTA's one thread acquires
+// and a CTA barrier orders the other threads' reads after it.
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+__device__ __forceinline__ void red_add_release_gpu(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *(uint32_t*)&v;

@@ -75,6 +75,7 @@ struct DitParams {
   int max_ctx;
   RowMap ctx_map;
   AttnMmaArgs attn;                   // one sequence, one noise draft
+  int attn_safe;                      // context rows below this are not written by the pass
 };
 
 struct DitShared {                    // after the ring and the union region
@@ -170,10 +171,7 @@ __device__ __forceinline__ bool dit_wait(const DitParams& P, const unsigned* ctr
 
 // Publish one completion (thread et == 0, after the CTA's writes are ordered
 // before it by a CTA barrier).
-__device__ __forceinline__ void dit_signal(unsigned* ctr) {
-  __threadfence();
-  atomicAdd(ctr, 1u);
-}
+__device__ __forceinline__ void dit_signal(unsigned* ctr) { red_add_release_gpu(ctr, 1u); }
 
 // Waits (one thread) for everything this CTA's unit of the phase reads:
 //   QKV(l)   the residual stream after the last block (all down tiles) or the
@@ -314,7 +312,6 @@ __device__ __forceinline__ void dit_fill_b(const DitParams& P, int kind, int l, 
                                            int kb0, int nkb, int brows, int Kd, int et,
                                            DitShared* sh) {
   const bool ln = (kind == DIT_QKV || kind == DIT_UP);
-  if (ln) dit_row_stats(P, et, sh);   // ends with a barrier
   const bf16* src = kind == DIT_O ? P.o : P.u;
   const int tile_bytes = brows * 128;
   const int items = nkb * brows * 8;
@@ -345,6 +342,9 @@ __device__ __forceinline__ void dit_fill_b(const DitParams& P, int kind, int l, 
         }
       }
     }
+    // the row statistics load while the first batch is in flight (ends with
+    // a CTA barrier)
+    if (ln && i0 == 0) dit_row_stats(P, et, sh);
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int idx = i0 + u * 128 + et;
@@ -548,13 +548,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
         active = cta < (N / TC_BM) * P.splits[kind];
       }
       if (!active) continue;
+      bool kv_pre = false;
+      if (kind == DIT_ATTN) {
+        // context chunks the pass does not write load while the QKV tiles
+        // are still being produced
+        const int h = cta % P.attn.n_heads, split = cta / P.attn.n_heads;
+        if (split < P.attn.n_ctx_splits) {
+          const AttnRange rg = attn_range(P.attn, 0, h, split);
+          kv_pre = rg.k0 + min(AM_CHUNK * (DIT_ATTN_ST - 1), rg.k1 - rg.k0) <= P.attn_safe;
+          if (kv_pre) attn_ctx_prologue<1, DIT_ATTN_ST>(P.Kc[l], P.Vc[l], P.attn, h, split, sU, et);
+        }
+      }
       if (kind != -1) {
         // wait for the units whose outputs this one reads
         if (et == 0) sh->ok[it & 1] = dit_wait_deps(P, kind, l, cta) ? 1 : 0;
         named_sync(1, 128);
         if (!sh->ok[it & 1]) { *abort = 1; break; }
         ++it;
-        asm volatile("fence.acq_rel.gpu;" ::: "memory");
       }
       if (kind == -1 || kind == -2) {
         // statistics of the embedded rows (-1) or the final LayerNorm (-2):
@@ -582,7 +592,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
           attn_item<1, DIT_ATTN_ST>(P.qkv, P.Kc[l], P.Vc[l], P.o, P.attn, cta % P.attn.n_heads,
                                     cta / P.attn.n_heads, sU, &sh->attn_last, et,
                                     [] __device__() { named_sync(1, 128); },
-                                    AttnBulkMerge{&sh->rbar, &r_phase, abort, (uint32_t)DIT_UNION});
+                                    AttnBulkMerge{&sh->rbar, &r_phase, abort, (uint32_t)DIT_UNION},
+                                    kv_pre);
           named_sync(1, 128);
           // the CTA that merged the head's splits publishes it
           if (et == 0 && sh->attn_last)
@@ -634,18 +645,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
           } else {
             float* part = P.partial + P.part_off[kind];
             unsigned* cnt = P.tile_cnt + kind * 1024;
-            float* mine = part + (((size_t)z * tiles + nt) * TC_BM + r) * brows;
+            // partial tile stored [row j][feature r]: every store and every
+            // later shared-memory read is consecutive across the lanes
+            float* mine = part + ((size_t)z * tiles + nt) * TC_BM * brows + r;
             for (int j0 = 0; j0 < brows; j0 += 16) {
               tmem_ld16(taddr + j0, v);
 #pragma unroll
-              for (int j = 0; j < 16; j += 4)
-                *(float4*)(mine + j0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+              for (int j = 0; j < 16; ++j) mine[(size_t)(j0 + j) * TC_BM] = v[j];
             }
             tc_fence_before();
             mbar_arrive(smem_u32(&sh->tempty[acc]));
-            __threadfence();
             named_sync(1, 128);
-            if (et == 0) sh->last = (atomicAdd(&cnt[nt], 1u) == (unsigned)(S - 1));
+            if (et == 0) sh->last = (atom_add_acq_rel_gpu(&cnt[nt], 1u) == (unsigned)(S - 1));
             named_sync(1, 128);
             if (sh->last) {
               // the S partial tiles of this output tile, one bulk copy each,
@@ -653,7 +664,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
               const uint32_t tile_bytes = (uint32_t)(TC_BM * brows * 4);
               const uint32_t rb = smem_u32(&sh->rbar);
               if (et == 0) {
-                __threadfence();
                 asm volatile("fence.proxy.async.global;" ::: "memory");
                 mbar_expect_tx(rb, tile_bytes * S);
                 for (int zz = 0; zz < S; ++zz)
@@ -672,17 +682,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
               ++it;
               (void)mbar_wait(rb, r_phase, abort);   // returns at once
               r_phase ^= 1;
-              const float* sp = (const float*)sU + (size_t)r * brows;
+              const float* sp = (const float*)sU + r;
               for (int j0 = 0; j0 < brows; j0 += 16) {
 #pragma unroll
                 for (int j = 0; j < 16; ++j) v[j] = 0.f;
                 for (int zz = 0; zz < S; ++zz) {
-                  const float4* t4 = (const float4*)(sp + (size_t)zz * TC_BM * brows + j0);
+                  const float* t = sp + ((size_t)zz * brows + j0) * TC_BM;
 #pragma unroll
-                  for (int j = 0; j < 4; ++j) {
-                    const float4 t = t4[j];
-                    v[4 * j] += t.x; v[4 * j + 1] += t.y; v[4 * j + 2] += t.z; v[4 * j + 3] += t.w;
-                  }
+                  for (int j = 0; j < 16; ++j) v[j] += t[j * TC_BM];
                 }
                 if (resid) dit_epilogue_residual(P, n, v, xo, gate, xn);
                 else dit_epilogue_chunk(P, kind, l, n, j0, v, xn);
