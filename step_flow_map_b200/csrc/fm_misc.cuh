@@ -211,8 +211,8 @@ k_select_tokens(const float* __restrict__ logits, int V, const float* __restrict
   float mx = -INFINITY;
   for (int v = threadIdx.x; v < V; v += blockDim.x) mx = fmaxf(mx, row[v]);
   mx = block_max(mx, shv);
-  const double dm = (double)mx, dT = (double)T;
-  auto wf = [&](int v) { return exp(((double)row[v] - dm) / dT); };
+  const double dm = (double)mx, iT = 1.0 / (double)T;
+  auto wf = [&](int v) { return exp(((double)row[v] - dm) * iT); };
   double s = 0.0;
   for (int v = threadIdx.x; v < V; v += blockDim.x) s += wf(v);
   s = block_sum_d(s, shd);

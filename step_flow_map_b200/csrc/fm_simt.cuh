@@ -2,6 +2,7 @@
 // each contraction, used for small shapes).  Epilogue functors are shared
 // with the tensor-core GEMM.
 #pragma once
+#include <type_traits>
 #include "fm_common.cuh"
 
 namespace fm {
@@ -54,7 +55,25 @@ struct EpiResidual {
   __device__ __forceinline__ void operator()(int m, int n, float v) const {
     x[(size_t)m * d + n] += gate[n] * v;
   }
+  // Rows m0 .. m0 + count - 1 (count <= 16) of feature n: every load is
+  // issued before the first store, so the read-modify-writes do not
+  // serialise on memory latency.
+  __device__ __forceinline__ void chunk16(int m0, int n, const float* v, int count) const {
+    const float g = gate[n];
+    float xo[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) xo[j] = j < count ? __ldcg(x + (size_t)(m0 + j) * d + n) : 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j < count) x[(size_t)(m0 + j) * d + n] = xo[j] + g * v[j];
+  }
 };
+
+// Epilogues with a whole-chunk form (chunk16) take it in the GEMM kernels.
+template <class E>
+struct has_chunk16 : std::false_type {};
+template <>
+struct has_chunk16<EpiResidual> : std::true_type {};
 
 template <typename TO>
 struct EpiGelu {

@@ -245,6 +245,10 @@ __device__ __forceinline__ void tc_finish_chunk(const Epi& epi, const TcArgs& a,
         red_i[q * BN + j0 + j] = am.i;
       }
     }
+  } else if constexpr (has_chunk16<Epi>::value) {
+    if (n >= a.N) return;
+    const int mb = m0 + j0;
+    epi.chunk16(mb, n, v, a.M - mb < 16 ? a.M - mb : 16);
   } else {
     if (n >= a.N) return;
 #pragma unroll
@@ -493,47 +497,45 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUte
         tc_fence_before();
         mbar_arrive(smem_u32(&tempty[acc]));
       } else {
-        float* mine = a.partial + (((size_t)z * tiles + tile) * TC_BM + r) * BN;
+        // partial tile stored [activation row][feature]: stores and loads are
+        // 128 contiguous bytes per warp
+        float* mine = a.partial + ((size_t)z * tiles + tile) * TC_BM * BN + r;
         for (int j0 = 0; j0 < BN; j0 += 16) {
           tmem_ld16(taddr + j0, v);
 #pragma unroll
-          for (int j = 0; j < 16; j += 4)
-            *(float4*)(mine + j0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+          for (int j = 0; j < 16; ++j) mine[(size_t)(j0 + j) * TC_BM] = v[j];
         }
         tc_fence_before();
         mbar_arrive(smem_u32(&tempty[acc]));
-        __threadfence();
+        // the CTA barrier orders every thread's partial stores before the
+        // one acq_rel arrival; the last arrival acquires the other splits'
         named_sync(1, 128);
         if (et == 0) {
-          unsigned prev = atomicAdd(&a.tile_cnt[tile], 1u);
+          unsigned prev = atom_add_acq_rel_gpu(&a.tile_cnt[tile], 1u);
           *s_last = (prev == (unsigned)(a.splits - 1));
         }
         named_sync(1, 128);
         const int last = *s_last;
         if (last) {
-          __threadfence();
           const size_t zstride = (size_t)tiles * TC_BM * BN;
-          const float* p0 = a.partial + ((size_t)tile * TC_BM + r) * BN;
+          const float* p0 = a.partial + (size_t)tile * TC_BM * BN + r;
           for (int j0 = 0; j0 < BN; j0 += 16) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] = 0.f;
             // four splits' loads in flight at a time; sums stay in split order
             for (int zz = 0; zz < a.splits; zz += 4) {
-              float4 t[4][4];
+              float t[4][16];
 #pragma unroll
               for (int u2 = 0; u2 < 4; ++u2)
                 if (zz + u2 < a.splits)
 #pragma unroll
-                  for (int j = 0; j < 4; ++j)
-                    t[u2][j] = __ldcg((const float4*)(p0 + (zz + u2) * zstride + j0 + 4 * j));
+                  for (int j = 0; j < 16; ++j)
+                    t[u2][j] = __ldcg(p0 + (zz + u2) * zstride + (size_t)(j0 + j) * TC_BM);
 #pragma unroll
               for (int u2 = 0; u2 < 4; ++u2)
                 if (zz + u2 < a.splits)
 #pragma unroll
-                  for (int j = 0; j < 4; ++j) {
-                    v[4 * j] += t[u2][j].x; v[4 * j + 1] += t[u2][j].y;
-                    v[4 * j + 2] += t[u2][j].z; v[4 * j + 3] += t[u2][j].w;
-                  }
+                  for (int j = 0; j < 16; ++j) v[j] += t[u2][j];
             }
             tc_finish_chunk<BN>(epi, a, n0, m0, r, j0, v, red_v, red_i, q);
           }
@@ -659,11 +661,18 @@ inline bool tc_make_maps(TcMaps& m, const void* W_lm, const void* Et, const void
 }
 inline void tc_free_maps(TcMaps&) {}
 
-inline int tc_pick_bn(int M) {
+inline int tc_pick_bn(int M, int n_tiles = 0, int sms = 0, int k_blocks = 0) {
   if (M <= 16) return 16;
   if (M <= 32) return 32;
   if (M <= 64) return 64;
   if (M <= 128) return 128;
+  // 256-row activation tiles unless they leave a quarter of the SMs idle
+  // while 128-row tiles would still fit in one round (reductions up to
+  // 32K deep; the vocabulary-deep X.E keeps 256 rows and splits K)
+  if (n_tiles > 0 && sms > 0 && k_blocks <= 512) {
+    const long t256 = (long)n_tiles * ((M + 255) / 256), t128 = (long)n_tiles * ((M + 127) / 128);
+    if (4 * t256 < 3L * sms && t128 <= sms) return 128;
+  }
   return 256;
 }
 
@@ -697,6 +706,8 @@ fm_status tc_launch(const TcMap& wm, const bf16* A, int lda, int M, Epi epi, flo
   a.m_tiles = (M + BN - 1) / BN;
   a.k_blocks = (wm.Kd + TC_BK - 1) / TC_BK;
   const int tiles = a.n_tiles * a.m_tiles;
+  // K splits only while tiles leave SMs idle (measured: more splits than
+  // that lose to the serial reduction of their partial tiles)
   int splits = 1;
   if (tiles < sms) {
     splits = sms / tiles;
@@ -734,7 +745,7 @@ fm_status tc_gemm(const TcMaps& maps, const TcMap& wm, const bf16* A, int lda, i
              Kd, wm.N, wm.Kd);
     return FM_ERR_ARG;
   }
-  switch (tc_pick_bn(M)) {
+  switch (tc_pick_bn(M, (wm.N + TC_BM - 1) / TC_BM, sms, (wm.Kd + TC_BK - 1) / TC_BK)) {
     case 16: return tc_launch<16>(wm, A, lda, M, epi, partial, partial_elems, tile_cnt, tile_cnt_n, sms, maps.err, st, err, errlen, n_launch);
     case 32: return tc_launch<32>(wm, A, lda, M, epi, partial, partial_elems, tile_cnt, tile_cnt_n, sms, maps.err, st, err, errlen, n_launch);
     case 64: return tc_launch<64>(wm, A, lda, M, epi, partial, partial_elems, tile_cnt, tile_cnt_n, sms, maps.err, st, err, errlen, n_launch);

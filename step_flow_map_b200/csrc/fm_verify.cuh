@@ -105,8 +105,8 @@ k_row_stats(const float* __restrict__ tgt, const float* __restrict__ dlog, int n
   for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x) mx = fmaxf(mx, r[v]);
   mx = block_max(mx, shf);
   double s = 0.0;
-  const double dm = (double)mx, dT = (double)T;
-  for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x) s += exp(((double)r[v] - dm) / dT);
+  const double dm = (double)mx, iT = 1.0 / (double)T;
+  for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x) s += exp(((double)r[v] - dm) * iT);
   s = block_sum_d(s, shd);
   if (threadIdx.x == 0) {
     pm[(size_t)row * chunks + c] = mx;
@@ -147,7 +147,7 @@ k_verify_sample_decide(const float* __restrict__ tgt, const float* __restrict__ 
   __shared__ int s_accept, s_mode, s_buf;
   __shared__ double s_mp, s_Sp, s_mq, s_Sq;
   const int b = blockIdx.x, tid = threadIdx.x;
-  const double dT = (double)T;
+  const double dT = (double)T, iT = 1.0 / dT;   // loops over V multiply by reciprocals
   const int n_tgt_rows = B * N * (K + 1);
   double* buf[2] = {resid + (size_t)b * 2 * V, resid + (size_t)b * 2 * V + V};
   int* o = out + (size_t)b * (K + 1);
@@ -182,23 +182,25 @@ k_verify_sample_decide(const float* __restrict__ tgt, const float* __restrict__ 
       if (s_accept >= 0) break;
       // residual r = max(0, p' - q_j), then p' = r / sum(r)
       const int mode = s_mode, src = s_buf, dst = mode == 0 ? 0 : 1 - src;
-      const double mp = s_mp, Sp = s_Sp, mq = s_mq, Sq = s_Sq;
+      const double mp = s_mp, mq = s_mq;
+      const double iSp = 1.0 / s_Sp, iSq = qp ? 1.0 / s_Sq : 0.0;
       double local = 0.0;
       for (int v = tid; v < V; v += blockDim.x) {
-        double p = (mode == 0) ? exp(((double)tp[v] - mp) / dT) / Sp : buf[src][v];
-        double q = qp ? exp(((double)qp[v] - mq) / dT) / Sq : (v == y ? 1.0 : 0.0);
+        double p = (mode == 0) ? exp(((double)tp[v] - mp) * iT) * iSp : buf[src][v];
+        double q = qp ? exp(((double)qp[v] - mq) * iT) * iSq : (v == y ? 1.0 : 0.0);
         double r = fmax(p - q, 0.0);
         buf[dst][v] = r;
         local += r;
       }
       const double Z = block_sum_d(local, shd);
       if (Z > 0.0) {
-        for (int v = tid; v < V; v += blockDim.x) buf[dst][v] /= Z;
+        const double iZ = 1.0 / Z;
+        for (int v = tid; v < V; v += blockDim.x) buf[dst][v] *= iZ;
         __syncthreads();
         if (tid == 0) { s_mode = 1; s_buf = dst; }
       } else if (mode == 0) {
         // p' stays the target row itself: materialise it for later steps
-        for (int v = tid; v < V; v += blockDim.x) buf[dst][v] = exp(((double)tp[v] - mp) / dT) / Sp;
+        for (int v = tid; v < V; v += blockDim.x) buf[dst][v] = exp(((double)tp[v] - mp) * iT) * iSp;
         __syncthreads();
         if (tid == 0) { s_mode = 1; s_buf = dst; }
       }
@@ -211,8 +213,8 @@ k_verify_sample_decide(const float* __restrict__ tgt, const float* __restrict__ 
       const double u = ures[b];
       int tok;
       if (s_mode == 0) {
-        const double mp = s_mp, Sp = s_Sp;
-        auto wf = [&](int v) { return exp(((double)tp[v] - mp) / dT) / Sp; };
+        const double mp = s_mp, iSp = 1.0 / s_Sp;
+        auto wf = [&](int v) { return exp(((double)tp[v] - mp) * iT) * iSp; };
         double tot = 0.0;
         for (int v = tid; v < V; v += blockDim.x) tot += wf(v);
         tot = block_sum_d(tot, shd);
@@ -244,8 +246,8 @@ k_verify_sample_decide(const float* __restrict__ tgt, const float* __restrict__ 
       s_mp = st.m; s_Sp = st.S;
     }
     __syncthreads();
-    const double mp = s_mp, Sp = s_Sp, u = ures[b];
-    auto wf = [&](int v) { return exp(((double)tp[v] - mp) / dT) / Sp; };
+    const double mp = s_mp, iSp = 1.0 / s_Sp, u = ures[b];
+    auto wf = [&](int v) { return exp(((double)tp[v] - mp) * iT) * iSp; };
     double tot = 0.0;
     for (int v = tid; v < V; v += blockDim.x) tot += wf(v);
     tot = block_sum_d(tot, shd);
