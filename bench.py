@@ -122,6 +122,43 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- algorithmic bytes
+def source_sha1() -> str:
+    """Hash of the kernel sources; a stored ncu traffic figure is reported
+    only while it matches (the kernels have not changed since the capture)."""
+    import hashlib
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "step_flow_map_b200", "csrc")
+    for f in sorted(os.listdir(csrc)) + ["../../include/flashmap.h"]:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()
+
+
+def stored_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from profiles/traffic.txt (JSON), or None."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel, {}).get(workload)
+    if e and e.get("source_sha1") == source_sha1():
+        return e["dram_bytes_per_launch"]
+    return None
+
+
+def algorithmic_flops(w: fs.Workload):
+    """FLOPs of each kernel class per step (2 per multiply-add)."""
+    s = w.shape
+    M, V, d, F, nb = w.M, s.V, s.d, s.mlp, s.n_blocks
+    steps = len(w.t_grid) - 1
+    ctx_rows = w.ctx + w.new_rows
+    dit_params = nb * (3 * d * d + d * d + 2 * d * F)
+    attn = nb * 4 * M * (ctx_rows + s.K) * d          # QK^T and PV over context + block
+    return {"embed": 2 * M * V * d * steps, "lm_head": 2 * M * V * d * steps,
+            "dit_gemm": 2 * M * dit_params * steps, "attn": attn * steps}
+
+
 def algorithmic_bytes(w: fs.Workload):
     """Bytes each kernel class must move per step (weights, activations, caches)."""
     s = w.shape
@@ -240,26 +277,36 @@ def run_fm(args, w, rank, world, local_rank):
     log(f"{R} rounds prepared in {setup_s:.1f} s; timing")
     for k in range(args.warmup):
         step(rounds[k % R], n_acc_round[k % R], stream)
-    if args.profile_all:
-        # diagnostic: every kernel class timed with events, eager launches
-        # (the event pairs serialise neighbouring kernels)
-        fmb.fm_profile(ctx.ctx, (1 << fmb.FM_PROF_N) - 1)
-        fmb.fm_profile_read(ctx.ctx, reset=True)
-        for k in range(20):
-            step(rounds[k % R], n_acc_round[k % R], stream)
-        torch.cuda.synchronize()
-        pm, pl = fmb.fm_profile_read(ctx.ctx, reset=True)
-        fmb.fm_profile(ctx.ctx, 0)
-        for name, i in sorted(fmb.FM_PROF.items(), key=lambda x: x[1]):
-            if pl[i]:
-                log(f"profile {name:9s}: {pm[i] / 20 * 1e3:8.1f} us/step, {pl[i] / 20:.0f} launches/step")
+    # untimed eager pass with every kernel class between CUDA events (the
+    # event pairs serialise neighbours): the per-class shares, and which
+    # class dominates the step
+    n_eager = 20 if args.profile_all else 3
+    fmb.fm_profile(ctx.ctx, (1 << fmb.FM_PROF_N) - 1)
+    fmb.fm_profile_read(ctx.ctx, reset=True)
+    for k in range(n_eager):
+        step(rounds[k % R], n_acc_round[k % R], stream)
+    torch.cuda.synchronize()
+    pm, pl = fmb.fm_profile_read(ctx.ctx, reset=True)
+    fmb.fm_profile(ctx.ctx, 0)
+    eager = {name: {"us_per_step": round(pm[i] / n_eager * 1e3, 1),
+                    "launches_per_step": round(pl[i] / n_eager, 2)}
+             for name, i in fmb.FM_PROF.items() if pl[i]}
+    for name, e in eager.items():
+        log(f"eager profile {name:9s}: {e['us_per_step']:8.1f} us/step, "
+            f"{e['launches_per_step']:.0f} launches/step")
     ab = algorithmic_bytes(w)
-    prof_classes = ["embed", "lm_head"]
-    mask = sum(1 << fmb.FM_PROF[c] for c in prof_classes)
+    candidates = ["embed", "lm_head", "dit_gemm", "attn"]
+    dominant = max((c for c in candidates if c in eager), key=lambda c: eager[c]["us_per_step"])
+    # only the dominant class carries event pairs, inside the timed graphs
+    # when it has few launches per step; a class of many short launches
+    # (event pairs break their programmatic overlap) is timed in separate
+    # replays of the same step instead
+    prof_classes = [dominant]
+    mask = 1 << fmb.FM_PROF[dominant]
+    inline_events = eager[dominant]["launches_per_step"] <= 8
     barrier()
-    # one CUDA graph per distinct round; the dominant kernels carry CUDA-event
-    # pairs inside the graphs, so their timings come from the timed replays
-    fmb.fm_profile(ctx.ctx, mask)
+    # one CUDA graph per distinct round
+    fmb.fm_profile(ctx.ctx, mask if inline_events else 0)
     fmb.fm_profile_read(ctx.ctx, reset=True)
     graphs = []
     if not args.no_graph:
@@ -291,6 +338,28 @@ def run_fm(args, w, rank, world, local_rank):
         timed_steps = args.steps
     else:
         timed_steps = R   # each graph's event pairs hold its last replay
+    if not inline_events:
+        fmb.fm_profile(ctx.ctx, mask)
+        fmb.fm_profile_read(ctx.ctx, reset=True)
+        if graphs:
+            pgraphs = []
+            for i in range(R):
+                gr = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gr):
+                    step(rounds[i], n_acc_round[i], torch.cuda.current_stream())
+                pgraphs.append(gr)
+            _, cap_launches = fmb.fm_profile_read(ctx.ctx, times=False)
+            for gr in pgraphs:
+                gr.replay()
+        else:
+            for k in range(R):
+                step(rounds[k], n_acc_round[k], stream)
+        torch.cuda.synchronize()
+        prof_ms, launches = fmb.fm_profile_read(ctx.ctx, reset=True)
+        fmb.fm_profile(ctx.ctx, 0)
+        timed_steps = R
+        if graphs:
+            del pgraphs
     barrier()
     ms = max_over_ranks(ev0.elapsed_time(ev1))
     n_round = n_acc_round.sum(dim=1).cpu().numpy()
@@ -307,24 +376,53 @@ def run_fm(args, w, rank, world, local_rank):
     value = blocks / sec
     tok_per_s = verified / sec
 
-    # roofline of the dominant kernel (largest timed share)
+    # roofline of the dominant kernel class (largest timed share).  The DiT
+    # class is one persistent launch per step (block weights and the
+    # context keys/values with the attention inside it) or one launch per
+    # GEMM, reported as their mean.
     pk, pk_kind = peaks()
+    af = algorithmic_flops(w)
+    n_steps = len(w.t_grid) - 1
+    ridge = pk["bf16_tflops_sustained"] * 1e12 / (pk["hbm_gbs"] * 1e9)
     per_class = {}
     for c in prof_classes:
         i = fmb.FM_PROF[c]
-        n_launch = launches[i]
-        if prof_ms[i] > 0:
-            avg = prof_ms[i] / (timed_steps * (len(w.t_grid) - 1))
-            per_class[c] = {"ms_per_launch": avg, "bytes_per_launch": ab[f"{c}_per_launch"],
-                            "gbs": ab[f"{c}_per_launch"] / (avg / 1e3) / 1e9,
-                            "share_of_step": prof_ms[i] / timed_steps / (ms / args.steps)}
+        if prof_ms[i] <= 0 or launches[i] == 0:
+            continue
+        per_step = launches[i] / timed_steps
+        if graphs:
+            per_step = cap_launches[i] / R
+        avg = prof_ms[i] / timed_steps / per_step
+        step_b, step_f = ab[c], af.get(c, 0)
+        kern = c
+        if c == "dit_gemm" and round(per_step) == n_steps:
+            kern = "k_dit_persistent"
+            step_b += ab["attn"]
+            step_f += af["attn"]
+        b_l, f_l = step_b / per_step, step_f / per_step
+        tensor = f_l / max(b_l, 1) > ridge
+        ach = (f_l / (avg / 1e3) / 1e12) if tensor else (b_l / (avg / 1e3) / 1e9)
+        peak = pk["bf16_tflops_sustained"] if tensor else pk["hbm_gbs"]
+        per_class[c] = {"kernel": kern, "launches_per_step": round(per_step, 2),
+                        "ms_per_launch": round(avg, 5), "bytes_per_launch": int(b_l),
+                        "flops_per_launch": int(f_l), "bound": "tensor" if tensor else "hbm",
+                        "achieved": round(ach, 1), "unit": "TFLOP/s" if tensor else "GB/s",
+                        "frac": round(ach / peak, 4),
+                        "share_of_step": round(prof_ms[i] / timed_steps / (ms / args.steps), 4)}
     dom = max(per_class, key=lambda c: per_class[c]["share_of_step"]) if per_class else None
     roof = None
     if dom:
-        a = per_class[dom]["gbs"]
-        roof = {"kernel": dom, "bound": "hbm", "achieved": round(a, 1), "peak": pk["hbm_gbs"],
-                "unit": "GB/s", "frac": round(a / pk["hbm_gbs"], 4), "traffic": None,
-                "peak_kind": pk_kind + " hbm_gbs (burst copy)"}
+        e = per_class[dom]
+        tensor = e["bound"] == "tensor"
+        roof = {"kernel": e["kernel"], "bound": e["bound"], "achieved": e["achieved"],
+                "peak": pk["bf16_tflops_sustained"] if tensor else pk["hbm_gbs"],
+                "unit": e["unit"], "frac": e["frac"],
+                "traffic": stored_traffic(e["kernel"], w.name),
+                "algorithmic_per_launch": e["flops_per_launch"] if tensor else e["bytes_per_launch"],
+                "peak_kind": pk_kind + (" bf16_tflops_sustained (kernel timed inside a long step)"
+                                        if tensor else " hbm_gbs (copy)"),
+                "timing": ("CUDA events inside the timed replays" if inline_events else
+                           "CUDA events in separate replays of the same steps")}
     step_bytes = sum(ab[k] for k in ("embed", "lm_head", "dit_gemm", "attn", "context", "verify"))
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "blocks/s", "n_gpus": world,
@@ -341,6 +439,7 @@ def run_fm(args, w, rank, world, local_rank):
         "step_hbm_gbs": round(step_bytes / (ms / args.steps / 1e3) / 1e9, 1),
         "step_hbm_frac": round(step_bytes / (ms / args.steps / 1e3) / 1e9 / pk["hbm_gbs"], 4),
         "roofline": roof, "kernels": per_class,
+        "eager_profile_us_per_step": {k: v["us_per_step"] for k, v in eager.items()},
         "gpu_launches": int(round(launches_per_step * args.steps)),
         "cuda_graphs": bool(graphs),
         "clocks": clk.summary(), "setup_s": round(setup_s, 1),

@@ -16,6 +16,7 @@ Princeton выпустили FlashMap", section "Как работает FlashMa
 * ``qwen3_8b_bs1``  as above with hidden 4096, ctx 1024 (the concurrency-1 bench)
 * ``qwen3_8b_2step_tree4``  two steps (0, 0.5, 1), 4 noise drafts, T=1, ctx 2048
 * ``qwen3_8b_bs64`` 64 sequences, ctx 4096, 32 greedy + 32 sampled at T=1
+* ``qwen3_8b_bs64_ctx256`` the same with 256 context rows (profiler captures)
 
 Seeds: weights use ``1000 + tensor_index``; round ``r`` draws its noise from
 ``2000 + r``, its new context rows from ``3000 + r``, its target-logit
@@ -125,6 +126,12 @@ WORKLOADS = {
         "qwen3_8b_bs64", QWEN3_8B, "bf16", B=64, n_noise=1, ctx=4096, new_rows=17,
         t_grid=(0.0, 1.0), temps=tuple([0.0] * 32 + [1.0] * 32), target="near_draft",
         target_std=1.5, rounds=1, description="64 sequences x K=16, mixed greedy / T=1"),
+    # the same M = 1024 GEMMs with 256 context rows: small enough on the
+    # device for a full-metric profiler capture
+    "qwen3_8b_bs64_ctx256": Workload(
+        "qwen3_8b_bs64_ctx256", QWEN3_8B, "bf16", B=64, n_noise=1, ctx=256, new_rows=17,
+        t_grid=(0.0, 1.0), temps=tuple([0.0] * 32 + [1.0] * 32), target="near_draft",
+        target_std=1.5, rounds=1, description="as qwen3_8b_bs64 with 256 context rows"),
 }
 
 

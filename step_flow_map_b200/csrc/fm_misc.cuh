@@ -99,72 +99,106 @@ k_softmax_rows(const float* __restrict__ logits, int V, TO* __restrict__ D) {
 }
 
 // ------------------------------------------------------------------ inverse CDF
-// Smallest v whose running sum of w(v), in vocabulary order, exceeds
-// `target`; if rounding leaves none, the last v with w(v) > 0.  Each thread
-// owns one contiguous chunk; chunk sums are scanned across the block in fp64
-// and the owning chunk is rescanned.  All threads return the answer.
+// One pass over the row: the smallest v whose running sum of w(v), in
+// vocabulary order, exceeds u * total, where total is the sum of all w(v);
+// if rounding leaves none, the last v with w(v) > 0.  Warp i sums segment i
+// of the row (its lanes strided, so loads are coalesced) while the total
+// forms; only the segment holding u * total is read again, by its warp with
+// each lane on a contiguous sub-chunk, and then the owning sub-chunk by its
+// lane.  blockDim.x is a multiple of 32, at most 1024.  All threads return
+// the answer.
 template <class WF>
-__device__ int block_inverse_cdf(const WF& w, int V, double target) {
-  __shared__ double wsum[32];
-  __shared__ int found;
-  __shared__ int lastpos;
-  const int nt = blockDim.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  const int chunk = (V + nt - 1) / nt;
-  const int v0 = min(V, tid * chunk), v1 = min(V, v0 + chunk);
-  double local = 0.0;
+__device__ int block_sample(const WF& w, int V, double u) {
+  __shared__ double seg_sum[32];
+  __shared__ double s_base, s_target;
+  __shared__ int s_last, s_owner, s_pick;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nw = blockDim.x >> 5;
+  const int seg = ((V + nw - 1) / nw + 31) / 32 * 32;   // a multiple of 32
+  const int s0 = min(V, wid * seg), s1 = min(V, s0 + seg);
+  if (tid == 0) {
+    s_last = -1;
+    s_pick = -1;
+  }
+  __syncthreads();
+  double acc = 0.0;
   int last = -1;
-  for (int v = v0; v < v1; ++v) {
-    double x = w(v);
-    local += x;
+  for (int v = s0 + lane; v < s1; v += 32) {
+    const double x = w(v);
+    acc += x;
     if (x > 0.0) last = v;
   }
-  // inclusive warp scan, then across warps
-  double incl = local;
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    double y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
+  for (int o = 16; o > 0; o >>= 1) {
+    acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
   }
-  if (tid == 0) { found = 0x7fffffff; lastpos = -1; }
-  if (lane == 31) wsum[wid] = incl;
+  if (lane == 0) {
+    seg_sum[wid] = acc;
+    if (last >= 0) atomicMax(&s_last, last);
+  }
   __syncthreads();
-  if (wid == 0) {
-    int nw = (nt + 31) >> 5;
-    double t = (lane < nw) ? wsum[lane] : 0.0;
+  if (tid == 0) {
+    double tot = 0.0;
+    for (int i = 0; i < nw; ++i) tot += seg_sum[i];
+    const double target = u * tot;
+    double pre = 0.0;
+    int own = -1;
+    for (int i = 0; i < nw; ++i) {
+      if (pre + seg_sum[i] > target) {
+        own = i;
+        break;
+      }
+      pre += seg_sum[i];
+    }
+    s_owner = own;
+    s_base = pre;
+    s_target = target;
+  }
+  __syncthreads();
+  const int own = s_owner;
+  if (own >= 0 && wid == own) {
+    const int L = seg / 32;
+    const int c0 = min(s1, s0 + lane * L), c1 = min(s1, c0 + L);
+    double sub = 0.0;
+    int lp = -1;
+    for (int v = c0; v < c1; ++v) {
+      const double x = w(v);
+      sub += x;
+      if (x > 0.0) lp = v;
+    }
+    double incl = sub;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      double y = __shfl_up_sync(0xffffffffu, t, o);
-      if (lane >= o) t += y;
+      const double y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
     }
-    if (lane < nw) wsum[lane] = t;  // inclusive totals per warp
-  }
-  __syncthreads();
-  if (wid > 0) incl += wsum[wid - 1];
-  double prev = __shfl_up_sync(0xffffffffu, incl, 1);
-  if (lane == 0) prev = (wid > 0) ? wsum[wid - 1] : 0.0;
-  if (incl > target && v1 > v0) atomicMin(&found, tid);
-  if (last >= 0) atomicMax(&lastpos, last);
-  __syncthreads();
-  __shared__ int pick_sh;
-  const int owner = found;
-  if (owner != 0x7fffffff) {
-    if (tid == owner) {
-      double r = 0.0;
-      int pick = -1, lp = -1;
-      for (int v = v0; v < v1; ++v) {
-        double x = w(v);
-        r += x;
-        if (x > 0.0) lp = v;
-        if (prev + r > target) { pick = v; break; }
+    const double base = s_base, target = s_target;
+    const unsigned hit = __ballot_sync(0xffffffffu, base + incl > target);
+    int seg_last = lp;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) seg_last = max(seg_last, __shfl_xor_sync(0xffffffffu, seg_last, o));
+    if (hit) {
+      if (lane == __ffs(hit) - 1) {
+        double r = base + incl - sub;   // mass before this sub-chunk
+        int pick = -1, lq = -1;
+        for (int v = c0; v < c1; ++v) {
+          const double x = w(v);
+          r += x;
+          if (x > 0.0) lq = v;
+          if (r > target) {
+            pick = v;
+            break;
+          }
+        }
+        s_pick = pick >= 0 ? pick : (lq >= 0 ? lq : c0);   // rounding at the sub-chunk end
       }
-      if (pick < 0) pick = lp >= 0 ? lp : v0;  // rounding tie at the chunk end
-      pick_sh = pick;
+    } else if (lane == 0) {
+      s_pick = seg_last;   // rounding: the segment's strided sum said it holds the target
     }
-  } else if (tid == 0) {
-    pick_sh = lastpos >= 0 ? lastpos : 0;
   }
   __syncthreads();
-  const int ans = pick_sh;
+  int ans = s_pick;
+  if (ans < 0) ans = s_last >= 0 ? s_last : 0;
   __syncthreads();
   return ans;
 }
@@ -186,7 +220,6 @@ k_select_tokens(const float* __restrict__ logits, int V, const float* __restrict
   pdl_trigger();
   __shared__ float shv[32];
   __shared__ int shi[32];
-  __shared__ double shd[32];
   const int m = blockIdx.x;
   const int q = m / (ta.n_noise * ta.K);
   const float T = ta.temp[q];
@@ -207,16 +240,14 @@ k_select_tokens(const float* __restrict__ logits, int V, const float* __restrict
     if (threadIdx.x == 0) tokens[m] = (a.i == 0x7fffffff) ? 0 : a.i;
     return;
   }
+  // weights exp((l - max)/T) in fp32, accumulated in fp64
   const float* row = logits + (size_t)m * V;
   float mx = -INFINITY;
   for (int v = threadIdx.x; v < V; v += blockDim.x) mx = fmaxf(mx, row[v]);
   mx = block_max(mx, shv);
-  const double dm = (double)mx, iT = 1.0 / (double)T;
-  auto wf = [&](int v) { return exp(((double)row[v] - dm) * iT); };
-  double s = 0.0;
-  for (int v = threadIdx.x; v < V; v += blockDim.x) s += wf(v);
-  s = block_sum_d(s, shd);
-  int tok = block_inverse_cdf(wf, V, u[m] * s);
+  const float iT = 1.f / T;
+  auto wf = [&](int v) { return (double)expf((row[v] - mx) * iT); };
+  int tok = block_sample(wf, V, u[m]);
   if (threadIdx.x == 0) tokens[m] = tok;
 }
 

@@ -132,7 +132,7 @@ __device__ __forceinline__ RowStat combine_stats(const float* pm, const double* 
 // Pass 2: one CTA per sequence walks the depths.  Residual distributions
 // are materialised, normalised, in a per-sequence fp64 ping-pong buffer
 // [2][V]; a residual whose mass rounds to zero leaves p' unchanged.
-constexpr int VS_DECIDE_THREADS = 1024;
+constexpr int VS_DECIDE_THREADS = 512;
 
 __global__ void __launch_bounds__(VS_DECIDE_THREADS)
 k_verify_sample_decide(const float* __restrict__ tgt, const float* __restrict__ dlog,
@@ -215,17 +215,11 @@ k_verify_sample_decide(const float* __restrict__ tgt, const float* __restrict__ 
       if (s_mode == 0) {
         const double mp = s_mp, iSp = 1.0 / s_Sp;
         auto wf = [&](int v) { return exp(((double)tp[v] - mp) * iT) * iSp; };
-        double tot = 0.0;
-        for (int v = tid; v < V; v += blockDim.x) tot += wf(v);
-        tot = block_sum_d(tot, shd);
-        tok = block_inverse_cdf(wf, V, u * tot);
+        tok = block_sample(wf, V, u);
       } else {
         const double* pb = buf[s_buf];
         auto wf = [&](int v) { return pb[v]; };
-        double tot = 0.0;
-        for (int v = tid; v < V; v += blockDim.x) tot += pb[v];
-        tot = block_sum_d(tot, shd);
-        tok = block_inverse_cdf(wf, V, u * tot);
+        tok = block_sample(wf, V, u);
       }
       if (tid == 0) o[i] = tok;
       n_done = i;
@@ -248,10 +242,7 @@ k_verify_sample_decide(const float* __restrict__ tgt, const float* __restrict__ 
     __syncthreads();
     const double mp = s_mp, iSp = 1.0 / s_Sp, u = ures[b];
     auto wf = [&](int v) { return exp(((double)tp[v] - mp) * iT) * iSp; };
-    double tot = 0.0;
-    for (int v = tid; v < V; v += blockDim.x) tot += wf(v);
-    tot = block_sum_d(tot, shd);
-    int tok = block_inverse_cdf(wf, V, u * tot);
+    int tok = block_sample(wf, V, u);
     if (tid == 0) o[K] = tok;
   } else {
     r0 = __ffs(alive) - 1;
