@@ -85,6 +85,7 @@ struct DitShared {                    // after the ring and the union region
   float stat[2 * DIT_BROWS_MAX];      // mean, rstd per row
   float ss[2][1024];                  // shift, scale of this CTA's column slice
   float red[4][DIT_M][2];             // per-warp row partials
+  int ctx_row[DIT_BROWS_MAX];         // cache row (slot * max_ctx + position) of each appended context row
 };
 
 static_assert(sizeof(DitShared) + 16 <= 12288, "shared bookkeeping region");
@@ -311,58 +312,98 @@ __device__ __forceinline__ void dit_stage_mods(const DitParams& P, int kind, int
 __device__ __forceinline__ void dit_fill_b(const DitParams& P, int kind, int l, uint8_t* sB,
                                            int kb0, int nkb, int brows, int Kd, int et,
                                            DitShared* sh) {
-  const bool ln = (kind == DIT_QKV || kind == DIT_UP);
-  const bf16* src = kind == DIT_O ? P.o : P.u;
+  // one loop per kind of row, so each unrolled batch holds one code path
   const int tile_bytes = brows * 128;
-  const int items = nkb * brows * 8;
-  // eight items per thread and batch: every load of a batch is in flight
-  // before any is used
-  for (int i0 = 0; i0 < items; i0 += 128 * 8) {
-    float4 xa[8], xb[8];
-    uint4 cp[8];
+  const int M = P.M;
+  auto put = [&](int kbi, int row, int ch, uint4 packed) {
+    *(uint4*)(sB + kbi * tile_bytes + row * 128 + ((ch ^ (row & 7)) << 4)) = packed;
+  };
+  if (kind == DIT_QKV || kind == DIT_UP) {
+    // block rows: LN0(x)(1 + scale) + shift, eight items per thread and
+    // batch with every load of the batch in flight before any is used
+    const int items = nkb * M * 8;
+    for (int i0 = 0; i0 < items; i0 += 128 * 8) {
+      float4 xa[8], xb[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int idx = i0 + u * 128 + et;
-      const int kbi = idx / (brows * 8), rem = idx - kbi * (brows * 8);
-      const int row = rem >> 3, ch = rem & 7;
-      const int col = (kb0 + kbi) * TC_BK + ch * 8;
-      cp[u] = make_uint4(0, 0, 0, 0);
-      xa[u] = xb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (idx < items && col < Kd) {
-        if (row < P.M) {
-          if (ln) {
-            const float* xr = P.x + (size_t)row * P.d + col;
-            xa[u] = __ldcg((const float4*)xr);
-            xb[u] = __ldcg((const float4*)(xr + 4));
-          } else {
-            cp[u] = __ldcg((const uint4*)(src + (size_t)row * Kd + col));
-          }
-        } else if (kind == DIT_QKV && row - P.M < P.n_ctx) {
-          cp[u] = __ldcg((const uint4*)(P.ctx_rows + (size_t)(row - P.M) * P.d + col));
+      for (int u = 0; u < 8; ++u) {
+        const int idx = i0 + u * 128 + et;
+        const int kbi = idx / (M * 8), rem = idx - kbi * (M * 8);
+        const int row = rem >> 3, col = (kb0 + kbi) * TC_BK + (rem & 7) * 8;
+        xa[u] = xb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (idx < items && col < Kd) {
+          const float* xr = P.x + (size_t)row * P.d + col;
+          xa[u] = __ldcg((const float4*)xr);
+          xb[u] = __ldcg((const float4*)(xr + 4));
         }
       }
-    }
-    // the row statistics load while the first batch is in flight (ends with
-    // a CTA barrier)
-    if (ln && i0 == 0) dit_row_stats(P, et, sh);
+      // the row statistics load while the first batch is in flight (ends
+      // with a CTA barrier)
+      if (i0 == 0) dit_row_stats(P, et, sh);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int idx = i0 + u * 128 + et;
-      if (idx >= items) break;
-      const int kbi = idx / (brows * 8), rem = idx - kbi * (brows * 8);
-      const int row = rem >> 3, ch = rem & 7;
-      const int cc = kbi * TC_BK + ch * 8;  // column within this CTA's slice
-      uint4 packed = cp[u];
-      if (ln && row < P.M) {
+      for (int u = 0; u < 8; ++u) {
+        const int idx = i0 + u * 128 + et;
+        if (idx >= items) break;
+        const int kbi = idx / (M * 8), rem = idx - kbi * (M * 8);
+        const int row = rem >> 3, ch = rem & 7;
+        const int cc = kbi * TC_BK + ch * 8;  // column within this CTA's slice
         const float mean = sh->stat[row], rstd = sh->stat[DIT_BROWS_MAX + row];
         const float* h = sh->ss[0] + cc;
         const float* c = sh->ss[1] + cc;
+        uint4 packed;
         packed.x = pack_bf16x2((xa[u].x - mean) * rstd * (1.f + c[0]) + h[0], (xa[u].y - mean) * rstd * (1.f + c[1]) + h[1]);
         packed.y = pack_bf16x2((xa[u].z - mean) * rstd * (1.f + c[2]) + h[2], (xa[u].w - mean) * rstd * (1.f + c[3]) + h[3]);
         packed.z = pack_bf16x2((xb[u].x - mean) * rstd * (1.f + c[4]) + h[4], (xb[u].y - mean) * rstd * (1.f + c[5]) + h[5]);
         packed.w = pack_bf16x2((xb[u].z - mean) * rstd * (1.f + c[6]) + h[6], (xb[u].w - mean) * rstd * (1.f + c[7]) + h[7]);
+        put(kbi, row, ch, packed);
       }
-      *(uint4*)(sB + kbi * tile_bytes + row * 128 + ((ch ^ (row & 7)) << 4)) = packed;
+    }
+    // rows after the block: appended context rows (already normalised),
+    // then zeros up to brows
+    const int xrows = brows - M;
+    if (xrows > 0) {
+      const int items_x = nkb * xrows * 8;
+      for (int i0 = 0; i0 < items_x; i0 += 128 * 8) {
+        uint4 cp[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int idx = i0 + u * 128 + et;
+          const int kbi = idx / (xrows * 8), rem = idx - kbi * (xrows * 8);
+          const int r = rem >> 3, col = (kb0 + kbi) * TC_BK + (rem & 7) * 8;
+          cp[u] = make_uint4(0, 0, 0, 0);
+          if (idx < items_x && r < P.n_ctx && col < Kd)
+            cp[u] = __ldcg((const uint4*)(P.ctx_rows + (size_t)r * P.d + col));
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int idx = i0 + u * 128 + et;
+          if (idx >= items_x) break;
+          const int kbi = idx / (xrows * 8), rem = idx - kbi * (xrows * 8);
+          put(kbi, M + (rem >> 3), rem & 7, cp[u]);
+        }
+      }
+    }
+  } else {
+    // copied rows: attention output (O) or MLP hidden (down)
+    const bf16* src = kind == DIT_O ? P.o : P.u;
+    const int items = nkb * brows * 8;
+    for (int i0 = 0; i0 < items; i0 += 128 * 8) {
+      uint4 cp[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int idx = i0 + u * 128 + et;
+        const int kbi = idx / (brows * 8), rem = idx - kbi * (brows * 8);
+        const int row = rem >> 3, col = (kb0 + kbi) * TC_BK + (rem & 7) * 8;
+        cp[u] = make_uint4(0, 0, 0, 0);
+        if (idx < items && row < M && col < Kd)
+          cp[u] = __ldcg((const uint4*)(src + (size_t)row * Kd + col));
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int idx = i0 + u * 128 + et;
+        if (idx >= items) break;
+        const int kbi = idx / (brows * 8), rem = idx - kbi * (brows * 8);
+        put(kbi, rem >> 3, rem & 7, cp[u]);
+      }
     }
   }
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -371,24 +412,29 @@ __device__ __forceinline__ void dit_fill_b(const DitParams& P, int kind, int l, 
 // Final epilogue of one 128-feature tile with the reduced accumulators v
 // (column j of the chunk j0 .. j0+15 = B row j0 + j).
 __device__ __forceinline__ void dit_epilogue_chunk(const DitParams& P, int kind, int l, int n,
-                                                   int j0, const float* v, float* xn) {
+                                                   int j0, const float* v, const int* ctx_row) {
   const int d = P.d;
+  if (kind == DIT_QKV) {
+    if (j0 < P.M) {
+      // block rows (P.M = 16: the whole chunk)
+      bf16* q = P.qkv + (size_t)j0 * 3 * d + n;
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const int m = j0 + j;
-    if (kind == DIT_QKV) {
-      if (m < P.M) {
-        P.qkv[(size_t)m * 3 * d + n] = __float2bfloat16_rn(v[j]);
-      } else if (m - P.M < P.n_ctx && n >= d) {
-        const int r = m - P.M;
-        const int q = r / P.ctx_map.n_new, k = r - q * P.ctx_map.n_new;
-        const size_t row = (size_t)P.ctx_map.slot[q] * P.max_ctx + P.ctx_map.pos0[q] + k;
-        if (n < 2 * d) P.Kc[l][row * d + n - d] = __float2bfloat16_rn(v[j]);
-        else P.Vc[l][row * d + n - 2 * d] = __float2bfloat16_rn(v[j]);
+      for (int j = 0; j < 16; ++j)
+        if (j0 + j < P.M) q[(size_t)j * 3 * d] = __float2bfloat16_rn(v[j]);
+    } else if (n >= d) {
+      // appended context rows: keys and values into the cache (queries dropped)
+      bf16* c = n < 2 * d ? P.Kc[l] + (n - d) : P.Vc[l] + (n - 2 * d);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int r = j0 + j - P.M;
+        if (r < P.n_ctx) c[(size_t)ctx_row[r] * d] = __float2bfloat16_rn(v[j]);
       }
-    } else if (kind == DIT_UP) {
-      if (m < P.M) P.u[(size_t)m * P.F + n] = __float2bfloat16_rn(gelu_tanh(v[j]));
     }
+  } else {
+    bf16* u = P.u + (size_t)j0 * P.F + n;
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j0 + j < P.M) u[(size_t)j * P.F] = __float2bfloat16_rn(gelu_tanh(v[j]));
   }
 }
 
@@ -519,6 +565,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
     const int et = threadIdx.x - 64;
     const int q = warp & 3;
     const int r = q * 32 + lane;          // feature row within a 128-row weight tile
+    if (et < P.n_ctx) {
+      const int cq = et / P.ctx_map.n_new, ck = et - cq * P.ctx_map.n_new;
+      sh->ctx_row[et] = P.ctx_map.slot[cq] * P.max_ctx + P.ctx_map.pos0[cq] + ck;
+    }
+    named_sync(1, 128);
     int acc = 0;
     uint32_t acc_phase = 0, r_phase = 0;
     int it = 0;
@@ -638,7 +689,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
             for (int j0 = 0; j0 < brows; j0 += 16) {
               tmem_ld16(taddr + j0, v);
               if (resid) dit_epilogue_residual(P, n, v, xo, gate, xn);
-              else dit_epilogue_chunk(P, kind, l, n, j0, v, xn);
+              else dit_epilogue_chunk(P, kind, l, n, j0, v, sh->ctx_row);
             }
             tc_fence_before();
             mbar_arrive(smem_u32(&sh->tempty[acc]));
@@ -692,7 +743,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
                   for (int j = 0; j < 16; ++j) v[j] += t[j * TC_BM];
                 }
                 if (resid) dit_epilogue_residual(P, n, v, xo, gate, xn);
-                else dit_epilogue_chunk(P, kind, l, n, j0, v, xn);
+                else dit_epilogue_chunk(P, kind, l, n, j0, v, sh->ctx_row);
               }
               if (et == 0) cnt[nt] = 0u;
             }
