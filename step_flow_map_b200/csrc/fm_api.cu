@@ -607,6 +607,8 @@ fm_status dit_persistent(fm_ctx* c, const float* mods, int slot, int ctx_len, bo
   if (g.n_heads * (s_ctx + 1) > G) return FM_ERR_UNSUPPORTED;
   if ((size_t)g.n_heads * (s_ctx + 1) * 16 * fm::AM_PSTRIDE > c->attn_part_elems)
     return FM_ERR_UNSUPPORTED;
+  // a head's split partials are merged in shared memory
+  if ((size_t)(s_ctx + 1) * 16 * fm::AM_PSTRIDE * 4 > (size_t)fm::DIT_UNION) return FM_ERR_UNSUPPORTED;
   am.n_ctx_splits = s_ctx;
   // context rows this pass appends (keys/values written by its QKV phases)
   P.attn_safe = ctx_len;

@@ -15,6 +15,7 @@
 // (sequence, head) -- arrival counter, no waiting -- merges the partials in
 // split order and writes O / l as bf16.
 #pragma once
+#include <type_traits>
 #include "fm_common.cuh"
 #include "fm_tc.cuh"
 
@@ -203,10 +204,12 @@ __device__ __forceinline__ void attn_ctx_prologue(const bf16* __restrict__ Kc,
   }
 }
 
-// Merge of a head's split partials through shared memory: one bulk copy of
-// all partials, completing on `bar` (phase parity `phase`, flipped on use),
-// when they fit in `smem_bytes`; `abort` bounds the wait.  Without it the
-// merging CTA reads the partials from global memory directly.
+// Merge of a head's split partials through shared memory (BULK items): one
+// bulk copy of all partials, completing on `bar` (phase parity `phase`,
+// flipped on use); they must fit in `smem_bytes` (the caller checks; a
+// merge that would not fit sets `abort` and is skipped); `abort` also bounds
+// the wait.  Without BULK the merging CTA reads the partials from global
+// memory directly.
 struct AttnBulkMerge {
   uint64_t* bar;
   uint32_t* phase;
@@ -218,7 +221,7 @@ struct AttnBulkMerge {
 // AM_THREADS threads (tid 0..AM_THREADS-1, four whole warps) that
 // synchronise with `sync()`.  ST context chunks are in flight; `smem_raw`
 // holds attn_mma_smem<N, ST>() bytes; `s_last` is one shared int.
-template <int N, int ST, class Sync>
+template <int N, int ST, bool BULK, class Sync>
 __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc,
                                           const bf16* __restrict__ Vc, bf16* __restrict__ out,
                                           const AttnMmaArgs& a, int pair, int split,
@@ -364,8 +367,14 @@ __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf
   // columns apart (the eight lanes of a row read 128 contiguous bytes)
   const float* pp = a.part + (size_t)pair * S_all * NQ * AM_PSTRIDE;
   const uint32_t merge_bytes = (uint32_t)((size_t)S_all * NQ * AM_PSTRIDE * 4);
-  const bool bulk = bm.bar != nullptr && merge_bytes <= bm.smem_bytes;
-  if (bulk) {
+  if constexpr (BULK) {
+    if (merge_bytes > bm.smem_bytes) {
+      if (tid == 0) {
+        *bm.abort = 1;
+        s_last = 0;   // nothing merged: the caller must not publish the head
+      }
+      return;
+    }
     // all partials of the pair are contiguous: one copy into shared memory
     const uint32_t mb = (uint32_t)__cvta_generic_to_shared(bm.bar);
     if (tid == 0) {
@@ -393,7 +402,7 @@ __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf
       for (int u2 = 0; u2 < 4; ++u2) {
         if (s0 + u2 < S_all) {
           const float* w = pp + ((size_t)(s0 + u2) * NQ + q) * AM_PSTRIDE;
-          if (bulk) {
+          if constexpr (BULK) {
             ml[u2] = *(const float2*)(w + AM_DH);
 #pragma unroll
             for (int i = 0; i < 4; ++i) os[u2][i] = *(const float4*)(w + cg + 32 * i);
@@ -444,7 +453,7 @@ k_attn_mma(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc, const bf16
   pdl_trigger();
   extern __shared__ __align__(16) uint8_t smem_raw[];
   __shared__ int s_last;
-  attn_item<N, AM_STAGES>(qkv, Kc, Vc, out, a, blockIdx.x, blockIdx.y, smem_raw, &s_last, threadIdx.x,
+  attn_item<N, AM_STAGES, false>(qkv, Kc, Vc, out, a, blockIdx.x, blockIdx.y, smem_raw, &s_last, threadIdx.x,
                [] __device__() { __syncthreads(); });
 }
 

@@ -640,7 +640,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
       } else if (kind == DIT_ATTN) {
         const int items = P.attn.n_heads * (P.attn.n_ctx_splits + 1);
         if (cta < items) {
-          attn_item<1, DIT_ATTN_ST>(P.qkv, P.Kc[l], P.Vc[l], P.o, P.attn, cta % P.attn.n_heads,
+          attn_item<1, DIT_ATTN_ST, true>(P.qkv, P.Kc[l], P.Vc[l], P.o, P.attn, cta % P.attn.n_heads,
                                     cta / P.attn.n_heads, sU, &sh->attn_last, et,
                                     [] __device__() { named_sync(1, 128); },
                                     AttnBulkMerge{&sh->rbar, &r_phase, abort, (uint32_t)DIT_UNION},
