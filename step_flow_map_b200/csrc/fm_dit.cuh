@@ -84,7 +84,6 @@ struct DitShared {                    // after the ring and the union region
   int abort, last, ok[2], attn_last;
   float stat[2 * DIT_BROWS_MAX];      // mean, rstd per row
   float ss[2][1024];                  // shift, scale of this CTA's column slice
-  float red[4][DIT_M][2];             // per-warp row partials
   int ctx_row[DIT_BROWS_MAX];         // cache row (slot * max_ctx + position) of each appended context row
 };
 
@@ -211,33 +210,41 @@ __device__ bool dit_wait_deps(const DitParams& P, int kind, int l, int cta) {
 }
 
 // Per-row mean and sum of squared deviations over the 128 features held by
-// the 128 epilogue threads (thread et holds feature et of every row).
-__device__ __forceinline__ void dit_tile_stats(const float* v, int M, int et, DitShared* sh,
+// the 128 epilogue threads (thread et holds feature et of every row):
+// transposed through shared memory `buf` [16][136] (the row stride keeps the
+// reads free of bank conflicts), then eight threads per row, each summing
+// sixteen features, combine with three shuffles.  Ends with a CTA barrier.
+constexpr int DIT_TS_LD = 136;
+constexpr int DIT_TS_BYTES = DIT_M * DIT_TS_LD * 4;
+__device__ __forceinline__ void dit_tile_stats(const float* v, int M, int et, float* buf,
                                                float* out /* [M][2] */) {
-  const int w = et >> 5, lane = et & 31;
-  float s[DIT_M];
 #pragma unroll
-  for (int j = 0; j < DIT_M; ++j) s[j] = warp_sum(j < M ? v[j] : 0.f);
-  if (lane == 0)
-#pragma unroll
-    for (int j = 0; j < DIT_M; ++j) sh->red[w][j][0] = s[j];
+  for (int j = 0; j < DIT_M; ++j) buf[j * DIT_TS_LD + et] = j < M ? v[j] : 0.f;
   named_sync(1, 128);
-  float mean[DIT_M];
+  const int row = et >> 3, g = et & 7;
+  float x[16];
+  float s = 0.f;
 #pragma unroll
-  for (int j = 0; j < DIT_M; ++j)
-    mean[j] = (sh->red[0][j][0] + sh->red[1][j][0] + sh->red[2][j][0] + sh->red[3][j][0]) / 128.f;
-#pragma unroll
-  for (int j = 0; j < DIT_M; ++j) {
-    const float dv = j < M ? v[j] - mean[j] : 0.f;
-    s[j] = warp_sum(dv * dv);
+  for (int i = 0; i < 16; ++i) {
+    x[i] = buf[row * DIT_TS_LD + i * 8 + g];
+    s += x[i];
   }
-  if (lane == 0)
+  s += __shfl_xor_sync(0xffffffffu, s, 1);
+  s += __shfl_xor_sync(0xffffffffu, s, 2);
+  s += __shfl_xor_sync(0xffffffffu, s, 4);
+  const float mean = s * (1.f / 128.f);
+  float q = 0.f;
 #pragma unroll
-    for (int j = 0; j < DIT_M; ++j) sh->red[w][j][1] = s[j];
-  named_sync(1, 128);
-  if (et < M) {
-    out[et * 2] = mean[et];
-    out[et * 2 + 1] = sh->red[0][et][1] + sh->red[1][et][1] + sh->red[2][et][1] + sh->red[3][et][1];
+  for (int i = 0; i < 16; ++i) {
+    const float dv = x[i] - mean;
+    q = fmaf(dv, dv, q);
+  }
+  q += __shfl_xor_sync(0xffffffffu, q, 1);
+  q += __shfl_xor_sync(0xffffffffu, q, 2);
+  q += __shfl_xor_sync(0xffffffffu, q, 4);
+  if (g == 0 && row < M) {
+    out[row * 2] = mean;
+    out[row * 2 + 1] = q;
   }
   named_sync(1, 128);
 }
@@ -626,7 +633,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
             float v[DIT_M];
 #pragma unroll
             for (int j = 0; j < DIT_M; ++j) v[j] = j < P.M ? __ldcg(P.x + (size_t)j * P.d + n) : 0.f;
-            dit_tile_stats(v, P.M, et, sh, P.stats + (size_t)cta * P.M * 2);
+            dit_tile_stats(v, P.M, et, (float*)(sU + DIT_UNION - DIT_TS_BYTES),
+                           P.stats + (size_t)cta * P.M * 2);
             if (et == 0) dit_signal(P.c_stats);
           } else {
             dit_row_stats(P, et, sh);
@@ -750,7 +758,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
           }
           const bool finished = (S == 1) || sh->last;
           if ((kind == DIT_O || kind == DIT_DOWN) && finished)
-            dit_tile_stats(xn, P.M, et, sh, P.stats + (size_t)nt * P.M * 2);
+            dit_tile_stats(xn, P.M, et, (float*)(sU + DIT_UNION - DIT_TS_BYTES),
+                           P.stats + (size_t)nt * P.M * 2);
           named_sync(1, 128);
           if (finished && et == 0) {
             if (kind == DIT_QKV) dit_signal(P.f_qkv + (size_t)l * tiles + nt);
