@@ -583,6 +583,9 @@ fm_status dit_persistent(fm_ctx* c, const float* mods, int slot, int ctx_len, bo
     const int nkb = (kbs[k] + P.splits[k] - 1) / P.splits[k];
     if ((size_t)nkb * brows * 128 > (size_t)fm::DIT_UNION) return FM_ERR_UNSUPPORTED;
     if (nkb * 64 > 1024) return FM_ERR_UNSUPPORTED;  // staged shift/scale slice
+    // the B operand is published in at most two batches of 8 k-blocks on one
+    // mbarrier, so the MMA issuer can never fall two phases behind
+    if (nkb > 16) return FM_ERR_UNSUPPORTED;
     // staged partial tiles, below the tile-statistics scratch at the end
     if ((size_t)P.splits[k] * 128 * brows * 4 > (size_t)(fm::DIT_UNION - fm::DIT_TS_BYTES))
       return FM_ERR_UNSUPPORTED;

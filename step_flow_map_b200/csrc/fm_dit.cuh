@@ -316,9 +316,43 @@ __device__ __forceinline__ void dit_stage_mods(const DitParams& P, int kind, int
   }
 }
 
-__device__ __forceinline__ void dit_fill_b(const DitParams& P, int kind, int l, uint8_t* sB,
-                                           int kb0, int nkb, int brows, int Kd, int et,
-                                           DitShared* sh) {
+// Rows M .. brows-1 of a QKV phase's B operand: the appended context rows
+// (normalised before the pass), then zeros.  They depend on nothing the
+// pass computes, so this runs before the phase's wait.
+__device__ __forceinline__ void dit_fill_extra(const DitParams& P, uint8_t* sB, int kb0, int nkb,
+                                               int brows, int Kd, int et) {
+  const int tile_bytes = brows * 128;
+  const int M = P.M, xrows = brows - M;
+  const int items_x = nkb * xrows * 8;
+  for (int i0 = 0; i0 < items_x; i0 += 128 * 8) {
+    uint4 cp[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int idx = i0 + u * 128 + et;
+      const int kbi = idx / (xrows * 8), rem = idx - kbi * (xrows * 8);
+      const int r = rem >> 3, col = (kb0 + kbi) * TC_BK + (rem & 7) * 8;
+      cp[u] = make_uint4(0, 0, 0, 0);
+      if (idx < items_x && r < P.n_ctx && col < Kd)
+        cp[u] = __ldcg((const uint4*)(P.ctx_rows + (size_t)r * P.d + col));
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int idx = i0 + u * 128 + et;
+      if (idx >= items_x) break;
+      const int kbi = idx / (xrows * 8), rem = idx - kbi * (xrows * 8);
+      const int row = M + (rem >> 3), ch = rem & 7;
+      *(uint4*)(sB + kbi * tile_bytes + row * 128 + ((ch ^ (row & 7)) << 4)) = cp[u];
+    }
+  }
+}
+
+// B operand rows 0 .. M-1 (M = 16: 128 items per k-block, so each batch of
+// 1024 items is 8 k-blocks).  Every batch is published on `bready` (all 128
+// threads arrive) as soon as it is stored, so the MMAs of its k-blocks, and
+// the ring refills they free, overlap the rest of the fill.
+__device__ __forceinline__ void dit_fill_b(const DitParams& P, int kind, uint8_t* sB, int kb0,
+                                           int nkb, int brows, int Kd, int et, DitShared* sh,
+                                           uint32_t bready) {
   // one loop per kind of row, so each unrolled batch holds one code path
   const int tile_bytes = brows * 128;
   const int M = P.M;
@@ -363,31 +397,8 @@ __device__ __forceinline__ void dit_fill_b(const DitParams& P, int kind, int l, 
         packed.w = pack_bf16x2((xb[u].z - mean) * rstd * (1.f + c[6]) + h[6], (xb[u].w - mean) * rstd * (1.f + c[7]) + h[7]);
         put(kbi, row, ch, packed);
       }
-    }
-    // rows after the block: appended context rows (already normalised),
-    // then zeros up to brows
-    const int xrows = brows - M;
-    if (xrows > 0) {
-      const int items_x = nkb * xrows * 8;
-      for (int i0 = 0; i0 < items_x; i0 += 128 * 8) {
-        uint4 cp[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int idx = i0 + u * 128 + et;
-          const int kbi = idx / (xrows * 8), rem = idx - kbi * (xrows * 8);
-          const int r = rem >> 3, col = (kb0 + kbi) * TC_BK + (rem & 7) * 8;
-          cp[u] = make_uint4(0, 0, 0, 0);
-          if (idx < items_x && r < P.n_ctx && col < Kd)
-            cp[u] = __ldcg((const uint4*)(P.ctx_rows + (size_t)r * P.d + col));
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int idx = i0 + u * 128 + et;
-          if (idx >= items_x) break;
-          const int kbi = idx / (xrows * 8), rem = idx - kbi * (xrows * 8);
-          put(kbi, M + (rem >> 3), rem & 7, cp[u]);
-        }
-      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(bready);
     }
   } else {
     // copied rows: attention output (O) or MLP hidden (down)
@@ -411,9 +422,10 @@ __device__ __forceinline__ void dit_fill_b(const DitParams& P, int kind, int l, 
         const int kbi = idx / (brows * 8), rem = idx - kbi * (brows * 8);
         put(kbi, rem >> 3, rem & 7, cp[u]);
       }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(bready);
     }
   }
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // Final epilogue of one 128-feature tile with the reduced accumulators v
@@ -545,13 +557,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
         const int brows = dit_brows(P, kind);
         const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(brows >> 3) << 17) |
                                ((uint32_t)(128 >> 4) << 24);
-        if (!mbar_wait(smem_u32(&sh->bready), b_phase, abort)) break;
-        b_phase ^= 1;
         if (!mbar_wait(smem_u32(&sh->tempty[acc]), acc_phase ^ 1, abort)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + acc * 64;
         bool ok = true;
         for (int kb = kb0; kb < kb1; ++kb) {
+          if (((kb - kb0) & 7) == 0) {
+            // the next 8 k-blocks of the B operand are in shared memory
+            if (!mbar_wait(smem_u32(&sh->bready), b_phase, abort)) { ok = false; break; }
+            b_phase ^= 1;
+            tc_fence_after();
+          }
           if (!mbar_wait(smem_u32(&sh->full[stage]), phase, abort)) { ok = false; break; }
           tc_fence_after();
           const uint64_t ad = desc_sw128(smem_u32(sA + stage * 16384));
@@ -617,6 +633,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
           if (kv_pre) attn_ctx_prologue<1, DIT_ATTN_ST>(P.Kc[l], P.Vc[l], P.attn, h, split, sU, et);
         }
       }
+      if (kind == DIT_QKV && P.n_ctx > 0) {
+        int N, Kd;
+        dit_gemm_shape(P, kind, &N, &Kd);
+        const int S = P.splits[kind], kbs = Kd / TC_BK, z = cta % S;
+        const int kb0 = z * kbs / S, kb1 = (z + 1) * kbs / S;
+        dit_fill_extra(P, sU, kb0, kb1 - kb0, dit_brows(P, kind), Kd, et);
+      }
       if (kind != -1) {
         // wait for the units whose outputs this one reads
         if (et == 0) sh->ok[it & 1] = dit_wait_deps(P, kind, l, cta) ? 1 : 0;
@@ -666,8 +689,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
           const int nt = cta / S, z = cta % S;
           const int kb0 = z * kbs / S, kb1 = (z + 1) * kbs / S;
           const int brows = dit_brows(P, kind);
-          dit_fill_b(P, kind, l, sU, kb0, kb1 - kb0, brows, Kd, et, sh);
-          mbar_arrive(smem_u32(&sh->bready));
+          dit_fill_b(P, kind, sU, kb0, kb1 - kb0, brows, Kd, et, sh, smem_u32(&sh->bready));
           const int n = nt * TC_BM + r;
           // residual phases: x and the gate, loaded while the MMAs run
           const bool resid = (kind == DIT_O || kind == DIT_DOWN);
