@@ -29,6 +29,7 @@ k_verify_greedy(const float* __restrict__ tgt, const int* __restrict__ draft, in
   __shared__ float shv[32];
   __shared__ int shi[32];
   __shared__ int amax[VG_MAX_ROWS];
+  __shared__ int ydraft[VG_MAX_ROWS];   // N*K < N*(K+1) <= VG_MAX_ROWS
   __shared__ int is_last;
   const int rows_b = N * (K + 1);
   const int row = blockIdx.x / chunks, c = blockIdx.x - row * chunks;
@@ -52,27 +53,40 @@ k_verify_greedy(const float* __restrict__ tgt, const int* __restrict__ draft, in
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  for (int rr = threadIdx.x; rr < rows_b; rr += blockDim.x) {
-    size_t base = ((size_t)b * rows_b + rr) * chunks;
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
-    for (int k = 0; k < chunks; ++k) {
-      float v = __ldcg(pv + base + k);
-      int i = __ldcg(pi + base + k);
-      if (am_better(v, i, bv, bi)) { bv = v; bi = i; }
+  // one warp per row: lanes take chunks (their loads in flight together),
+  // the warp combines in chunk-index order of ties (lowest token wins)
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  for (int rr = warp; rr < rows_b; rr += nwarps) {
+    const size_t base = ((size_t)b * rows_b + rr) * chunks;
+    ArgMax m{-INFINITY, 0x7fffffff};
+    for (int k0 = 0; k0 < chunks; k0 += 64) {
+      float v[2];
+      int i[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int k = k0 + u * 32 + lane;
+        v[u] = k < chunks ? __ldcg(pv + base + k) : -INFINITY;
+        i[u] = k < chunks ? __ldcg(pi + base + k) : 0x7fffffff;
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+        if (am_better(v[u], i[u], m.v, m.i)) { m.v = v[u]; m.i = i[u]; }
     }
-    amax[rr] = (bi == 0x7fffffff) ? 0 : bi;
+    m = warp_argmax(m);
+    if (lane == 0) amax[rr] = (m.i == 0x7fffffff) ? 0 : m.i;
   }
+  // the drafts of the sequence, staged by all threads
+  for (int e = threadIdx.x; e < N * K; e += blockDim.x) ydraft[e] = draft[(size_t)b * N * K + e];
   __syncthreads();
   if (threadIdx.x == 0) {
     int best_n = -1, best_j = 0;
     for (int j = 0; j < N; ++j) {
-      const int* y = draft + ((size_t)b * N + j) * K;
+      const int* y = ydraft + j * K;
       int n = 0;
       while (n < K && y[n] == amax[j * (K + 1) + n]) ++n;
       if (n > best_n) { best_n = n; best_j = j; }
     }
-    const int* y = draft + ((size_t)b * N + best_j) * K;
+    const int* y = ydraft + best_j * K;
     int* o = out + (size_t)b * (K + 1);
     for (int i = 0; i < best_n; ++i) o[i] = y[i];
     o[best_n] = amax[best_j * (K + 1) + best_n];
@@ -117,15 +131,22 @@ k_row_stats(const float* __restrict__ tgt, const float* __restrict__ dlog, int n
 struct RowStat {
   double m, S;
 };
-__device__ __forceinline__ RowStat combine_stats(const float* pm, const double* ps, int row,
-                                                 int chunks, double T) {
+// Row statistics (max m, S = sum of exp((l - m)/T)) from the chunk partials,
+// combined by one warp: lanes over chunks, a fixed shuffle tree
+// (deterministic); every lane returns the result.
+__device__ __forceinline__ RowStat warp_combine_stats(const float* pm, const double* ps, int row,
+                                                      int chunks, double T, int lane) {
   double m = -INFINITY;
-  for (int c = 0; c < chunks; ++c) m = fmax(m, (double)pm[(size_t)row * chunks + c]);
+  for (int c = lane; c < chunks; c += 32) m = fmax(m, (double)pm[(size_t)row * chunks + c]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
   double S = 0.0;
-  for (int c = 0; c < chunks; ++c) {
-    double mc = (double)pm[(size_t)row * chunks + c];
+  for (int c = lane; c < chunks; c += 32) {
+    const double mc = (double)pm[(size_t)row * chunks + c];
     if (mc > -INFINITY) S += ps[(size_t)row * chunks + c] * exp((mc - m) / T);
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
   return RowStat{m, S};
 }
 
@@ -158,9 +179,9 @@ k_verify_sample_decide(const float* __restrict__ tgt, const float* __restrict__ 
     r0 = __ffs(alive) - 1;
     const int trow = (b * N + r0) * (K + 1) + i;
     const float* tp = tgt + (size_t)trow * V;
-    if (tid == 0) {
-      RowStat st = combine_stats(pm, ps, trow, chunks, dT);
-      s_mp = st.m; s_Sp = st.S; s_mode = 0; s_buf = 0; s_accept = -1;
+    if (tid < 32) {
+      RowStat st = warp_combine_stats(pm, ps, trow, chunks, dT, tid);
+      if (tid == 0) { s_mp = st.m; s_Sp = st.S; s_mode = 0; s_buf = 0; s_accept = -1; }
     }
     __syncthreads();
     for (int j = 0; j < N; ++j) {
@@ -168,15 +189,18 @@ k_verify_sample_decide(const float* __restrict__ tgt, const float* __restrict__ 
       const int y = draft[((size_t)b * N + j) * K + i];
       const int drow = (b * N + j) * K + i;
       const float* qp = dlog ? dlog + (size_t)drow * V : nullptr;
-      if (tid == 0) {
-        double qy = 1.0;
-        if (qp) {
-          RowStat sq = combine_stats(pm, ps, n_tgt_rows + drow, chunks, dT);
-          s_mq = sq.m; s_Sq = sq.S;
-          qy = exp(((double)qp[y] - sq.m) / dT) / sq.S;
+      if (tid < 32) {
+        RowStat sq{0.0, 1.0};
+        if (qp) sq = warp_combine_stats(pm, ps, n_tgt_rows + drow, chunks, dT, tid);
+        if (tid == 0) {
+          double qy = 1.0;
+          if (qp) {
+            s_mq = sq.m; s_Sq = sq.S;
+            qy = exp(((double)qp[y] - sq.m) / dT) / sq.S;
+          }
+          double py = (s_mode == 0) ? exp(((double)tp[y] - s_mp) / dT) / s_Sp : buf[s_buf][y];
+          s_accept = (ua[((size_t)b * N + j) * K + i] * qy < py) ? y : -1;
         }
-        double py = (s_mode == 0) ? exp(((double)tp[y] - s_mp) / dT) / s_Sp : buf[s_buf][y];
-        s_accept = (ua[((size_t)b * N + j) * K + i] * qy < py) ? y : -1;
       }
       __syncthreads();
       if (s_accept >= 0) break;
@@ -235,9 +259,9 @@ k_verify_sample_decide(const float* __restrict__ tgt, const float* __restrict__ 
     r0 = __ffs(alive) - 1;
     const int trow = (b * N + r0) * (K + 1) + K;
     const float* tp = tgt + (size_t)trow * V;
-    if (tid == 0) {
-      RowStat st = combine_stats(pm, ps, trow, chunks, dT);
-      s_mp = st.m; s_Sp = st.S;
+    if (tid < 32) {
+      RowStat st = warp_combine_stats(pm, ps, trow, chunks, dT, tid);
+      if (tid == 0) { s_mp = st.m; s_Sp = st.S; }
     }
     __syncthreads();
     const double mp = s_mp, iSp = 1.0 / s_Sp, u = ures[b];
