@@ -147,6 +147,17 @@ def stored_traffic(kernel: str, workload: str):
     return None
 
 
+def workload_config(w: fs.Workload, rounds: int, world: int) -> dict:
+    """The `config` object of both arms' JSON lines."""
+    s = w.shape
+    step_bytes = sum(v for k, v in algorithmic_bytes(w).items() if not k.endswith("_per_launch"))
+    return {"workload": w.name, "sequences_per_gpu": w.B, "noise_drafts": w.n_noise, "K": s.K,
+            "V": s.V, "d": s.d, "n_blocks": s.n_blocks, "context_rows": w.ctx + w.new_rows,
+            "num_steps": len(w.t_grid) - 1, "temperatures": sorted(set(w.temps)),
+            "distinct_rounds": rounds, "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2: every step streams ~%.2f GB" % (step_bytes / 1e9)}
+
+
 def algorithmic_flops(w: fs.Workload):
     """FLOPs of each kernel class per step (2 per multiply-add)."""
     s = w.shape
@@ -429,11 +440,7 @@ def run_fm(args, w, rank, world, local_rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": w.dtype, "data": "synthetic (seeded fm_synth inputs; no trained weights)",
-        "config": {"workload": w.name, "sequences_per_gpu": B, "noise_drafts": N, "K": K, "V": V,
-                   "d": s.d, "n_blocks": s.n_blocks, "context_rows": w.ctx + w.new_rows,
-                   "num_steps": len(w.t_grid) - 1, "temperatures": sorted(set(w.temps)),
-                   "distinct_rounds": R, "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2: every step streams ~%.2f GB" % (step_bytes / 1e9)},
+        "config": workload_config(w, R, world),
         "verified_tokens_per_s": round(tok_per_s, 1),
         "mean_accepted": round(n_sum / (args.steps * B), 3),
         "step_hbm_gbs": round(step_bytes / (ms / args.steps / 1e3) / 1e9, 1),
@@ -453,32 +460,54 @@ def run_fm(args, w, rank, world, local_rank):
         for i in range(RE):
             rd = rounds[i]
             pin.append({k: (v.cpu().pin_memory() if v is not None else None) for k, v in rd.items()})
-        dev_in = {k: (torch.empty_like(v) if v is not None else None) for k, v in rounds[0].items()}
+        # two device input buffers: a copy stream uploads step k+1's inputs
+        # while step k runs (events order each upload after the step that
+        # last read its buffer, and each step after its upload)
+        dev_in = [{k: (torch.empty_like(v) if v is not None else None) for k, v in rounds[0].items()}
+                  for _ in range(2)]
         n_stage = torch.zeros(B, dtype=torch.int32, device="cuda")
         host_n = torch.empty((args.steps, B), dtype=torch.int32).pin_memory()
         host_tok = torch.empty((args.steps, B, K + 1), dtype=torch.int32).pin_memory()
         h2d = sum(v.numel() * v.element_size() for v in pin[0].values() if v is not None)
         d2h = B * 4 + B * (K + 1) * 4
-        gstage = None
+        gstage = [None, None]
         if graphs:
-            for key, v in pin[0].items():
-                if v is not None:
-                    dev_in[key].copy_(v)
-            gstage = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gstage):
-                step(dev_in, n_stage, torch.cuda.current_stream())
+            for bi in range(2):
+                for key, v in pin[0].items():
+                    if v is not None:
+                        dev_in[bi][key].copy_(v)
+                gstage[bi] = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gstage[bi]):
+                    step(dev_in[bi], n_stage, torch.cuda.current_stream())
+        torch.cuda.synchronize()
         barrier()
+        cs = torch.cuda.Stream()
+        copied = [torch.cuda.Event(), torch.cuda.Event()]
+        used = [torch.cuda.Event(), torch.cuda.Event()]
+
+        def upload(k: int, bi: int):
+            with torch.cuda.stream(cs):
+                if k >= 2:
+                    cs.wait_event(used[bi])
+                for key, v in pin[k % RE].items():
+                    if v is not None:
+                        dev_in[bi][key].copy_(v, non_blocking=True)
+                copied[bi].record(cs)
+
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
+        cs.wait_event(e0)
+        upload(0, 0)
         for k in range(args.steps):
-            src = pin[k % RE]
-            for key, v in src.items():
-                if v is not None:
-                    dev_in[key].copy_(v, non_blocking=True)
-            if gstage is not None:
-                gstage.replay()
+            bi = k % 2
+            if k + 1 < args.steps:
+                upload(k + 1, 1 - bi)
+            stream.wait_event(copied[bi])
+            if gstage[bi] is not None:
+                gstage[bi].replay()
             else:
-                step(dev_in, n_stage, stream)
+                step(dev_in[bi], n_stage, stream)
+            used[bi].record(stream)
             host_n[k].copy_(n_stage, non_blocking=True)
             host_tok[k].copy_(out_tok, non_blocking=True)
         e1.record(stream)
@@ -549,7 +578,7 @@ def run_reference(args, w):
             "ms_per_step": round(sec / len(times) * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded fm_synth inputs; no trained weights)",
-            "config": {"workload": w.name, "sequences_per_gpu": 1},
+            "config": workload_config(w, len(times) + args.warmup, 1),
             "cpu_baseline": {"value": round(v, 5), "unit": "blocks/s", "cores": cores,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(v, 5), "unit": "blocks/s", "h2d_bytes_per_step": 0,

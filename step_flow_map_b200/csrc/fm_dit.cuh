@@ -154,17 +154,22 @@ __device__ __forceinline__ int dit_brows(const DitParams& P, int kind) {
   return 16;
 }
 
-// Bounded wait (one thread) until the counter reaches `target`.
+// Bounded wait (one thread) until the counter reaches `target`.  The abort
+// word and the clock are read every 32 polls only: a load after an acquire
+// load cannot start before it, so checking them on every poll would double
+// the poll's round trip.
 __device__ __forceinline__ bool dit_wait(const DitParams& P, const unsigned* ctr, unsigned target) {
   const unsigned long long t0 = gtimer();
-  while (true) {
+  for (unsigned n = 1;; ++n) {
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
     if (v >= target) return true;
-    if (*(volatile int*)P.abort_g) return false;
-    if (gtimer() - t0 > TC_TIMEOUT_NS) {
-      atomicExch(P.abort_g, 1);
-      return false;
+    if ((n & 31) == 0) {
+      if (*(volatile int*)P.abort_g) return false;
+      if (gtimer() - t0 > TC_TIMEOUT_NS) {
+        atomicExch(P.abort_g, 1);
+        return false;
+      }
     }
   }
 }
