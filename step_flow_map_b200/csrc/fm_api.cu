@@ -98,6 +98,9 @@ struct fm_ctx {
   float* dit_stats = nullptr;
   void* dit_hf = nullptr;
   bool dit_ok = false;           // the persistent pass fits this configuration and device
+  // final LayerNorm built by the LM head instead of the persistent pass
+  // (measured: LM head 105 -> 133 us for 7 us saved in the pass; off)
+  bool dit_final_in_lm = false;
   int dit_l2_ahead = 0;          // weight k-blocks the persistent pass prefetches into L2 (measured: no gain)
   float* attn_part = nullptr;   // split-KV attention partials
   unsigned* attn_cnt = nullptr;
@@ -247,9 +250,9 @@ fm_status gemm_w(fm_ctx* c, int cls, const T* A, int lda, const T* W, int M, int
 template <class Epi>
 fm_status gemm_ln(fm_ctx* c, int cls, const float* x, const float* shift, const float* scale,
                   int M, Epi epi, cudaStream_t st, const fm::TcMap* map, bool* done,
-                  const bf16* extra = nullptr, int n_extra = 0) {
+                  const bf16* extra = nullptr, int n_extra = 0, bool force = false) {
   *done = false;
-  if (!c->use_tc || !map || !map->valid || M > 32 || !c->ln_in_gemm) return FM_OK;
+  if (!c->use_tc || !map || !map->valid || M > 32 || !(c->ln_in_gemm || force)) return FM_OK;
   Prof prof(c, cls, st);
   int n_launch = 0;
   fm_status s = fm::tc_gemm_ln(c->tc, *map, x, shift, scale, M, extra, M + n_extra, epi, c->splitk,
@@ -539,6 +542,7 @@ fm_status dit_persistent(fm_ctx* c, const float* mods, int slot, int ctx_len, bo
   P.F = g.mlp;
   P.M = fm::DIT_M;
   P.l2_ahead = c->dit_l2_ahead;
+  P.skip_final = (c->dit_final_in_lm && c->use_tc && c->tc.lm.valid) ? 1 : 0;
   // K splits per GEMM kind: about one unit per SM
   const int tiles[5] = {3 * d / 128, 0, d / 128, g.mlp / 128, d / 128};
   const int kbs[5] = {d / 64, 0, d / 64, d / 64, g.mlp / 64};
@@ -808,7 +812,26 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
     bool have_partials = false, fused = false;
     if (persistent) {
       fused = true;
-      if (need_logits) {
+      bool lnf = false;
+      if (c->dit_final_in_lm && c->tc.lm.valid) {   // matches the pass's skip_final
+        // the persistent pass left x un-normalised: the LM head builds its
+        // B operand as LN0(x)(1 + scale_f) + shift_f in shared memory
+        if (need_logits)
+          FM_TRY(gemm_ln(c, FM_PROF_LM_HEAD, c->x, mf, mf + d, M, fm::EpiStoreF32{logits, V}, st,
+                         &c->tc.lm, &lnf, nullptr, 0, true));
+        else
+          FM_TRY(gemm_ln(c, FM_PROF_LM_HEAD, c->x, mf, mf + d, M,
+                         fm::EpiArgmax{c->part_v, c->part_i, c->n_part}, st, &c->tc.lm, &lnf,
+                         nullptr, 0, true));
+        have_partials = lnf && !need_logits;
+        if (!lnf) {
+          Prof prof(c, FM_PROF_NORM, st);
+          FM_LAUNCH(c, FM_PROF_NORM, (fm::k_adaln<float, T>), M, 256, 0, st, c->x, d, mf, mf + d,
+                    (T*)c->dit_hf);
+        }
+      }
+      if (lnf) {
+      } else if (need_logits) {
         FM_TRY(gemm_w<T>(c, FM_PROF_LM_HEAD, (const T*)c->dit_hf, d, (const T*)c->w.W_lm, M, V, d,
                          fm::EpiStoreF32{logits, V}, st, &c->tc.lm));
       } else {

@@ -48,6 +48,7 @@ struct DitParams {
   int n_blocks, d, F, M;              // M <= 16 block rows
   int splits[5];                      // per GEMM kind (index by DIT_*; [1] = attention splits)
   int l2_ahead;                       // weight k-blocks prefetched into L2 beyond the ring
+  int skip_final;                     // the LM head applies the final LayerNorm itself
   float* x;                           // residual stream [M][d] fp32
   float* stats;                       // [d/128 tiles][M][2]: tile mean, tile sum of squared deviations
   float* partial;                     // split-K partials, one region per GEMM kind
@@ -618,6 +619,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
       }
       int l = 0;
       const int kind = dit_phase_kind(p, nb, &l);
+      if (kind == -2 && P.skip_final) continue;
       bool active;
       if (kind == -1 || kind == -2) active = cta < P.d / TC_BM;
       else if (kind == DIT_ATTN) active = cta < P.attn.n_heads * (P.attn.n_ctx_splits + 1);
