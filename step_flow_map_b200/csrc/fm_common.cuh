@@ -168,11 +168,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 // GELU, tanh form: 0.5 u (1 + tanh(z)) with z = sqrt(2/pi) (u + 0.044715 u^3).
 // Since 1 + tanh(z) = 2 / (1 + e^{-2z}), this is u / (1 + e^{-2z}): one
-// exponential and one reciprocal (e^{-2z} overflowing to +inf gives -0).
+// exponential and one fast division.  The exponent is clamped at 80
+// (e^80 < 2^126, the fast division's range; the quotient there is below
+// |u| * 2e-35 anyway).
 __device__ __forceinline__ float gelu_tanh(float u) {
   const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
   const float z = k0 * (u + 0.044715f * u * u * u);
-  return u * __frcp_rn(1.f + __expf(-2.f * z));
+  return __fdividef(u, 1.f + __expf(fminf(-2.f * z, 80.f)));
 }
 __device__ __forceinline__ float silu(float u) { return u / (1.f + expf(-u)); }
 
