@@ -134,9 +134,9 @@ def source_sha1() -> str:
     return h.hexdigest()
 
 
-def stored_traffic(kernel: str, workload: str):
+def stored_traffic(kernel: str, workload: str, path: str | None = None):
     """DRAM bytes per launch from profiles/traffic.txt (JSON), or None."""
-    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    p = path or os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None
     with open(p) as f:
@@ -145,6 +145,28 @@ def stored_traffic(kernel: str, workload: str):
     if e and e.get("source_sha1") == source_sha1():
         return e["dram_bytes_per_launch"]
     return None
+
+
+RANK_SEED_STRIDE = 100000   # round seeds of rank k start at k * stride: replicas see distinct inputs
+
+
+def round_seed(i: int, rank: int) -> int:
+    """Seed index of the i-th distinct round of a rank."""
+    return i + RANK_SEED_STRIDE * rank
+
+
+def reduce_over_ranks(dist, device, ms: float, verified: float, world: int):
+    """Whole-job figures of the replicas: the slowest rank's device time and
+    the sum of verified tokens (each rank drafts its own sequences; no
+    exchange on the data path).  `dist` None means one process."""
+    if dist is None:
+        return ms, verified * world
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    v = torch.tensor([float(verified)], dtype=torch.float64, device=device)
+    dist.all_reduce(v)
+    return float(t.item()), float(v.item())
 
 
 def workload_config(w: fs.Workload, rounds: int, world: int) -> dict:
@@ -237,7 +259,7 @@ def run_fm(args, w, rank, world, local_rank):
     dlog = torch.empty((B, N, K, V), dtype=torch.float32, device="cuda") if need_logits else None
     rounds = []
     for i in range(R):
-        r = i + 100000 * rank
+        r = round_seed(i, rank)
         ri = fs.round_inputs(w, r)
         rd = {"noise": to_device(ri.noise, w.dtype),
               "hidden": to_device(ri.new_hidden, w.dtype) if w.new_rows else None,
@@ -372,16 +394,10 @@ def run_fm(args, w, rank, world, local_rank):
         if graphs:
             del pgraphs
     barrier()
-    ms = max_over_ranks(ev0.elapsed_time(ev1))
     n_round = n_acc_round.sum(dim=1).cpu().numpy()
     n_sum = int(sum(n_round[(args.warmup + k) % R] for k in range(args.steps)))
     verified = n_sum + args.steps * B           # accepted + one target token per sequence
-    if dist is not None:
-        t = torch.tensor([float(verified)], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t)
-        verified = float(t.item())
-    else:
-        verified *= world
+    ms, verified = reduce_over_ranks(dist, "cuda", ev0.elapsed_time(ev1), verified, world)
     sec = ms / 1e3
     blocks = B * N * args.steps * world
     value = blocks / sec

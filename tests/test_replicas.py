@@ -1,0 +1,82 @@
+"""Replica (multi-process) host logic of the benchmark, on CPU with gloo.
+
+Each rank drafts its own sequences with its own inputs; the only cross-rank
+steps are the barrier, the slowest rank's device time and the sum of
+verified tokens.  Two gloo ranks check that reduction and that replicas
+draw distinct seeded inputs.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+import fm_synth as fs
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    import datetime
+
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        ms, verified = bench.reduce_over_ranks(dist, "cpu", 1.5 + rank, 10.0 * (rank + 1), world)
+        out.put((rank, ms, verified))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_reduce_over_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    for rank, ms, verified in res:
+        assert ms == pytest.approx(2.5)          # the slowest rank's time
+        assert verified == pytest.approx(30.0)   # tokens of both replicas
+
+
+def test_single_process_reduction():
+    assert bench.reduce_over_ranks(None, "cpu", 3.0, 7.0, 1) == (3.0, 7.0)
+
+
+def test_replicas_draw_distinct_rounds():
+    seeds = {bench.round_seed(i, r) for r in range(8) for i in range(32)}
+    assert len(seeds) == 8 * 32
+    w = fs.WORKLOADS["tiny_f32"]
+    a = fs.round_inputs(w, bench.round_seed(0, 0))
+    b = fs.round_inputs(w, bench.round_seed(0, 1))
+    assert not np.array_equal(a.noise, b.noise)
+    assert not np.array_equal(a.u_draft, b.u_draft)
+
+
+def test_stored_traffic_follows_the_sources(tmp_path):
+    # a DRAM-traffic record counts only while the kernel sources are the
+    # ones it was captured on
+    import json
+    rec = {"k": {"wl": {"dram_bytes_per_launch": 123, "source_sha1": bench.source_sha1()}}}
+    p = tmp_path / "t.txt"
+    p.write_text(json.dumps(rec))
+    assert bench.stored_traffic("k", "wl", str(p)) == 123
+    assert bench.stored_traffic("k", "other", str(p)) is None
+    rec["k"]["wl"]["source_sha1"] = "0" * 40
+    p.write_text(json.dumps(rec))
+    assert bench.stored_traffic("k", "wl", str(p)) is None
