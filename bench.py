@@ -169,6 +169,19 @@ def reduce_over_ranks(dist, device, ms: float, verified: float, world: int):
     return float(t.item()), float(v.item())
 
 
+def acceptance_stats(n, K: int) -> dict:
+    """Accepted-length statistics of timed rounds: `n` holds one accepted
+    length (0..K) per (round, sequence).  hist[i] = rounds with n = i;
+    p_reach[i-1] = P(n >= i), the chance the verifier reaches draft position
+    i with every earlier position accepted."""
+    a = np.asarray(n, dtype=np.int64).reshape(-1)
+    hist = np.bincount(np.clip(a, 0, K), minlength=K + 1)
+    tot = max(int(a.size), 1)
+    reach = [round(float((a >= i).sum()) / tot, 4) for i in range(1, K + 1)]
+    return {"mean": round(float(a.mean()) if a.size else 0.0, 3),
+            "hist": [int(x) for x in hist], "p_reach": reach}
+
+
 def workload_config(w: fs.Workload, rounds: int, world: int) -> dict:
     """The `config` object of both arms' JSON lines."""
     s = w.shape
@@ -394,8 +407,10 @@ def run_fm(args, w, rank, world, local_rank):
         if graphs:
             del pgraphs
     barrier()
-    n_round = n_acc_round.sum(dim=1).cpu().numpy()
+    n_all = n_acc_round.cpu().numpy()          # [R, B] accepted lengths
+    n_round = n_all.sum(axis=1)
     n_sum = int(sum(n_round[(args.warmup + k) % R] for k in range(args.steps)))
+    acc = acceptance_stats(np.stack([n_all[(args.warmup + k) % R] for k in range(args.steps)]), K)
     verified = n_sum + args.steps * B           # accepted + one target token per sequence
     ms, verified = reduce_over_ranks(dist, "cuda", ev0.elapsed_time(ev1), verified, world)
     sec = ms / 1e3
@@ -459,6 +474,7 @@ def run_fm(args, w, rank, world, local_rank):
         "config": workload_config(w, R, world),
         "verified_tokens_per_s": round(tok_per_s, 1),
         "mean_accepted": round(n_sum / (args.steps * B), 3),
+        "acceptance": acc,
         "step_hbm_gbs": round(step_bytes / (ms / args.steps / 1e3) / 1e9, 1),
         "step_hbm_frac": round(step_bytes / (ms / args.steps / 1e3) / 1e9 / pk["hbm_gbs"], 4),
         "roofline": roof, "kernels": per_class,

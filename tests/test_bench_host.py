@@ -1,9 +1,11 @@
-"""Replica (multi-process) host logic of the benchmark, on CPU with gloo.
+"""Host logic of the benchmark, on CPU.
 
-Each rank drafts its own sequences with its own inputs; the only cross-rank
-steps are the barrier, the slowest rank's device time and the sum of
-verified tokens.  Two gloo ranks check that reduction and that replicas
-draw distinct seeded inputs.
+Replicas: each rank drafts its own sequences with its own inputs; the only
+cross-rank steps are the barrier, the slowest rank's device time and the
+sum of verified tokens.  Two gloo ranks check that reduction and that
+replicas draw distinct seeded inputs.  Also: the DRAM-traffic record is
+honoured only for the sources it was captured on, and the accepted-length
+statistics.
 """
 import os
 import socket
@@ -80,3 +82,13 @@ def test_stored_traffic_follows_the_sources(tmp_path):
     rec["k"]["wl"]["source_sha1"] = "0" * 40
     p.write_text(json.dumps(rec))
     assert bench.stored_traffic("k", "wl", str(p)) is None
+
+
+def test_acceptance_stats():
+    st = bench.acceptance_stats([[0, 3], [16, 3]], 16)
+    assert st["mean"] == pytest.approx(5.5)
+    assert st["hist"][0] == 1 and st["hist"][3] == 2 and st["hist"][16] == 1
+    assert sum(st["hist"]) == 4
+    assert st["p_reach"][0] == 0.75      # three of four reach position 1
+    assert st["p_reach"][3] == 0.25      # only the full block passes position 4
+    assert st["p_reach"][15] == 0.25
