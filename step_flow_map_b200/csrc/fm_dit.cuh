@@ -179,7 +179,7 @@ __device__ __forceinline__ bool dit_wait(const DitParams& P, const unsigned* ctr
 // before it by a CTA barrier).
 __device__ __forceinline__ void dit_signal(unsigned* ctr) { red_add_release_gpu(ctr, 1u); }
 
-// Waits (one thread) for everything this CTA's unit of the phase reads:
+// Waits for everything this CTA's unit of the phase reads:
 //   QKV(l)   the residual stream after the last block (all down tiles) or the
 //            embedded rows' statistics;
 //   ATTN(l)  the Q, K and V tiles of its head;
@@ -190,29 +190,35 @@ __device__ __forceinline__ void dit_signal(unsigned* ctr) { red_add_release_gpu(
 // Every write-after-read hazard on the shared buffers is ordered through the
 // same chain: a unit that overwrites a buffer depends, through full-row
 // LayerNorm waits, on every unit that read the previous contents.
-__device__ bool dit_wait_deps(const DitParams& P, int kind, int l, int cta) {
+//
+// One warp waits: each lane polls its own counters (a single counter on lane
+// 0; attention's three tiles or a k-slice's heads / up tiles spread over the
+// lanes), so their acquire loads are in flight together; the warp vote and
+// the CTA barrier that follows order every thread after all of them.
+__device__ bool dit_wait_deps_warp(const DitParams& P, int kind, int l, int cta, int lane) {
   const unsigned tiles_d = (unsigned)(P.d / TC_BM);
   const int H = P.attn.n_heads;
-  if (kind == -1) return true;
-  if (kind == -2) return dit_wait(P, P.c_down + P.n_blocks - 1, tiles_d);
-  if (kind == DIT_QKV)
-    return l == 0 ? dit_wait(P, P.c_stats, tiles_d) : dit_wait(P, P.c_down + l - 1, tiles_d);
-  if (kind == DIT_UP) return dit_wait(P, P.c_o + l, tiles_d);
-  if (kind == DIT_ATTN) {
+  bool ok = true;
+  if (kind == -2) {
+    if (lane == 0) ok = dit_wait(P, P.c_down + P.n_blocks - 1, tiles_d);
+  } else if (kind == DIT_QKV) {
+    if (lane == 0) ok = dit_wait(P, l == 0 ? P.c_stats : P.c_down + l - 1, tiles_d);
+  } else if (kind == DIT_UP) {
+    if (lane == 0) ok = dit_wait(P, P.c_o + l, tiles_d);
+  } else if (kind == DIT_ATTN) {
     const int h = cta % H;
-    const unsigned* f = P.f_qkv + (size_t)l * 3 * H;
-    return dit_wait(P, f + h, 1) && dit_wait(P, f + H + h, 1) && dit_wait(P, f + 2 * H + h, 1);
+    if (lane < 3) ok = dit_wait(P, P.f_qkv + (size_t)l * 3 * H + (size_t)lane * H + h, 1);
+  } else if (kind == DIT_O || kind == DIT_DOWN) {
+    int N, Kd;
+    dit_gemm_shape(P, kind, &N, &Kd);
+    const int S = P.splits[kind], kbs = Kd / TC_BK, z = cta % S;
+    const int c0 = (z * kbs / S) * TC_BK, c1 = ((z + 1) * kbs / S) * TC_BK;
+    // 128-column groups of the input this k-slice reads (a head, or an up tile)
+    const int g0 = c0 / 128, g1 = (c1 - 1) / 128;
+    const unsigned* f = kind == DIT_O ? P.f_head + (size_t)l * H : P.f_up + (size_t)l * (P.F / TC_BM);
+    for (int g = g0 + lane; g <= g1 && ok; g += 32) ok = dit_wait(P, f + g, 1);
   }
-  int N, Kd;
-  dit_gemm_shape(P, kind, &N, &Kd);
-  const int S = P.splits[kind], kbs = Kd / TC_BK, z = cta % S;
-  const int c0 = (z * kbs / S) * TC_BK, c1 = ((z + 1) * kbs / S) * TC_BK;
-  // 128-column groups of the input this k-slice reads (a head, or an up tile)
-  const int g0 = c0 / 128, g1 = (c1 - 1) / 128;
-  const unsigned* f = kind == DIT_O ? P.f_head + (size_t)l * H : P.f_up + (size_t)l * (P.F / TC_BM);
-  for (int g = g0; g <= g1; ++g)
-    if (!dit_wait(P, f + g, 1)) return false;
-  return true;
+  return __all_sync(0xffffffffu, ok);
 }
 
 // Per-row mean and sum of squared deviations over the 128 features held by
@@ -649,7 +655,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
       }
       if (kind != -1) {
         // wait for the units whose outputs this one reads
-        if (et == 0) sh->ok[it & 1] = dit_wait_deps(P, kind, l, cta) ? 1 : 0;
+        if (et < 32) {
+          const bool ok = dit_wait_deps_warp(P, kind, l, cta, et);
+          if (et == 0) sh->ok[it & 1] = ok ? 1 : 0;
+        }
         named_sync(1, 128);
         if (!sh->ok[it & 1]) { *abort = 1; break; }
         ++it;
