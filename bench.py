@@ -597,7 +597,7 @@ def dataclasses_replace_B1(w):
     return dataclasses.replace(w, B=1, temps=w.temps[:1])
 
 
-def run_reference(args, w):
+def run_reference(args, w, world: int = 1):
     wr = dataclasses_replace_B1(w)
     times, cores = oracle_rounds(w, budget_s=1e9, max_rounds=args.steps, warmup=args.warmup)
     sec = sum(times)
@@ -606,11 +606,11 @@ def run_reference(args, w):
     sample = (f"{len(times)} whole rounds of sequence 0 of {w.name} (context rows, "
               f"{wr.n_noise} noise draft(s) x K={w.shape.K}, verify) per timed step set")
     return {"impl": "reference", "metric": METRIC, "value": round(v, 5), "unit": "blocks/s",
-            "n_gpus": 1, "steps": len(times), "warmup": args.warmup,
+            "n_gpus": world, "steps": len(times), "warmup": args.warmup,
             "ms_per_step": round(sec / len(times) * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded fm_synth inputs; no trained weights)",
-            "config": workload_config(w, len(times) + args.warmup, 1),
+            "config": workload_config(w, len(times) + args.warmup, world),
             "cpu_baseline": {"value": round(v, 5), "unit": "blocks/s", "cores": cores,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(v, 5), "unit": "blocks/s", "h2d_bytes_per_step": 0,
@@ -631,7 +631,8 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return 0
-        print(json.dumps(run_reference(args, w)), flush=True)
+        # rank 0 alone times the oracle on the host cores for the job
+        print(json.dumps(run_reference(args, w, world)), flush=True)
         return 0
     line = run_fm(args, w, rank, world, local_rank)
     if rank == 0:
