@@ -122,15 +122,41 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- algorithmic bytes
-def source_sha1() -> str:
-    """Hash of the kernel sources; a stored ncu traffic figure is reported
-    only while it matches (the kernels have not changed since the capture)."""
+def _strip_comments(text: str) -> str:
+    """C/C++/CUDA source without comments and blank lines (string and
+    character literals kept)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (ln.rstrip() for ln in "".join(out).splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
+def source_sha1(root: str = ROOT) -> str:
+    """Hash of the kernel sources without comments; a stored ncu traffic
+    figure is reported only while it matches (the kernels have not changed
+    since the capture)."""
     import hashlib
     h = hashlib.sha1()
-    csrc = os.path.join(ROOT, "step_flow_map_b200", "csrc")
+    csrc = os.path.join(root, "step_flow_map_b200", "csrc")
     for f in sorted(os.listdir(csrc)) + ["../../include/flashmap.h"]:
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            h.update(f.encode() + _strip_comments(fh.read()).encode())
     return h.hexdigest()
 
 

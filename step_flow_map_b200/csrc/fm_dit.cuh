@@ -7,22 +7,27 @@
 //
 //   stats, then per block l: QKV, attention, O (+ gated residual),
 //   MLP-up (+ GELU), MLP-down (+ gated residual); then the final modulated
-//   LayerNorm that feeds the LM head,
+//   LayerNorm that feeds the LM head.
 //
-// separated by grid barriers.  The producer warp never waits on a barrier:
-// it streams the weight tiles of the next phase into the shared-memory ring
-// while the current phase finishes, so the HBM weight stream runs
-// back to back.  Activations (the B operand, at most 64 rows) are written
-// straight into shared memory by the epilogue warps: the modulated
-// LayerNorm LN0(x)(1 + scale) + shift for QKV and MLP-up, a copy for O and
-// MLP-down.  LayerNorm statistics travel as per-128-feature partials (mean,
-// sum of squared deviations) written by the producing epilogue and combined
-// in a fixed order (Chan et al.'s pairwise update), so no phase re-reads
-// whole rows.  Context rows appended since the last draft ride along in the
-// QKV phases as extra B rows and get their keys and values written to the
-// cache.  Split-K partials are reduced by the last arriving CTA of a tile;
-// every wait (mbarrier or grid barrier) is bounded and an expired wait
-// aborts the pass with an error code.
+// There is no grid barrier: each unit of a phase (an output tile x K split,
+// or an attention item) waits only for the counters of the units whose
+// outputs it reads (release/acquire handoffs; one epilogue warp polls a
+// counter per lane).  The producer warp never waits on another CTA: it
+// streams the weight tiles of the next units into the shared-memory ring
+// while the current one finishes.  Activations (the B operand, at most 64
+// rows) are written straight into shared memory by the epilogue warps —
+// the modulated LayerNorm LN0(x)(1 + scale) + shift for QKV and MLP-up, a
+// copy for O and MLP-down — and published to the MMA warp per 8 k-blocks.
+// LayerNorm statistics travel as per-128-feature partials (mean, sum of
+// squared deviations) written by the producing epilogue and combined in a
+// fixed order (Chan et al.'s pairwise update), so no phase re-reads whole
+// rows.  Context rows appended since the last draft ride along in the QKV
+// phases as extra B rows and get their keys and values written to the
+// cache.  Split-K partials are pulled by the last arriving CTA of a tile
+// with bulk copies and reduced in shared memory.  Every wait (mbarrier or
+// counter) is bounded and an expired wait aborts the pass with an error
+// code.  Unrolled loops hold one code path each: rare cases inside them cost
+// as much as common ones.
 #pragma once
 #include "fm_attn.cuh"
 #include "fm_simt.cuh"

@@ -92,3 +92,9 @@ def test_acceptance_stats():
     assert st["p_reach"][0] == 0.75      # three of four reach position 1
     assert st["p_reach"][3] == 0.25      # only the full block passes position 4
     assert st["p_reach"][15] == 0.25
+
+
+def test_source_hash_ignores_comments_only():
+    src = 'const char* s = "a // b"; // note\n/* block */ int x = 1;  \n\n'
+    assert bench._strip_comments(src) == 'const char* s = "a // b";\n int x = 1;'
+    assert bench._strip_comments("int y = '\\''; // c") == "int y = '\\'';"
