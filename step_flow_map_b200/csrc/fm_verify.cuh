@@ -38,9 +38,20 @@ k_verify_greedy(const float* __restrict__ tgt, const int* __restrict__ draft, in
   const int v0 = min(V, c * per), v1 = min(V, v0 + per);
   const float* r = tgt + (size_t)row * V;
   ArgMax a{-INFINITY, 0x7fffffff};
-  for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x) {
-    float x = r[v];
-    if (am_better(x, v, a.v, a.i)) { a.v = x; a.i = v; }
+  // eight strided loads in flight per thread before they are compared (the
+  // comparison is order-independent: ties go to the lowest index)
+  for (int base = v0 + (int)threadIdx.x; base < v1; base += 8 * (int)blockDim.x) {
+    float x[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int v = base + u * (int)blockDim.x;
+      x[u] = v < v1 ? __ldcs(r + v) : -INFINITY;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int v = base + u * (int)blockDim.x;
+      if (v < v1 && am_better(x[u], v, a.v, a.i)) { a.v = x[u]; a.i = v; }
+    }
   }
   a = block_argmax(a, shv, shi);
   if (threadIdx.x == 0) {
