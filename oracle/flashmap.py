@@ -185,8 +185,16 @@ def flow_map_update(x: np.ndarray, D: np.ndarray, s: float, t: float) -> np.ndar
 
 # ---------------------------------------------------------------- token choice
 def argmax_lowest(row: np.ndarray) -> int:
-    """Index of the largest entry; ties go to the lowest index."""
-    return int(np.argmax(row))
+    """Index of the largest entry; ties go to the lowest index.
+
+    NaN entries never win: they rank below every number, -inf included.  A
+    row with no entry other than NaN gives index 0.
+    """
+    row = np.asarray(row)
+    ok = np.flatnonzero(~np.isnan(row))
+    if ok.size == 0:
+        return 0
+    return int(ok[np.argmax(row[ok])])
 
 
 def inverse_cdf(weights: np.ndarray, u: float) -> int:

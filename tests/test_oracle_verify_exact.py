@@ -86,7 +86,11 @@ def _target_table(rng, V, K):
     return table
 
 
-def _check_lossless(V, K, N, seed, greedy_draft=False):
+def _check_lossless(V, K, N, seed, greedy_draft=False, T=1.0):
+    """Exact output distribution of the oracle's stochastic verify at
+    temperature T.  Logits are T * log(probabilities), so softmax(logits / T)
+    is the intended distribution: a verify that multiplies by T where it should
+    divide (or ignores T) breaks the equality unless T = 1."""
     rng = np.random.default_rng(seed)
     table = _target_table(rng, V, K)
     qs = []
@@ -99,8 +103,8 @@ def _check_lossless(V, K, N, seed, greedy_draft=False):
         drafts = [tuple(tuple(int(np.argmax(qs[j][i])) for i in range(K)) for j in range(N))]
     for ys in drafts:
         pq = 1.0 if greedy_draft else float(np.prod([qs[j][i][ys[j][i]] for j in range(N) for i in range(K)]))
-        target = np.array([[np.log(table[ys[j][:i]]) for i in range(K + 1)] for j in range(N)])
-        dlog = None if greedy_draft else np.array([np.log(qs[j]) for j in range(N)])
+        target = T * np.array([[np.log(table[ys[j][:i]]) for i in range(K + 1)] for j in range(N)])
+        dlog = None if greedy_draft else T * np.array([np.log(qs[j]) for j in range(N)])
         qd = [[(np.eye(V)[ys[j][i]] if greedy_draft else qs[j][i]) for i in range(K)] for j in range(N)]
 
         # every distribution any uniform can be compared against
@@ -132,7 +136,7 @@ def _check_lossless(V, K, N, seed, greedy_draft=False):
         def run(assign):
             ua = _LazyRows(assign, N, K)
             ur = _LazyU(assign, ("r",))
-            n, branch, toks = fm.verify_sample(target, dlog, ys, 1.0, ua, ur)
+            n, branch, toks = fm.verify_sample(target, dlog, ys, T, ua, ur)
             return tuple(toks)
 
         for toks, w in _enumerate(run, bps).items():
@@ -160,6 +164,23 @@ def test_lossless_tree_two_drafts_V4_K2():
 
 def test_lossless_greedy_draft_stochastic_verify():
     _check_lossless(V=5, K=3, N=1, seed=13, greedy_draft=True)
+
+
+# Temperature other than 1: the target and draft distributions are
+# softmax(logits / T) (page "FlashMap并行草拟加速大模型解码", section "能拿来做什么":
+# probabilistic draft sampling at T > 0; lossless at the same sampling settings,
+# page "FlashMap Drafts 16 Dependent Tokens at Once…", "Why drafting still costs time").
+@pytest.mark.parametrize("T", [2.0, 0.5])
+def test_lossless_single_draft_V5_K2_temperature(T):
+    _check_lossless(V=5, K=2, N=1, seed=14, T=T)
+
+
+def test_lossless_tree_two_drafts_V4_K2_T2():
+    _check_lossless(V=4, K=2, N=2, seed=12, T=2.0)
+
+
+def test_lossless_greedy_draft_T2():
+    _check_lossless(V=5, K=3, N=1, seed=13, greedy_draft=True, T=2.0)
 
 
 def test_accept_probabilities():
