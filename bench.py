@@ -72,7 +72,7 @@ class ClockSampler:
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, torch_dev: int, period=0.02):
+    def __init__(self, torch_dev: int, period=0.002):
         self.samples, self.reasons, self.ok = [], set(), False
         self.period, self.stop_ev = period, threading.Event()
         try:
@@ -231,6 +231,16 @@ def algorithmic_flops(w: fs.Workload):
             "dit_gemm": 2 * M * dit_params * steps, "attn": attn * steps}
 
 
+def persistent_pass(w: fs.Workload) -> bool:
+    """True when the library runs the DiT as its persistent pass (one
+    sequence, one noise draft, bf16, 128-wide heads) and so projects the
+    round's new context rows inside that pass's QKV phases, with the key and
+    value weights it streams anyway."""
+    s = w.shape
+    return (w.dtype == "bf16" and w.B == 1 and w.n_noise == 1 and s.K == 16 and s.dh == 128
+            and s.K + w.new_rows <= 64)
+
+
 def algorithmic_bytes(w: fs.Workload):
     """Bytes each kernel class must move per step (weights, activations, caches)."""
     s = w.shape
@@ -247,7 +257,10 @@ def algorithmic_bytes(w: fs.Workload):
     dit = nb * (3 * d * d + d * d + 2 * d * F) * e                     # block weights
     attn = nb * w.B * ctx_rows * 2 * d * e                             # context keys/values
     ctx = (w.B * w.new_rows * (s.n_taps * s.hidden * e + d * 4)
-           + s.n_taps * s.hidden * d * e + nb * 2 * d * d * e)        # hidden, fc, K/V weights
+           + s.n_taps * s.hidden * d * e)                              # hidden rows, fc
+    if w.new_rows and not persistent_pass(w):
+        ctx += nb * 2 * d * d * e    # K/V weights of a separate projection; inside the persistent
+        #                              pass they are the QKV weights the DiT already streams
     verify = w.B * w.n_noise * (s.K + 1) * V * 4
     return {"embed": embed * steps, "lm_head": lm * steps, "dit_gemm": dit * steps,
             "attn": attn * steps, "context": ctx, "verify": verify,
@@ -647,11 +660,55 @@ def log(msg):
     print(f"[bench] {msg}", file=sys.stderr, flush=True)
 
 
+# ---------------------------------------------------------------- local ranks
+def _rank_entry(env: dict, entry, entry_args) -> None:
+    os.environ.update(env)
+    rc = entry(*entry_args)
+    sys.exit(int(rc or 0))
+
+
+def launch_local(n: int, entry, *entry_args, timeout_s: float = 3600.0) -> None:
+    """Start n local ranks, one process each, with the environment a torchrun
+    launch gives them (RANK, LOCAL_RANK, WORLD_SIZE, MASTER_ADDR=127.0.0.1,
+    MASTER_PORT), run entry(*entry_args) in each, and wait.  Raises when a
+    rank fails or outlives the timeout (it is then terminated)."""
+    import socket
+
+    import torch.multiprocessing as mp
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    ctx = mp.get_context("spawn")
+    procs = []
+    for r in range(n):
+        env = {"RANK": str(r), "LOCAL_RANK": str(r), "WORLD_SIZE": str(n),
+               "LOCAL_WORLD_SIZE": str(n), "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)}
+        p = ctx.Process(target=_rank_entry, args=(env, entry, entry_args))
+        p.start()
+        procs.append(p)
+    t_end = time.time() + timeout_s
+    codes = []
+    for p in procs:
+        p.join(max(1.0, t_end - time.time()))
+        if p.is_alive():
+            p.terminate()
+            p.join(30)
+        codes.append(p.exitcode)
+    if any(c != 0 for c in codes):
+        raise RuntimeError(f"local ranks exited with codes {codes}")
+
+
 def main():
     faulthandler.enable()
     args = parse()
+    launched = "WORLD_SIZE" in os.environ
+    if args.impl == "fm" and args.gpus > 1 and not launched:
+        # no launcher: start one rank per GPU here (replicas, NCCL for the
+        # barrier and the two reductions), each re-running this entry point
+        launch_local(args.gpus, main)
+        return 0
     rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
+    world = int(os.environ.get("WORLD_SIZE", str(args.gpus if args.impl == "reference" else 1)))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     w = fs.WORKLOADS[args.workload]
     if args.impl == "reference":

@@ -134,7 +134,8 @@ fm_status fm_project_context(fm_ctx *ctx, const int32_t *seq_ids, int n_seqs,
  *   noise        device [n_seqs, n_noise, K, V] dtype
  *   t_grid       host [num_steps + 1], 0 = t0 < t1 < ... < t_S = 1
  *   num_steps    1 .. FM_MAX_STEPS (one step is the flow map's single jump)
- *   temperature  host [n_seqs]; 0 selects the argmax (lowest index on ties),
+ *   temperature  host [n_seqs]; 0 selects the argmax (lowest index on ties;
+ *                a NaN logit never wins, a row of NaN gives token 0),
  *                T > 0 samples softmax(logits / T) by inverse CDF
  *   u_draft      device [n_seqs, n_noise, K] uniforms in [0, 1) for sampled
  *                sequences; may be NULL when every temperature is 0
@@ -160,7 +161,8 @@ fm_status fm_draft(fm_ctx *ctx, const int32_t *seq_ids, int n_seqs,
  *   branch        device [B] out: the draft with the largest n (lowest on ties)
  *   out_tokens    device [B, K+1] out: the n accepted tokens, then the
  *                 target argmax at position n+1, then -1 padding
- * Argmax ties go to the lowest index; NaN never wins.  Bit-exact. */
+ * Argmax ties go to the lowest index; NaN never wins (it ranks below every
+ * number, -inf included; a row of NaN gives token 0).  Bit-exact. */
 fm_status fm_verify_greedy(fm_ctx *ctx, const float *target_logits, const int32_t *draft,
                            int B, int N, int K, int V,
                            int32_t *n_acc, int32_t *branch, int32_t *out_tokens,
@@ -191,8 +193,9 @@ fm_status fm_verify_sample(fm_ctx *ctx, const float *target_logits, const float 
  * cannot allocate device memory -- servers whose arena owns the whole
  * device, or verify-only users without a drafter context.  Its scratch is a
  * fixed device array inside the library (about 260 KB on every GPU that
- * loads it, kept until exit), so: B <= 1024, N*(K+1) <= 1024 and
- * B*N*(K+1) <= 32768, else FM_ERR_UNSUPPORTED.  The first call on a device
+ * loads it, kept until exit), so: B <= 1024, N*(K+1) <= 1024,
+ * B*N*(K+1) <= 32768 and V <= 2^28, else FM_ERR_UNSUPPORTED (checked on
+ * the host before anything is queued).  The first call on a device
  * looks the array up (cudaGetSymbolAddress) and should come before any
  * stream capture.  Each call clears the scratch counters it uses; all calls
  * share the one array, so calls that overlap on the same GPU (issued on

@@ -1120,6 +1120,7 @@ extern "C" fm_status fm_device_status(fm_ctx* c, fm_stream stream) {
 // library holds this array (about 260 KB) until the process exits.
 #define FM_NOALLOC_PARTIALS 32768  /* (row, vocabulary chunk) partials */
 #define FM_NOALLOC_SEQS 1024       /* sequences per call */
+#define FM_NOALLOC_MAX_V (1 << 28)  /* vocabulary entries per row */
 
 namespace {
 struct NoallocScratch {
@@ -1161,23 +1162,31 @@ extern "C" fm_status fm_verify_greedy_noalloc(const float* target_logits, const 
   if (!target_logits || !draft || !n_acc || !branch || !out_tokens)
     return set_err(FM_ERR_ARG, "NULL argument");
   if (B < 1 || N < 1 || K < 1 || V < 1) return set_err(FM_ERR_ARG, "sizes must be positive");
+  // each factor is bounded before any product is formed, and every product
+  // is taken in 64 bits, so no size can wrap past these checks
   if (B > FM_NOALLOC_SEQS)
     return set_err(FM_ERR_UNSUPPORTED, "B=%d exceeds the no-allocation limit of %d sequences", B,
                    FM_NOALLOC_SEQS);
-  if (N * (K + 1) > fm::VG_MAX_ROWS)
-    return set_err(FM_ERR_UNSUPPORTED, "N*(K+1)=%d exceeds %d rows per sequence", N * (K + 1),
+  if (N > fm::VG_MAX_ROWS || K > fm::VG_MAX_ROWS - 1)
+    return set_err(FM_ERR_UNSUPPORTED, "N=%d or K=%d exceeds %d rows per sequence", N, K,
                    fm::VG_MAX_ROWS);
-  const long rows = (long)B * N * (K + 1);
+  if (V > FM_NOALLOC_MAX_V)
+    return set_err(FM_ERR_UNSUPPORTED, "V=%d exceeds %d", V, FM_NOALLOC_MAX_V);
+  const int64_t rows_b = (int64_t)N * ((int64_t)K + 1);
+  if (rows_b > fm::VG_MAX_ROWS)
+    return set_err(FM_ERR_UNSUPPORTED, "N*(K+1)=%lld exceeds %d rows per sequence",
+                   (long long)rows_b, fm::VG_MAX_ROWS);
+  const int64_t rows = (int64_t)B * rows_b;
   if (rows > FM_NOALLOC_PARTIALS)
-    return set_err(FM_ERR_UNSUPPORTED, "B*N*(K+1)=%ld exceeds the no-allocation limit of %d rows",
-                   rows, FM_NOALLOC_PARTIALS);
+    return set_err(FM_ERR_UNSUPPORTED, "B*N*(K+1)=%lld exceeds the no-allocation limit of %d rows",
+                   (long long)rows, FM_NOALLOC_PARTIALS);
   NoallocScratch* s = nullptr;
   int sms = 148;
   FM_TRY(noalloc_scratch(&s, &sms));
-  long want = (2L * sms + rows - 1) / rows;
-  int ch = (int)std::min<long>(want, 64);
+  const int64_t want = (2 * (int64_t)sms + rows - 1) / rows;
+  int ch = (int)std::min<int64_t>(want, 64);
   ch = std::min(ch, std::max(1, V / 1024));
-  ch = (int)std::min<long>(ch, FM_NOALLOC_PARTIALS / rows);
+  ch = (int)std::min<int64_t>(ch, FM_NOALLOC_PARTIALS / rows);
   ch = std::max(ch, 1);
   cudaStream_t st = (cudaStream_t)stream;
   // the counters start at zero (the kernel also returns them to zero)

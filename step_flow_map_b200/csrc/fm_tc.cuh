@@ -238,7 +238,10 @@ __device__ __forceinline__ void tc_finish_chunk(const Epi& epi, const TcArgs& a,
     const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-      ArgMax am{n < a.N ? v[j] : -INFINITY, n < a.N ? n : 0x7fffffff};
+      // a NaN logit enters as "no candidate", so it never wins (not even
+      // against -inf) and cannot stick in the shuffle tree
+      const bool ok = n < a.N && v[j] == v[j];
+      ArgMax am{ok ? v[j] : -INFINITY, ok ? n : 0x7fffffff};
       am = warp_argmax(am);
       if (lane == 0) {
         red_v[q * BN + j0 + j] = am.v;

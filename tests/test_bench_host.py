@@ -98,3 +98,60 @@ def test_source_hash_ignores_comments_only():
     src = 'const char* s = "a // b"; // note\n/* block */ int x = 1;  \n\n'
     assert bench._strip_comments(src) == 'const char* s = "a // b";\n int x = 1;'
     assert bench._strip_comments("int y = '\\''; // c") == "int y = '\\'';"
+
+
+def _env_rank_main(out_dir):
+    # a rank started by bench.launch_local: everything comes from the
+    # environment, as under torchrun
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    rank, world = int(os.environ["RANK"]), int(os.environ["WORLD_SIZE"])
+    assert os.environ["MASTER_ADDR"] == "127.0.0.1"
+    dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    try:
+        ms, verified = bench.reduce_over_ranks(dist, "cpu", 2.0 * (rank + 1), 5.0, world)
+        t = torch.tensor([float(rank)])
+        dist.all_reduce(t)
+        with open(os.path.join(out_dir, f"r{rank}"), "w") as f:
+            f.write(f"{world} {int(os.environ['LOCAL_RANK'])} {ms} {verified} {t.item()}")
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+    return 0
+
+
+def _failing_rank():
+    return 3 if os.environ["RANK"] == "1" else 0
+
+
+def test_self_launch_two_gloo_ranks(tmp_path):
+    # `bench.py --gpus N` without torchrun starts its N ranks itself
+    bench.launch_local(2, _env_rank_main, str(tmp_path), timeout_s=180)
+    for r in range(2):
+        world, local, ms, verified, s = (tmp_path / f"r{r}").read_text().split()
+        assert (int(world), int(local)) == (2, r)
+        assert float(ms) == pytest.approx(4.0) and float(verified) == pytest.approx(10.0)
+        assert float(s) == pytest.approx(1.0)
+
+
+def test_self_launch_reports_a_failed_rank():
+    with pytest.raises(RuntimeError):
+        bench.launch_local(2, _failing_rank, timeout_s=120)
+
+
+def test_8b_bs1_step_bytes_match_the_survey_count():
+    # the concurrency-1 8B round moves ~1.999 GB: E, W_lm, block weights,
+    # fc, context keys/values, noise and target logits; the key/value
+    # weights of the round's new context rows are the QKV weights the
+    # persistent pass streams anyway and are not counted twice
+    w = fs.WORKLOADS["qwen3_8b_bs1"]
+    ab = bench.algorithmic_bytes(w)
+    total = sum(ab[k] for k in ("embed", "lm_head", "dit_gemm", "attn", "context", "verify"))
+    assert bench.persistent_pass(w)
+    assert total == pytest.approx(1.999e9, rel=2e-3)
+    w5 = fs.WORKLOADS["qwen3_8b_bs64"]
+    assert not bench.persistent_pass(w5)
+    d = w5.shape.d
+    assert bench.algorithmic_bytes(w5)["context"] > 6 * 2 * d * d * 2   # separate K/V projection

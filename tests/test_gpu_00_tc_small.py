@@ -118,3 +118,34 @@ def test_tc_two_step():
             y, sure = gu.sampled_token_sure(ref["logits"][j, i], 1.0, ri.u_draft[0, j, i])
             if sure:
                 assert tok[0, j, i] == y
+
+
+def test_nan_logit_never_wins():
+    # a NaN row of the LM head makes one token's logit NaN in every row; the
+    # fused LM-head argmax (no logits written) and the stored-logits path
+    # must both skip it, as the oracle's argmax does
+    w = _workload(1, 1)
+    ref0 = gu.oracle_draft(w, 0, 0)
+    vstar = int(np.argmax(ref0["logits"][0, 0]))
+    W = {k: v.copy() for k, v in gu.weights(w.shape, w.dtype).items()}
+    W["W_lm"][vstar] = np.nan
+    W64 = {k: v.astype(np.float64) for k, v in W.items()}
+    rows = np.concatenate([fs.prefill_hidden(w, 0), fs.round_inputs(w, 0).new_hidden[0]], axis=0)
+    _, kv = om.project_context(W64, w.shape.n_blocks, rows)
+    ri = fs.round_inputs(w, 0)
+    ref = om.draft(W64, w.shape, kv, ri.noise[0], w.t_grid)
+    assert (ref["tokens"] != vstar).all()
+    clean = np.where(np.isnan(ref["logits"]), -np.inf, ref["logits"])
+    sure = om.margins(clean) > gu.MARGIN
+    assert sure.sum() >= 4
+    for logits in (False, True):
+        ctx = Context(w.shape, w.dtype, W, max_ctx=w.ctx + 40, max_seqs=1, max_noise=1, max_new=64)
+        gu.gpu_prefill(ctx, w, [0], max_new=64)
+        gu.gpu_new_rows(ctx, w, 0, [0])
+        tok, _ = ctx.draft([0], to_device(ri.noise, "bf16"), w.t_grid, w.temps, logits=logits)
+        torch.cuda.synchronize()
+        fm_device_status(ctx.ctx)
+        got = gu.to_np(tok)[0]
+        assert (got != vstar).all(), logits
+        np.testing.assert_array_equal(got[sure], ref["tokens"][sure])
+        ctx.close()

@@ -111,6 +111,29 @@ def test_verify_greedy_exact(B, N):
     ctx.close()
 
 
+def test_verify_greedy_nan_rows():
+    # NaN never wins (it ranks below -inf); a row of NaN gives token 0
+    V, K, B = 2053, 16, 3
+    w = dataclasses.replace(fs.WORKLOADS["qwen3_8b_bs1"], B=B,
+                            shape=dataclasses.replace(fs.QWEN3_8B, V=V, K=K))
+    rng = np.random.default_rng(9)
+    tgt = rng.normal(size=(B, 1, K + 1, V)).astype(np.float32)
+    tok = tgt.argmax(-1)[:, :, :K].astype(np.int64)
+    tgt[0, 0, 2, tok[0, 0, 2]] = np.nan          # the argmax itself turns NaN: n = 2
+    tgt[1, 0, 0, :] = np.nan
+    tok[1, 0, 0] = 0
+    tgt[2, 0, 4, :] = -np.inf
+    tgt[2, 0, 4, :100] = np.nan
+    tok[2, 0, 4] = 100
+    ctx = gu.make_ctx(dataclasses.replace(w, ctx=4, new_rows=1), max_new=4)
+    n, br, out = ctx.verify_greedy(to_device(tgt), to_device(tok.astype(np.int32)))
+    want = gu.verify_oracle_all(tgt, None, tok, 0, None, None, True)
+    np.testing.assert_array_equal(gu.to_np(n), want[0])
+    np.testing.assert_array_equal(gu.to_np(out), want[2])
+    assert list(want[0]) == [2, 16, 16]
+    ctx.close()
+
+
 def test_verify_greedy_ties_and_ragged_vocab():
     # constant rows: every index ties, the lowest wins; odd V leaves a ragged tail
     V, K, B = 1001, 16, 2
@@ -205,6 +228,40 @@ def test_two_step_tree_sampled():
     ctx.close()
 
 
+def test_bench_path_8b_bs1_fused_argmax_rounds():
+    # the exact path the concurrency-1 bench times: the round's new context
+    # rows projected inside the persistent DiT pass, then the LM head with
+    # the fused per-tile argmax (no logits written) and the token selection
+    # over its 1,187 tile partials -- over four rounds whose appended rows
+    # accumulate in the cache
+    w = fs.WORKLOADS["qwen3_8b_bs1"]
+    rounds = 4
+    ctx = gu.Context(w.shape, w.dtype, gu.weights(w.shape, w.dtype),
+                     max_ctx=w.ctx + rounds * w.new_rows + 8, max_seqs=1, max_noise=1, max_new=512)
+    gu.gpu_prefill(ctx, w, [0])
+    rows = [fs.prefill_hidden(w, 0)]
+    W = gu.weights64(w.shape, w.dtype)
+    checked = 0
+    for r in range(rounds):
+        ri = fs.round_inputs(w, r)
+        ctx.project([0], to_device(ri.new_hidden, "bf16"), [w.ctx + r * w.new_rows])
+        rows.append(ri.new_hidden[0])
+        tok, none = ctx.draft([0], to_device(ri.noise, "bf16"), w.t_grid, w.temps, logits=False)
+        assert none is None
+        _, kv = om.project_context(W, w.shape.n_blocks, np.concatenate(rows, axis=0))
+        ref = om.draft(W, w.shape, kv, ri.noise[0], w.t_grid)
+        checked += gu.assert_tokens_on_margin(gu.to_np(tok)[0], ref["logits"], f"round {r}")
+    assert checked >= 8
+    ctx.close()
+
+
+# sequences of the batch-64 round checked against the oracle: both halves
+# (greedy 0..31, sampled 32..63) and every 128-row activation tile; the
+# oracle projects 4,113 context rows per sequence, so the whole batch would
+# take minutes on the host
+BS64_CHECK = (0, 5, 13, 21, 30, 31, 32, 33, 40, 47, 55, 63)
+
+
 def test_bs64_mixed_sampled_rows():
     w = fs.WORKLOADS["qwen3_8b_bs64"]
     ctx = gu.make_ctx(w, max_new=1024)
@@ -217,11 +274,15 @@ def test_bs64_mixed_sampled_rows():
                         u_draft=to_device(ri.u_draft))
     lg_np = gu.to_np(lg)
     tok_np = gu.to_np(tok)
-    for b in (0, 47):
+    for b in BS64_CHECK:
         ref = gu.oracle_draft(w, b, r)
         gu.assert_logits_close(lg_np[b], ref["logits"], "bf16", f"bs64 seq {b}")
         if w.temps[b] == 0:
             gu.assert_tokens_on_margin(tok_np[b], ref["logits"], f"bs64 seq {b}")
+        else:
+            for i in range(w.shape.K):
+                assert gu.sampled_token_near(ref["logits"][0, i], w.temps[b], ri.u_draft[b, 0, i],
+                                             int(tok_np[b, 0, i])), (b, i)
     del lg
     # mixed verify on synthetic inputs: greedy for the first half, T=1 for the rest
     rng = np.random.default_rng(3)

@@ -61,6 +61,31 @@ def test_noalloc_matches_context_verify_twice():
         for g, wv in zip(got, want):
             np.testing.assert_array_equal(g, wv)
     assert want1[0].max() > 0 and want2[0].max() > 0
+    # and both against the fp64 oracle's greedy verify directly
+    for got, tgt, tok in ((got1, tgt1, tok1), (got2, tgt2, tok2)):
+        ref = gu.verify_oracle_all(gu.to_np(tgt), None, gu.to_np(tok), 0, None, None, True)
+        for g, wv in zip(got, ref):
+            np.testing.assert_array_equal(g, wv)
+
+
+def test_noalloc_nan_and_ties_match_the_oracle():
+    # NaN never wins (it ranks below -inf), ties go to the lowest index, a
+    # row of NaN gives token 0
+    B, N, K, V = 2, 1, 16, 4099
+    tgt = np.zeros((B, N, K + 1, V), np.float32)
+    tok = np.zeros((B, N, K), np.int64)
+    tgt[0, 0, :, 7] = 1.0
+    tok[0, 0, :] = 7
+    tgt[0, 0, 3, 7] = np.nan                 # row 3: 7 is NaN, so the argmax is the lowest tie 0
+    tgt[1, 0, 0, :] = np.nan                 # a row of NaN -> token 0
+    tgt[1, 0, 1, :] = -np.inf
+    tgt[1, 0, 1, :5] = np.nan                # NaN below -inf: the argmax is 5
+    tok[1, 0, 1] = 5
+    got = _noalloc(to_device(tgt), to_device(tok.astype(np.int32)))
+    ref = gu.verify_oracle_all(tgt, None, tok, 0, None, None, True)
+    for g, wv in zip(got, ref):
+        np.testing.assert_array_equal(g, wv)
+    assert list(ref[0]) == [3, 16]
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
@@ -68,6 +93,13 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     tgt = torch.zeros((1, 1, 17, 8), dtype=torch.float32, device="cuda")
     tok = torch.zeros((1, 1, 16), dtype=torch.int32, device="cuda")
     o = torch.zeros(4096, dtype=torch.int32, device="cuda")
-    with pytest.raises(FlashmapError) as e:   # B beyond 1024 sequences: no launch happens
-        fm_verify_greedy_noalloc(tgt, tok, 2000, 1, 16, 8, o, o, o)
-    assert e.value.status == FM_ERR_UNSUPPORTED
+    # every limit is checked on the host, before anything is queued
+    for B, N, K, V in ((2000, 1, 16, 8),          # more than 1024 sequences
+                       (1, 64, 16, 8),            # N*(K+1) = 1088 rows per sequence
+                       (1024, 2, 16, 8),          # B*N*(K+1) = 34816 rows
+                       (1, 1, 2**31 - 1, 8),      # K so large that N*(K+1) would wrap
+                       (1, 2**31 - 1, 16, 8),
+                       (1, 1, 16, 2**30)):        # V beyond 2^28
+        with pytest.raises(FlashmapError) as e:
+            fm_verify_greedy_noalloc(tgt, tok, B, N, K, V, o, o, o)
+        assert e.value.status == FM_ERR_UNSUPPORTED, (B, N, K, V)
