@@ -53,6 +53,9 @@ def parse():
     ap.add_argument("--profile-all", action="store_true", help="log per-class kernel times")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--factorised", action="store_true",
+                    help="also draft every round factorised (position i from its own noise "
+                         "block) and report both accepted-length histograms (untimed)")
     return ap.parse_args()
 
 
@@ -292,8 +295,9 @@ def run_fm(args, w, rank, world, local_rank):
     W = fs.make_weights(s, w.dtype)
     log("loading context")
     max_new = max(1, min(1024, w.ctx))
+    factorised = args.factorised and B <= 4 and all(t == 0 for t in w.temps)
     ctx = Context(s, w.dtype, W, max_ctx=w.ctx + max(w.new_rows, 1) + 8, max_seqs=B,
-                  max_noise=N, max_new=max(max_new, w.new_rows))
+                  max_noise=max(N, s.K) if factorised else N, max_new=max(max_new, w.new_rows))
     del W
     for b in seqs:
         h = fs.prefill_hidden(w, b)
@@ -587,6 +591,28 @@ def run_fm(args, w, rank, world, local_rank):
         line["e2e"] = {"value": round(B * N * args.steps * world / (ems / 1e3), 3),
                        "unit": "blocks/s", "h2d_bytes_per_step": int(h2d),
                        "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ems / args.steps, 5)}
+    if factorised:
+        # ablation, untimed: the same rounds drafted factorised (position i
+        # from its own independent noise block), verified against the same
+        # synthetic targets; those targets are built around the joint draft
+        # of a random-weight drafter, so this compares the two paths on one
+        # footing, not the trained drafters of the pages
+        n_f = torch.zeros((R, B), dtype=torch.int32, device="cuda")
+        for i in range(R):
+            rd = rounds[i]
+            if w.new_rows:
+                fmb.fm_project_context(ctx.ctx, seqs, rd["hidden"], w.new_rows, [w.ctx] * B, stream)
+            Xf = to_device(fs.factorised_noise(w, round_seed(i, rank)), w.dtype)
+            tok_f, _ = ctx.draft_factorised(seqs, Xf, w.t_grid, w.temps, logits=False)
+            fmb.fm_verify_greedy(ctx.ctx, rd["target"], tok_f.view(B, 1, K).contiguous(), B, 1, K, V,
+                                 n_f[i], branch, out_tok, stream)
+            del Xf
+        torch.cuda.synchronize()
+        line["ablation"] = {
+            "joint": acceptance_stats(n_all, K),
+            "factorised": acceptance_stats(n_f.cpu().numpy(), K),
+            "rounds": R,
+            "targets": "the joint draft's synthetic targets (random-weight drafter)"}
     ctx.close()
     if dist is not None:
         dist.destroy_process_group()

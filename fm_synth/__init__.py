@@ -239,6 +239,14 @@ def round_inputs(w: Workload, r: int) -> RoundInputs:
     return RoundInputs(noise, hid, u_draft, u_accept, u_res)
 
 
+def factorised_noise(w: Workload, r: int) -> np.ndarray:
+    """[B, K, K, V] noise of round r for factorised drafting: block i drafts
+    position i only, each block an independent N(0, 1) draw (seed 2000 + r,
+    stream 1; the joint draft of the same round uses stream 0)."""
+    s = w.shape
+    return _store(normal(2000 + r, (w.B, s.K, s.K, s.V), sub=1), w.dtype)
+
+
 def target_logits(w: Workload, r: int, draft_tokens: np.ndarray,
                   draft_logits: np.ndarray | None = None) -> np.ndarray:
     """Synthetic target rows [B, N, K+1, V] fp32 standing in for the target model.

@@ -151,6 +151,22 @@ fm_status fm_draft(fm_ctx *ctx, const int32_t *seq_ids, int n_seqs,
                    const float *temperature, const double *u_draft,
                    int32_t *tokens, float *draft_logits, fm_stream stream);
 
+/* Factorised drafting, the foil of the joint draft (P2 "Почему
+ * diffusion-драфтеры теряют в доле принятых токенов?": a drafter that picks
+ * each position on its own mixes modes, "new diego" / "san york", half the
+ * time): position i of the block comes from its own independent noise block,
+ * as if each position were drafted by a separate flow-map pass.
+ *   noise        device [n_seqs, K, K, V] dtype: noise block i for position i
+ *   u_draft      device [n_seqs, K] uniforms (position i), or NULL when greedy
+ *   tokens       device [n_seqs, K] out: token i of the draft of noise block i
+ *   draft_logits device [n_seqs, K, V] out (that draft's row i), or NULL
+ * Other arguments as for fm_draft.  Runs the K drafts of a sequence as one
+ * batched draft, so it needs max_noise >= K (else FM_ERR_UNSUPPORTED). */
+fm_status fm_draft_factorised(fm_ctx *ctx, const int32_t *seq_ids, int n_seqs,
+                              const void *noise, const float *t_grid, int num_steps,
+                              const float *temperature, const double *u_draft,
+                              int32_t *tokens, float *draft_logits, fm_stream stream);
+
 /* Greedy verify (P5 "Why drafting still costs time": keep the longest valid
  * prefix, resume from a target token; P2 "Что такое FlashMap?": the result
  * equals the target's own greedy output).
@@ -187,6 +203,59 @@ fm_status fm_verify_sample(fm_ctx *ctx, const float *target_logits, const float 
                            int32_t *n_acc, int32_t *branch, int32_t *out_tokens,
                            fm_stream stream);
 
+/* ---- Target-side tree scoring of a sequence's noise drafts (P1 "6.14 倍是最好
+ * 成绩…": four noise drafts scored as a tree add about 11 % mean speedup).
+ * Drafts that share a prefix need the target's distribution after it once:
+ * the target scores the nodes of the drafts' prefix trie in one pass, each
+ * node attending to the context and to its ancestors.  Node order is breadth
+ * first, and within a depth the order of the first draft that creates the
+ * node.  Node n is a prefix of length depth + 1 ending in its token; parent
+ * -1 at depth 0.  Target rows of a tree: row 0 is the root (the first
+ * drafted position's distribution), row 1 + n node n's. */
+
+/* Builds the trie of each sequence's N drafts.  No context, no allocation.
+ *   draft        device [B, N, K]
+ *   node_token, node_parent, node_depth  device [B, N*K] out; entries past
+ *                the sequence's node count are -1
+ *   n_nodes      device [B] out
+ *   draft_node   device [B, N, K] out: the node of draft j's prefix of
+ *                length i + 1
+ *   anc_mask     device [B, N*K, W] out, W = ceil(N*K / 64): bit m of node
+ *                n's words is set iff m is n or one of its ancestors
+ * Requires N <= 32 and N*K <= 1024 (else FM_ERR_UNSUPPORTED).  Exact. */
+fm_status fm_build_tree(const int32_t *draft, int B, int N, int K, int32_t *node_token,
+                        int32_t *node_parent, int32_t *node_depth, int32_t *n_nodes,
+                        int32_t *draft_node, uint64_t *anc_mask, fm_stream stream);
+
+/* The attention that scores a tree's nodes in one pass: node n's query
+ * attends over the context rows and over the rows of n and its ancestors
+ * (softmax scale 1/sqrt(dh)), per head.  fp32, no context, no allocation;
+ * a reference of the mask's meaning for a target's own attention.
+ *   q, k_nodes, v_nodes device [B, NN, n_heads*dh]; k_ctx, v_ctx device
+ *   [B, L, n_heads*dh] (L may be 0); anc_mask, n_nodes from fm_build_tree
+ *   (NN = N*K); out device [B, NN, n_heads*dh], rows past n_nodes untouched.
+ * Requires NN <= 1024 and dh <= 128. */
+fm_status fm_tree_attention(const float *q, const float *k_ctx, const float *v_ctx,
+                            const float *k_nodes, const float *v_nodes, const uint64_t *anc_mask,
+                            const int32_t *n_nodes, int B, int NN, int L, int n_heads, int dh,
+                            float *out, fm_stream stream);
+
+/* Greedy and stochastic verify of a tree whose target rows are given per
+ * node: node_logits device [B, R, V] fp32, R >= 1 + N*K (row 0 the root,
+ * row 1 + n node n), draft_node from fm_build_tree.  Results are those of
+ * fm_verify_greedy / fm_verify_sample on the per-draft rows the nodes stand
+ * for (shared prefixes share rows). */
+fm_status fm_verify_greedy_tree(fm_ctx *ctx, const float *node_logits, int R, const int32_t *draft,
+                                const int32_t *draft_node, int B, int N, int K, int V,
+                                int32_t *n_acc, int32_t *branch, int32_t *out_tokens,
+                                fm_stream stream);
+fm_status fm_verify_sample_tree(fm_ctx *ctx, const float *node_logits, int R,
+                                const float *draft_logits, const int32_t *draft,
+                                const int32_t *draft_node, int B, int N, int K, int V,
+                                float temperature, const double *u_accept, const double *u_res,
+                                int32_t *n_acc, int32_t *branch, int32_t *out_tokens,
+                                fm_stream stream);
+
 /* Greedy verify that allocates nothing and needs no context: same inputs,
  * outputs and bit-exact results as fm_verify_greedy (the pages have no
  * counterpart; this is a deployment variant).  It is for callers that
@@ -208,9 +277,12 @@ fm_status fm_verify_greedy_noalloc(const float *target_logits, const int32_t *dr
                                    fm_stream stream);
 
 /* Reads and clears the context's device error word: FM_OK, or
- * FM_ERR_TIMEOUT when a bounded wait inside a kernel gave up (the kernel
- * then stopped early and its outputs are invalid).  Waits for the work
- * queued on `stream`. */
+ * FM_ERR_TIMEOUT when a bounded wait inside a kernel gave up (about two
+ * seconds; the kernel then stopped early and the outputs of the calls since
+ * the last check are invalid).  On FM_ERR_TIMEOUT it also returns the
+ * context's arrival counters to zero, so the next call starts clean; context
+ * rows projected by the failed calls may be missing from the cache and are
+ * projected again by the caller.  Waits for the work queued on `stream`. */
 fm_status fm_device_status(fm_ctx *ctx, fm_stream stream);
 
 /* Kernel classes for launch counting and optional device timing. */

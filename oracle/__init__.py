@@ -25,9 +25,12 @@ Modules:
   "san diego"), used to check the flow-map update and shared-noise drafting.
 
 Parity status: the verify functions are pinned by exact enumeration of the
-target distribution and by the greedy-equals-target-greedy invariant; the
-zero-DiT draft by a hand-computed fixture; attention, LayerNorm, GELU,
-SiLU, the time features and the conditioning by closed forms.  The
+target distribution (at temperatures 1, 2 and 0.5) and by the
+greedy-equals-target-greedy invariant; the zero-DiT draft by hand-computed
+fixtures, one single-step and one two-step (the chain between flow-map
+steps at a sampling temperature other than 1); attention, LayerNorm, GELU,
+SiLU, the time features, the conditioning, tempered sampling and the
+argmax rule (ties lowest, NaN never wins) by closed forms.  The
 random-weight DiT as a whole has no printed values on the pages to pin it
 to, so its numeric identity with the authors' trained model is "parity
 unpinned": only its parts and the two independent formulations agree.

@@ -25,7 +25,8 @@ FM_MAX_STEPS = 8
 EXPORTS = (
     "fm_load_weights", "fm_free", "fm_last_error", "fm_project_context",
     "fm_draft", "fm_verify_greedy", "fm_verify_sample", "fm_profile", "fm_profile_read", "fm_device_status",
-    "fm_verify_greedy_noalloc",
+    "fm_verify_greedy_noalloc", "fm_draft_factorised", "fm_build_tree", "fm_tree_attention",
+    "fm_verify_greedy_tree", "fm_verify_sample_tree",
 )
 FM_PROF = {"embed": 0, "dit_gemm": 1, "attn": 2, "norm": 3, "lm_head": 4, "context": 5,
            "verify": 6, "other": 7}
@@ -80,6 +81,17 @@ def load_library(path: str = LIB_PATH):
     lib.fm_project_context.argtypes = [p, i32p, i, p, i, i32p, st]
     lib.fm_draft.restype = i
     lib.fm_draft.argtypes = [p, i32p, i, p, i, ctypes.POINTER(f), i, ctypes.POINTER(f), p, p, p, st]
+    lib.fm_draft_factorised.restype = i
+    lib.fm_draft_factorised.argtypes = [p, i32p, i, p, ctypes.POINTER(f), i, ctypes.POINTER(f), p, p,
+                                        p, st]
+    lib.fm_build_tree.restype = i
+    lib.fm_build_tree.argtypes = [p, i, i, i, p, p, p, p, p, p, st]
+    lib.fm_tree_attention.restype = i
+    lib.fm_tree_attention.argtypes = [p, p, p, p, p, p, p, i, i, i, i, i, p, st]
+    lib.fm_verify_greedy_tree.restype = i
+    lib.fm_verify_greedy_tree.argtypes = [p, p, i, p, p, i, i, i, i, p, p, p, st]
+    lib.fm_verify_sample_tree.restype = i
+    lib.fm_verify_sample_tree.argtypes = [p, p, i, p, p, p, i, i, i, i, f, p, p, p, p, p, st]
     lib.fm_verify_greedy.restype = i
     lib.fm_verify_greedy.argtypes = [p, p, p, i, i, i, i, p, p, p, st]
     lib.fm_verify_sample.restype = i
@@ -170,6 +182,46 @@ def fm_draft(ctx, seq_ids, noise, n_noise, t_grid, temperature, u_draft, tokens,
                                    _f32(t_grid), len(t_grid) - 1, _f32(temperature),
                                    _ptr(u_draft), _ptr(tokens), _ptr(draft_logits),
                                    _stream(stream)))
+
+
+def fm_draft_factorised(ctx, seq_ids, noise, t_grid, temperature, u_draft, tokens,
+                        draft_logits=None, stream=None) -> None:
+    """Position i from its own noise block: noise [n_seqs, K, K, V]."""
+    _check(load_library().fm_draft_factorised(ctx, _i32(seq_ids), len(seq_ids), _ptr(noise),
+                                              _f32(t_grid), len(t_grid) - 1, _f32(temperature),
+                                              _ptr(u_draft), _ptr(tokens), _ptr(draft_logits),
+                                              _stream(stream)))
+
+
+def fm_build_tree(draft, B, N, K, node_token, node_parent, node_depth, n_nodes, draft_node,
+                  anc_mask, stream=None) -> None:
+    _check(load_library().fm_build_tree(_ptr(draft), B, N, K, _ptr(node_token), _ptr(node_parent),
+                                        _ptr(node_depth), _ptr(n_nodes), _ptr(draft_node),
+                                        _ptr(anc_mask), _stream(stream)))
+
+
+def fm_tree_attention(q, k_ctx, v_ctx, k_nodes, v_nodes, anc_mask, n_nodes, B, NN, L, n_heads, dh,
+                      out, stream=None) -> None:
+    _check(load_library().fm_tree_attention(_ptr(q), _ptr(k_ctx), _ptr(v_ctx), _ptr(k_nodes),
+                                            _ptr(v_nodes), _ptr(anc_mask), _ptr(n_nodes), B, NN, L,
+                                            n_heads, dh, _ptr(out), _stream(stream)))
+
+
+def fm_verify_greedy_tree(ctx, node_logits, R, draft, draft_node, B, N, K, V, n_acc, branch,
+                          out_tokens, stream=None) -> None:
+    _check(load_library().fm_verify_greedy_tree(ctx, _ptr(node_logits), R, _ptr(draft),
+                                                _ptr(draft_node), B, N, K, V, _ptr(n_acc),
+                                                _ptr(branch), _ptr(out_tokens), _stream(stream)))
+
+
+def fm_verify_sample_tree(ctx, node_logits, R, draft_logits, draft, draft_node, B, N, K, V,
+                          temperature, u_accept, u_res, n_acc, branch, out_tokens,
+                          stream=None) -> None:
+    _check(load_library().fm_verify_sample_tree(ctx, _ptr(node_logits), R, _ptr(draft_logits),
+                                                _ptr(draft), _ptr(draft_node), B, N, K, V,
+                                                float(temperature), _ptr(u_accept), _ptr(u_res),
+                                                _ptr(n_acc), _ptr(branch), _ptr(out_tokens),
+                                                _stream(stream)))
 
 
 def fm_verify_greedy(ctx, target_logits, draft, B, N, K, V, n_acc, branch, out_tokens,

@@ -15,6 +15,7 @@
 #include "fm_tc.cuh"
 #include "fm_attn.cuh"
 #include "fm_dit.cuh"
+#include "fm_tree.cuh"
 
 using fm::bf16;
 
@@ -77,6 +78,10 @@ struct fm_ctx {
   void *h = nullptr, *qkv = nullptr, *o = nullptr, *u = nullptr, *D = nullptr;
   float* part_v = nullptr;
   int* part_i = nullptr;
+  float* smp_max = nullptr;      // chunked sampling: chunk maxima and weight sums per row
+  double* smp_sum = nullptr;
+  int32_t* fac_tok = nullptr;    // factorised drafting: tokens and uniforms of all K drafts
+  double* fac_u = nullptr;
   int n_part = 0;
   float* splitk = nullptr;
   size_t splitk_elems = 0;
@@ -93,14 +98,13 @@ struct fm_ctx {
   float* vg_pv = nullptr;
   int* vg_pi = nullptr;
   unsigned* vg_cnt = nullptr;
+  int* tree_rowmap = nullptr;    // target row of each (sequence, draft, position) of a tree
   unsigned* dit_flags = nullptr; // persistent DiT pass: abort word, completion counters and
   size_t dit_flags_n = 0;        //   flags, LayerNorm tile statistics, final LayerNorm output
   float* dit_stats = nullptr;
   void* dit_hf = nullptr;
   bool dit_ok = false;           // the persistent pass fits this configuration and device
-  // final LayerNorm built by the LM head instead of the persistent pass
-  // (measured: LM head 105 -> 133 us for 7 us saved in the pass; off)
-  bool dit_final_in_lm = false;
+  bool dit_stall_once = false;   // test hook (FM_TEST_STALL=1): the next pass's first wait never ends
   int dit_l2_ahead = 0;          // weight k-blocks the persistent pass prefetches into L2 (measured: no gain)
   float* attn_part = nullptr;   // split-KV attention partials
   unsigned* attn_cnt = nullptr;
@@ -109,6 +113,8 @@ struct fm_ctx {
   float* vs_pm = nullptr;
   double* vs_ps = nullptr;
   double* vs_resid = nullptr;
+  fm::Vs1Plan* vs1_plan = nullptr;   // one-draft stochastic verify: the draw of each sequence
+  double* vs1_csum = nullptr;        //   and its per-chunk weight sums
   bool use_tc = false;
   // LayerNorm inside the consuming GEMM (measured slower than a LayerNorm
   // kernel followed by the GEMM at 16 rows; kept off)
@@ -360,6 +366,10 @@ fm_status load_impl(fm_ctx* c, cudaStream_t st) {
   FM_TRY(dalloc_t(c, &c->logits, M * g.V));
   FM_TRY(dalloc(c, &c->D, M * g.V * sizeof(T)));
   c->n_part = (g.V + 127) / 128;
+  FM_TRY(dalloc_t(c, &c->smp_max, M * fm::SAMPLE_CHUNKS));
+  FM_TRY(dalloc_t(c, &c->smp_sum, M * fm::SAMPLE_CHUNKS));
+  FM_TRY(dalloc_t(c, &c->fac_tok, M));
+  FM_TRY(dalloc_t(c, &c->fac_u, M));
   FM_TRY(dalloc_t(c, &c->part_v, M * c->n_part));
   FM_TRY(dalloc_t(c, &c->part_i, M * c->n_part));
   c->splitk_elems = std::max<size_t>((size_t)1 << 22, 8 * M * (size_t)std::max(3 * d, g.mlp));
@@ -386,10 +396,13 @@ fm_status load_impl(fm_ctx* c, cudaStream_t st) {
   FM_TRY(dalloc_t(c, &c->vg_pv, vrows * c->v_chunks));
   FM_TRY(dalloc_t(c, &c->vg_pi, vrows * c->v_chunks));
   FM_TRY(dalloc_t(c, &c->vg_cnt, (size_t)g.max_seqs));
+  FM_TRY(dalloc_t(c, &c->tree_rowmap, (size_t)g.max_seqs * g.max_noise * (g.K + 1)));
   FM_CUDA(cudaMemsetAsync(c->vg_cnt, 0, g.max_seqs * sizeof(unsigned), st));
   FM_TRY(dalloc_t(c, &c->vs_pm, vrows * c->v_chunks));
   FM_TRY(dalloc_t(c, &c->vs_ps, vrows * c->v_chunks));
   FM_TRY(dalloc_t(c, &c->vs_resid, (size_t)g.max_seqs * 2 * g.V));
+  FM_TRY(dalloc_t(c, &c->vs1_plan, (size_t)g.max_seqs));
+  FM_TRY(dalloc_t(c, &c->vs1_csum, (size_t)g.max_seqs * fm::VS1_CHUNKS * 2));
   FM_TRY(dalloc_t(c, &c->tc.err, 1));
   FM_CUDA(cudaMemsetAsync(c->tc.err, 0, sizeof(int), st));
   if constexpr (sizeof(T) == 2) {
@@ -416,6 +429,10 @@ fm_status load_impl(fm_ctx* c, cudaStream_t st) {
                                                             fm::TC_THREADS, fm::DIT_SMEM));
       c->dit_ok = per_sm >= 1;
     }
+    // test hook: the next persistent pass waits for a count no phase
+    // reaches, so its bounded wait runs out (failure-path test; no fault)
+    const char* stall = getenv("FM_TEST_STALL");
+    c->dit_stall_once = stall && *stall == '1';
     // diagnostic: L2 prefetch depth of the persistent pass (k-blocks, 0 = off)
     const char* ahead = getenv("FM_DIT_L2_AHEAD");
     if (ahead) c->dit_l2_ahead = std::max(0, std::min(256, atoi(ahead)));
@@ -542,7 +559,8 @@ fm_status dit_persistent(fm_ctx* c, const float* mods, int slot, int ctx_len, bo
   P.F = g.mlp;
   P.M = fm::DIT_M;
   P.l2_ahead = c->dit_l2_ahead;
-  P.skip_final = (c->dit_final_in_lm && c->use_tc && c->tc.lm.valid) ? 1 : 0;
+  P.skip_final = 0;
+  P.stall = c->dit_stall_once ? 1 : 0;
   // K splits per GEMM kind: about one unit per SM
   const int tiles[5] = {3 * d / 128, 0, d / 128, g.mlp / 128, d / 128};
   const int kbs[5] = {d / 64, 0, d / 64, d / 64, g.mlp / 64};
@@ -635,8 +653,12 @@ fm_status dit_persistent(fm_ctx* c, const float* mods, int slot, int ctx_len, bo
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  FM_CUDA(cudaLaunchKernelEx(&cfg, fm::k_dit_persistent, P));
+  {
+    Prof prof(c, FM_PROF_DIT_GEMM, st);
+    FM_CUDA(cudaLaunchKernelEx(&cfg, fm::k_dit_persistent, P));
+  }
   c->launches[FM_PROF_DIT_GEMM]++;
+  c->dit_stall_once = false;
   if (P.n_ctx) c->pending_rows = 0;
   return FM_OK;
 }
@@ -731,7 +753,6 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
     bool persistent = false;
     if constexpr (sizeof(T) == 2) {
       if (will_persist) {
-        Prof prof(c, FM_PROF_DIT_GEMM, st);
         fm_status ps = dit_persistent(c, mods, seq_ids[0], c->ctx_len[seq_ids[0]], k == 0, st);
         if (ps == FM_OK) persistent = true;
         else if (ps != FM_ERR_UNSUPPORTED) return ps;
@@ -812,26 +833,7 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
     bool have_partials = false, fused = false;
     if (persistent) {
       fused = true;
-      bool lnf = false;
-      if (c->dit_final_in_lm && c->tc.lm.valid) {   // matches the pass's skip_final
-        // the persistent pass left x un-normalised: the LM head builds its
-        // B operand as LN0(x)(1 + scale_f) + shift_f in shared memory
-        if (need_logits)
-          FM_TRY(gemm_ln(c, FM_PROF_LM_HEAD, c->x, mf, mf + d, M, fm::EpiStoreF32{logits, V}, st,
-                         &c->tc.lm, &lnf, nullptr, 0, true));
-        else
-          FM_TRY(gemm_ln(c, FM_PROF_LM_HEAD, c->x, mf, mf + d, M,
-                         fm::EpiArgmax{c->part_v, c->part_i, c->n_part}, st, &c->tc.lm, &lnf,
-                         nullptr, 0, true));
-        have_partials = lnf && !need_logits;
-        if (!lnf) {
-          Prof prof(c, FM_PROF_NORM, st);
-          FM_LAUNCH(c, FM_PROF_NORM, (fm::k_adaln<float, T>), M, 256, 0, st, c->x, d, mf, mf + d,
-                    (T*)c->dit_hf);
-        }
-      }
-      if (lnf) {
-      } else if (need_logits) {
+      if (need_logits) {
         FM_TRY(gemm_w<T>(c, FM_PROF_LM_HEAD, (const T*)c->dit_hf, d, (const T*)c->w.W_lm, M, V, d,
                          fm::EpiStoreF32{logits, V}, st, &c->tc.lm));
       } else {
@@ -872,9 +874,21 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
       FM_LAUNCH(c, FM_PROF_NORM, (fm::k_softmax_rows<T>), M, 1024, 0, st,
               logits, V, (T*)c->D);
     } else {
+      // greedy rows (and, with few sampled rows, the sampled ones) one CTA
+      // per row; many sampled rows through the chunked sampler
+      const bool chunked = any_sample && !have_partials && M >= 64;
       FM_LAUNCH(c, FM_PROF_NORM, (fm::k_select_tokens), M, 1024, 0, st,
               have_partials ? nullptr : logits, V, have_partials ? c->part_v : nullptr,
-                    have_partials ? c->part_i : nullptr, c->n_part, u_draft, ta, tokens);
+                    have_partials ? c->part_i : nullptr, c->n_part, u_draft, ta, tokens,
+                    chunked ? 1 : 0);
+      if (chunked) {
+        FM_LAUNCH(c, FM_PROF_NORM, fm::k_sample_chunk_max, M * fm::SAMPLE_CHUNKS, 256, 0, st,
+                  (const float*)logits, V, ta, c->smp_max);
+        FM_LAUNCH(c, FM_PROF_NORM, fm::k_sample_chunk_sum, M * fm::SAMPLE_CHUNKS, 256, 0, st,
+                  (const float*)logits, V, ta, (const float*)c->smp_max, c->smp_sum);
+        FM_LAUNCH(c, FM_PROF_NORM, fm::k_sample_pick, M, 512, 0, st, (const float*)logits, V,
+                  u_draft, ta, (const float*)c->smp_max, (const double*)c->smp_sum, tokens);
+      }
     }
   }
   return FM_OK;
@@ -973,10 +987,10 @@ extern "C" fm_status fm_project_context(fm_ctx* c, const int32_t* seq_ids, int n
                             : project_impl<float>(c, seq_ids, n_seqs, hidden, n_new, pos0, st);
 }
 
-extern "C" fm_status fm_draft(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* noise,
-                              int n_noise, const float* t_grid, int num_steps,
-                              const float* temperature, const double* u_draft, int32_t* tokens,
-                              float* draft_logits, fm_stream stream) {
+static fm_status check_draft(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* noise,
+                             int n_noise, const float* t_grid, int num_steps,
+                             const float* temperature, const double* u_draft,
+                             const int32_t* tokens) {
   if (!c || !seq_ids || !noise || !t_grid || !temperature || !tokens)
     return set_err(FM_ERR_ARG, "NULL argument");
   const fm_config& g = c->cfg;
@@ -997,12 +1011,52 @@ extern "C" fm_status fm_draft(fm_ctx* c, const int32_t* seq_ids, int n_seqs, con
     if (temperature[q] > 0.f && !u_draft)
       return set_err(FM_ERR_ARG, "u_draft is NULL but sequence %d samples", q);
   }
+  return FM_OK;
+}
+
+extern "C" fm_status fm_draft(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* noise,
+                              int n_noise, const float* t_grid, int num_steps,
+                              const float* temperature, const double* u_draft, int32_t* tokens,
+                              float* draft_logits, fm_stream stream) {
+  FM_TRY(check_draft(c, seq_ids, n_seqs, noise, n_noise, t_grid, num_steps, temperature, u_draft,
+                     tokens));
+  const fm_config& g = c->cfg;
   cudaStream_t st = (cudaStream_t)stream;
   return g.dtype == FM_BF16
              ? draft_impl<bf16>(c, seq_ids, n_seqs, noise, n_noise, t_grid, num_steps, temperature,
                                 u_draft, tokens, draft_logits, st)
              : draft_impl<float>(c, seq_ids, n_seqs, noise, n_noise, t_grid, num_steps,
                                  temperature, u_draft, tokens, draft_logits, st);
+}
+
+extern "C" fm_status fm_draft_factorised(fm_ctx* c, const int32_t* seq_ids, int n_seqs,
+                                         const void* noise, const float* t_grid, int num_steps,
+                                         const float* temperature, const double* u_draft,
+                                         int32_t* tokens, float* draft_logits, fm_stream stream) {
+  if (!c) return set_err(FM_ERR_ARG, "NULL argument");
+  const fm_config& g = c->cfg;
+  const int K = g.K, V = g.V;
+  FM_TRY(check_draft(c, seq_ids, n_seqs, noise, 1, t_grid, num_steps, temperature, u_draft, tokens));
+  if (g.max_noise < K)
+    return set_err(FM_ERR_UNSUPPORTED, "factorised drafting needs max_noise >= K = %d", K);
+  bool any_sample = false;
+  for (int q = 0; q < n_seqs; ++q) any_sample |= temperature[q] > 0.f;
+  cudaStream_t st = (cudaStream_t)stream;
+  // position i of every draft uses the uniform of position i; only draft i's
+  // position i is kept
+  if (any_sample)
+    FM_LAUNCH(c, FM_PROF_NORM, fm::k_repeat_u, grid_1d((size_t)n_seqs * K * K, 256), 256, 0, st,
+              u_draft, c->fac_u, n_seqs, K);
+  float* all_logits = draft_logits ? c->logits : nullptr;
+  fm_status s = g.dtype == FM_BF16
+                    ? draft_impl<bf16>(c, seq_ids, n_seqs, noise, K, t_grid, num_steps, temperature,
+                                       any_sample ? c->fac_u : nullptr, c->fac_tok, all_logits, st)
+                    : draft_impl<float>(c, seq_ids, n_seqs, noise, K, t_grid, num_steps, temperature,
+                                        any_sample ? c->fac_u : nullptr, c->fac_tok, all_logits, st);
+  FM_TRY(s);
+  FM_LAUNCH(c, FM_PROF_NORM, fm::k_take_diagonal, n_seqs * K, 256, 0, st, (const int*)c->fac_tok,
+            (const float*)all_logits, n_seqs, K, V, tokens, draft_logits);
+  return FM_OK;
 }
 
 static fm_status check_verify(fm_ctx* c, const void* tgt, const void* draft, int B, int N, int K,
@@ -1022,18 +1076,57 @@ static int verify_chunks(fm_ctx* c, long rows, int V) {
   return std::max(ch, 1);
 }
 
-extern "C" fm_status fm_verify_greedy(fm_ctx* c, const float* target_logits, const int32_t* draft,
-                                      int B, int N, int K, int V, int32_t* n_acc,
-                                      int32_t* branch, int32_t* out_tokens, fm_stream stream) {
-  FM_TRY(check_verify(c, target_logits, draft, B, N, K, V, n_acc, branch, out_tokens));
-  cudaStream_t st = (cudaStream_t)stream;
+static fm_status verify_greedy_impl(fm_ctx* c, const float* target_logits, const int32_t* draft,
+                                    int B, int N, int K, int V, int32_t* n_acc, int32_t* branch,
+                                    int32_t* out_tokens, const int* rowmap, cudaStream_t st) {
   const long rows = (long)B * N * (K + 1);
   const int ch = verify_chunks(c, rows, V);
   Prof prof(c, FM_PROF_VERIFY, st);
   FM_LAUNCH(c, FM_PROF_VERIFY, (fm::k_verify_greedy), (unsigned)(rows * ch), fm::VG_THREADS, 0, st,
-              target_logits, draft, B, N, K, V, ch, c->vg_pv, c->vg_pi, c->vg_cnt, n_acc, branch,
-      out_tokens);
+            target_logits, draft, B, N, K, V, ch, c->vg_pv, c->vg_pi, c->vg_cnt, n_acc, branch,
+            out_tokens, rowmap);
   return FM_OK;
+}
+
+static fm_status verify_sample_impl(fm_ctx* c, const float* target_logits,
+                                    const float* draft_logits, const int32_t* draft, int B, int N,
+                                    int K, int V, float temperature, const double* u_accept,
+                                    const double* u_res, int32_t* n_acc, int32_t* branch,
+                                    int32_t* out_tokens, const int* rowmap, cudaStream_t st) {
+  if (!(temperature > 0.f)) return set_err(FM_ERR_ARG, "temperature must be > 0");
+  if (!u_accept || !u_res) return set_err(FM_ERR_ARG, "uniforms are NULL");
+  const int n_tgt = B * N * (K + 1);
+  const int n_rows = n_tgt + (draft_logits ? B * N * K : 0);
+  const int ch = verify_chunks(c, n_rows, V);
+  Prof prof(c, FM_PROF_VERIFY, st);
+  FM_LAUNCH(c, FM_PROF_VERIFY, (fm::k_row_stats), (unsigned)((long)n_rows * ch), fm::VS_THREADS, 0, st,
+            target_logits, draft_logits, n_tgt, n_rows, V, ch, temperature, c->vs_pm, c->vs_ps,
+            rowmap);
+  if (N == 1) {
+    // one draft: a warp per sequence walks the depths, then the one draw is
+    // summed and searched over many CTAs per sequence
+    FM_LAUNCH(c, FM_PROF_VERIFY, fm::k_vs1_walk, (B + 3) / 4, 128, 0, st, target_logits, draft_logits,
+              draft, B, K, V, temperature, u_accept, c->vs_pm, c->vs_ps, ch, c->vs1_plan, n_acc,
+              branch, out_tokens, rowmap);
+    FM_LAUNCH(c, FM_PROF_VERIFY, fm::k_vs1_sums, B * fm::VS1_CHUNKS, 256, 0, st, target_logits,
+              draft_logits, V, temperature, (const fm::Vs1Plan*)c->vs1_plan, c->vs1_csum, rowmap);
+    FM_LAUNCH(c, FM_PROF_VERIFY, fm::k_vs1_pick, B, 512, 0, st, target_logits, draft_logits, K, V,
+              temperature, u_res, (const fm::Vs1Plan*)c->vs1_plan, (const double*)c->vs1_csum,
+              out_tokens, rowmap);
+    return FM_OK;
+  }
+  FM_LAUNCH(c, FM_PROF_VERIFY, (fm::k_verify_sample_decide), B, fm::VS_DECIDE_THREADS, 0, st,
+            target_logits, draft_logits, draft, B, N, K, V, temperature, u_accept, u_res, c->vs_pm,
+            c->vs_ps, ch, c->vs_resid, n_acc, branch, out_tokens, rowmap);
+  return FM_OK;
+}
+
+extern "C" fm_status fm_verify_greedy(fm_ctx* c, const float* target_logits, const int32_t* draft,
+                                      int B, int N, int K, int V, int32_t* n_acc,
+                                      int32_t* branch, int32_t* out_tokens, fm_stream stream) {
+  FM_TRY(check_verify(c, target_logits, draft, B, N, K, V, n_acc, branch, out_tokens));
+  return verify_greedy_impl(c, target_logits, draft, B, N, K, V, n_acc, branch, out_tokens, nullptr,
+                            (cudaStream_t)stream);
 }
 
 extern "C" fm_status fm_verify_sample(fm_ctx* c, const float* target_logits,
@@ -1042,19 +1135,88 @@ extern "C" fm_status fm_verify_sample(fm_ctx* c, const float* target_logits,
                                       const double* u_res, int32_t* n_acc, int32_t* branch,
                                       int32_t* out_tokens, fm_stream stream) {
   FM_TRY(check_verify(c, target_logits, draft, B, N, K, V, n_acc, branch, out_tokens));
-  if (!(temperature > 0.f)) return set_err(FM_ERR_ARG, "temperature must be > 0");
-  if (!u_accept || !u_res) return set_err(FM_ERR_ARG, "uniforms are NULL");
-  cudaStream_t st = (cudaStream_t)stream;
-  const int n_tgt = B * N * (K + 1);
-  const int n_rows = n_tgt + (draft_logits ? B * N * K : 0);
-  const int ch = verify_chunks(c, n_rows, V);
-  Prof prof(c, FM_PROF_VERIFY, st);
-  FM_LAUNCH(c, FM_PROF_VERIFY, (fm::k_row_stats), (unsigned)((long)n_rows * ch), fm::VS_THREADS, 0, st,
-              target_logits, draft_logits, n_tgt, n_rows, V, ch, temperature, c->vs_pm, c->vs_ps);
-  FM_LAUNCH(c, FM_PROF_VERIFY, (fm::k_verify_sample_decide), B, fm::VS_DECIDE_THREADS, 0, st,
-              target_logits, draft_logits, draft, B, N, K, V, temperature, u_accept, u_res, c->vs_pm,
-      c->vs_ps, ch, c->vs_resid, n_acc, branch, out_tokens);
+  return verify_sample_impl(c, target_logits, draft_logits, draft, B, N, K, V, temperature, u_accept,
+                            u_res, n_acc, branch, out_tokens, nullptr, (cudaStream_t)stream);
+}
+
+// ------------------------------------------------------------------ tree of noise drafts
+static fm_status check_tree_sizes(int B, int N, int K) {
+  if (B < 1 || N < 1 || K < 1) return set_err(FM_ERR_ARG, "sizes must be positive");
+  // each factor bounded before the product
+  if (N > fm::TREE_MAX_DRAFTS || K > fm::TREE_MAX_NODES || N * K > fm::TREE_MAX_NODES)
+    return set_err(FM_ERR_UNSUPPORTED, "a tree holds at most %d drafts and %d nodes",
+                   fm::TREE_MAX_DRAFTS, fm::TREE_MAX_NODES);
   return FM_OK;
+}
+
+extern "C" fm_status fm_build_tree(const int32_t* draft, int B, int N, int K, int32_t* node_token,
+                                   int32_t* node_parent, int32_t* node_depth, int32_t* n_nodes,
+                                   int32_t* draft_node, uint64_t* anc_mask, fm_stream stream) {
+  if (!draft || !node_token || !node_parent || !node_depth || !n_nodes || !draft_node || !anc_mask)
+    return set_err(FM_ERR_ARG, "NULL argument");
+  FM_TRY(check_tree_sizes(B, N, K));
+  const int NN = N * K, W = (NN + 63) / 64;
+  cudaError_t e = fm::launch_pdl(fm::k_build_tree, dim3(B), dim3(32), 0, (cudaStream_t)stream,
+                                 (const int*)draft, N, K, NN, W, (int*)node_token,
+                                 (int*)node_parent, (int*)node_depth, (int*)n_nodes,
+                                 (int*)draft_node, anc_mask);
+  if (e != cudaSuccess) return set_err(FM_ERR_CUDA, "tree build launch failed: %s", cudaGetErrorString(e));
+  return FM_OK;
+}
+
+extern "C" fm_status fm_tree_attention(const float* q, const float* k_ctx, const float* v_ctx,
+                                       const float* k_nodes, const float* v_nodes,
+                                       const uint64_t* anc_mask, const int32_t* n_nodes, int B,
+                                       int NN, int L, int n_heads, int dh, float* out,
+                                       fm_stream stream) {
+  if (!q || !k_nodes || !v_nodes || !anc_mask || !n_nodes || !out || (L > 0 && (!k_ctx || !v_ctx)))
+    return set_err(FM_ERR_ARG, "NULL argument");
+  if (B < 1 || NN < 1 || L < 0 || n_heads < 1 || dh < 1)
+    return set_err(FM_ERR_ARG, "sizes must be positive");
+  if (NN > fm::TREE_MAX_NODES || dh > 128 || n_heads > 1024)
+    return set_err(FM_ERR_UNSUPPORTED, "at most %d nodes, head width 128", fm::TREE_MAX_NODES);
+  const long warps = (long)B * NN * n_heads;
+  if (warps > (1L << 31)) return set_err(FM_ERR_UNSUPPORTED, "too many (node, head) pairs");
+  const int W = (NN + 63) / 64;
+  cudaError_t e = fm::launch_pdl(fm::k_tree_attention, dim3((unsigned)((warps + 3) / 4)), dim3(128), 0,
+                                 (cudaStream_t)stream, q, k_ctx, v_ctx, k_nodes, v_nodes, anc_mask,
+                                 (const int*)n_nodes, B, NN, L, n_heads, dh, W,
+                                 (float)(1.0 / sqrt((double)dh)), out);
+  if (e != cudaSuccess) return set_err(FM_ERR_CUDA, "tree attention launch failed: %s", cudaGetErrorString(e));
+  return FM_OK;
+}
+
+static fm_status tree_rowmap(fm_ctx* c, const int32_t* draft_node, int B, int N, int K, int R,
+                             cudaStream_t st) {
+  if (!draft_node) return set_err(FM_ERR_ARG, "NULL argument");
+  if (R < 1 + N * K) return set_err(FM_ERR_ARG, "R=%d rows per sequence < 1 + N*K", R);
+  FM_LAUNCH(c, FM_PROF_VERIFY, fm::k_tree_rowmap, grid_1d((size_t)B * N * (K + 1), 256), 256, 0, st,
+            (const int*)draft_node, B, N, K, R, c->tree_rowmap);
+  return FM_OK;
+}
+
+extern "C" fm_status fm_verify_greedy_tree(fm_ctx* c, const float* node_logits, int R,
+                                           const int32_t* draft, const int32_t* draft_node, int B,
+                                           int N, int K, int V, int32_t* n_acc, int32_t* branch,
+                                           int32_t* out_tokens, fm_stream stream) {
+  FM_TRY(check_verify(c, node_logits, draft, B, N, K, V, n_acc, branch, out_tokens));
+  cudaStream_t st = (cudaStream_t)stream;
+  FM_TRY(tree_rowmap(c, draft_node, B, N, K, R, st));
+  return verify_greedy_impl(c, node_logits, draft, B, N, K, V, n_acc, branch, out_tokens,
+                            c->tree_rowmap, st);
+}
+
+extern "C" fm_status fm_verify_sample_tree(fm_ctx* c, const float* node_logits, int R,
+                                           const float* draft_logits, const int32_t* draft,
+                                           const int32_t* draft_node, int B, int N, int K, int V,
+                                           float temperature, const double* u_accept,
+                                           const double* u_res, int32_t* n_acc, int32_t* branch,
+                                           int32_t* out_tokens, fm_stream stream) {
+  FM_TRY(check_verify(c, node_logits, draft, B, N, K, V, n_acc, branch, out_tokens));
+  cudaStream_t st = (cudaStream_t)stream;
+  FM_TRY(tree_rowmap(c, draft_node, B, N, K, R, st));
+  return verify_sample_impl(c, node_logits, draft_logits, draft, B, N, K, V, temperature, u_accept,
+                            u_res, n_acc, branch, out_tokens, c->tree_rowmap, st);
 }
 
 extern "C" fm_status fm_profile(fm_ctx* c, int mask) {
@@ -1101,7 +1263,14 @@ extern "C" fm_status fm_device_status(fm_ctx* c, fm_stream stream) {
   FM_CUDA(cudaMemcpyAsync(&v, c->tc.err, sizeof(int), cudaMemcpyDeviceToHost, st));
   FM_CUDA(cudaStreamSynchronize(st));
   if (v) {
+    // a kernel that gave up may have left arrival counters mid-count: they
+    // return to zero here, so the context's next call starts clean (the
+    // persistent pass's handoff words need no reset: their flags name the
+    // launch that wrote them)
     FM_CUDA(cudaMemsetAsync(c->tc.err, 0, sizeof(int), st));
+    FM_CUDA(cudaMemsetAsync(c->tile_cnt, 0, c->tile_cnt_n * sizeof(unsigned), st));
+    FM_CUDA(cudaMemsetAsync(c->attn_cnt, 0, c->attn_pairs_max * sizeof(unsigned), st));
+    FM_CUDA(cudaMemsetAsync(c->vg_cnt, 0, c->cfg.max_seqs * sizeof(unsigned), st));
     FM_CUDA(cudaStreamSynchronize(st));
     return set_err(FM_ERR_TIMEOUT, "a bounded wait inside a tensor-core kernel gave up (code %d)", v);
   }
@@ -1193,7 +1362,8 @@ extern "C" fm_status fm_verify_greedy_noalloc(const float* target_logits, const 
   FM_CUDA(cudaMemsetAsync(s->cnt, 0, (size_t)B * sizeof(unsigned), st));
   cudaError_t e = fm::launch_pdl(fm::k_verify_greedy, dim3((unsigned)(rows * ch)),
                                  dim3(fm::VG_THREADS), 0, st, target_logits, draft, B, N, K, V, ch,
-                                 s->pv, s->pi, s->cnt, n_acc, branch, out_tokens);
+                                 s->pv, s->pi, s->cnt, n_acc, branch, out_tokens,
+                                 (const int*)nullptr);
   if (e != cudaSuccess)
     return set_err(FM_ERR_CUDA, "greedy verify launch failed: %s", cudaGetErrorString(e));
   return FM_OK;

@@ -54,6 +54,7 @@ struct DitParams {
   int splits[5];                      // per GEMM kind (index by DIT_*; [1] = attention splits)
   int l2_ahead;                       // weight k-blocks prefetched into L2 beyond the ring
   int skip_final;                     // the LM head applies the final LayerNorm itself
+  int stall;                          // test hook: the first QKV wait targets a count never reached
   float* x;                           // residual stream [M][d] fp32
   float* stats;                       // [d/128 tiles][M][2]: tile mean, tile sum of squared deviations
   float* partial;                     // split-K partials, one region per GEMM kind
@@ -207,7 +208,9 @@ __device__ bool dit_wait_deps_warp(const DitParams& P, int kind, int l, int cta,
   if (kind == -2) {
     if (lane == 0) ok = dit_wait(P, P.c_down + P.n_blocks - 1, tiles_d);
   } else if (kind == DIT_QKV) {
-    if (lane == 0) ok = dit_wait(P, l == 0 ? P.c_stats : P.c_down + l - 1, tiles_d);
+    if (lane == 0)
+      ok = dit_wait(P, l == 0 ? P.c_stats : P.c_down + l - 1,
+                    tiles_d + ((P.stall && l == 0) ? 1u : 0u));
   } else if (kind == DIT_UP) {
     if (lane == 0) ok = dit_wait(P, P.c_o + l, tiles_d);
   } else if (kind == DIT_ATTN) {

@@ -215,7 +215,7 @@ struct TempArgs {
 __global__ void __launch_bounds__(1024)
 k_select_tokens(const float* __restrict__ logits, int V, const float* __restrict__ part_v,
                 const int* __restrict__ part_i, int n_part, const double* __restrict__ u,
-                TempArgs ta, int* __restrict__ tokens) {
+                TempArgs ta, int* __restrict__ tokens, int skip_sampled) {
   pdl_wait();
   pdl_trigger();
   __shared__ float shv[32];
@@ -223,6 +223,7 @@ k_select_tokens(const float* __restrict__ logits, int V, const float* __restrict
   const int m = blockIdx.x;
   const int q = m / (ta.n_noise * ta.K);
   const float T = ta.temp[q];
+  if (T > 0.f && skip_sampled) return;   // drawn by the chunked sampler below
   if (T == 0.f) {
     ArgMax a{-INFINITY, 0x7fffffff};
     if (part_v) {
@@ -249,6 +250,130 @@ k_select_tokens(const float* __restrict__ logits, int V, const float* __restrict
   auto wf = [&](int v) { return (double)expf((row[v] - mx) * iT); };
   int tok = block_sample(wf, V, u[m]);
   if (threadIdx.x == 0) tokens[m] = tok;
+}
+
+// ------------------------------------------------------------------ chunked sampling
+// Sampled rows (T > 0) of a batch, spread over SAMPLE_CHUNKS vocabulary
+// chunks per row: the chunk maxima, then per chunk the sum of the row's fp32
+// weights exp((l - max) / T) in fp64, then one CTA per row finds the chunk
+// holding u * total (chunk sums in fixed order) and draws inside it by the
+// inverse CDF -- the same weights and rule as one CTA per row, with every
+// pass over the logits spread over the whole GPU.  Greedy rows return at
+// once.
+constexpr int SAMPLE_CHUNKS = 16;
+
+__global__ void __launch_bounds__(256)
+k_sample_chunk_max(const float* __restrict__ logits, int V, TempArgs ta, float* __restrict__ cmax) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ float sh[32];
+  const int m = blockIdx.x / SAMPLE_CHUNKS, c = blockIdx.x - m * SAMPLE_CHUNKS;
+  if (ta.temp[m / (ta.n_noise * ta.K)] == 0.f) return;
+  const int per = (V + SAMPLE_CHUNKS - 1) / SAMPLE_CHUNKS;
+  const int v0 = min(V, c * per), v1 = min(V, v0 + per);
+  const float* row = logits + (size_t)m * V;
+  float mx = -INFINITY;
+  for (int v = v0 + (int)threadIdx.x; v < v1; v += blockDim.x) mx = fmaxf(mx, row[v]);
+  mx = block_max(mx, sh);
+  if (threadIdx.x == 0) cmax[(size_t)m * SAMPLE_CHUNKS + c] = mx;
+}
+
+__global__ void __launch_bounds__(256)
+k_sample_chunk_sum(const float* __restrict__ logits, int V, TempArgs ta,
+                   const float* __restrict__ cmax, double* __restrict__ csum) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ double sh[32];
+  const int m = blockIdx.x / SAMPLE_CHUNKS, c = blockIdx.x - m * SAMPLE_CHUNKS;
+  const float T = ta.temp[m / (ta.n_noise * ta.K)];
+  if (T == 0.f) return;
+  float mx = -INFINITY;
+  for (int k = 0; k < SAMPLE_CHUNKS; ++k) mx = fmaxf(mx, cmax[(size_t)m * SAMPLE_CHUNKS + k]);
+  const int per = (V + SAMPLE_CHUNKS - 1) / SAMPLE_CHUNKS;
+  const int v0 = min(V, c * per), v1 = min(V, v0 + per);
+  const float* row = logits + (size_t)m * V;
+  const float iT = 1.f / T;
+  double s = 0.0;
+  for (int v = v0 + (int)threadIdx.x; v < v1; v += blockDim.x) s += (double)expf((row[v] - mx) * iT);
+  s = block_sum_d(s, sh);
+  if (threadIdx.x == 0) csum[(size_t)m * SAMPLE_CHUNKS + c] = s;
+}
+
+__global__ void __launch_bounds__(512)
+k_sample_pick(const float* __restrict__ logits, int V, const double* __restrict__ u, TempArgs ta,
+              const float* __restrict__ cmax, const double* __restrict__ csum,
+              int* __restrict__ tokens) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ int s_c;
+  __shared__ double s_u;
+  const int m = blockIdx.x;
+  const float T = ta.temp[m / (ta.n_noise * ta.K)];
+  if (T == 0.f) return;
+  const double* cs = csum + (size_t)m * SAMPLE_CHUNKS;
+  float mx = -INFINITY;
+  for (int k = 0; k < SAMPLE_CHUNKS; ++k) mx = fmaxf(mx, cmax[(size_t)m * SAMPLE_CHUNKS + k]);
+  if (threadIdx.x == 0) {
+    double tot = 0.0;
+    for (int k = 0; k < SAMPLE_CHUNKS; ++k) tot += cs[k];
+    const double target = u[m] * tot;
+    double pre = 0.0;
+    int own = -1, last_pos = 0;
+    for (int k = 0; k < SAMPLE_CHUNKS; ++k) {
+      if (cs[k] > 0.0) last_pos = k;
+      if (own < 0 && pre + cs[k] > target) own = k;
+      else if (own < 0) pre += cs[k];
+    }
+    if (own < 0) {                        // rounding: the last chunk with mass
+      own = last_pos;
+      pre = 0.0;
+      for (int k = 0; k < own; ++k) pre += cs[k];
+    }
+    s_c = own;
+    s_u = cs[own] > 0.0 ? fmin(fmax((target - pre) / cs[own], 0.0), 1.0) : 0.0;
+  }
+  __syncthreads();
+  const int per = (V + SAMPLE_CHUNKS - 1) / SAMPLE_CHUNKS;
+  const int v0 = min(V, s_c * per), v1 = min(V, v0 + per);
+  const float* row = logits + (size_t)m * V;
+  const float iT = 1.f / T;
+  auto wf = [&](int v) { return (double)expf((row[v0 + v] - mx) * iT); };
+  const int tok = v0 + block_sample(wf, v1 - v0, s_u);
+  if (threadIdx.x == 0) tokens[m] = tok;
+}
+
+// ------------------------------------------------------------------ factorised drafting
+// u_full[b][j][i] = u[b][i]: every draft j of sequence b samples position i
+// with that position's uniform.
+__global__ void k_repeat_u(const double* __restrict__ u, double* __restrict__ u_full, int n_seqs,
+                           int K) {
+  pdl_wait();
+  pdl_trigger();
+  const size_t n = (size_t)n_seqs * K * K;
+  for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n;
+       e += (size_t)gridDim.x * blockDim.x) {
+    const size_t b = e / ((size_t)K * K);
+    const int i = (int)(e % K);
+    u_full[e] = u[b * K + i];
+  }
+}
+
+// tokens[b][i] = all_tok[b][i][i] and, when both are given, logits[b][i][:]
+// = all_logits[b][i][i][:]: position i of the factorised block comes from
+// the draft of noise block i.  One CTA per (b, i).
+__global__ void k_take_diagonal(const int* __restrict__ all_tok, const float* __restrict__ all_logits,
+                                int n_seqs, int K, int V, int* __restrict__ tokens,
+                                float* __restrict__ logits) {
+  pdl_wait();
+  pdl_trigger();
+  const int bi = blockIdx.x, b = bi / K, i = bi - b * K;
+  const size_t src = ((size_t)b * K + i) * K + i;
+  if (threadIdx.x == 0) tokens[bi] = all_tok[src];
+  if (all_logits && logits) {
+    const float* r = all_logits + src * V;
+    float* o = logits + (size_t)bi * V;
+    for (int v = threadIdx.x; v < V; v += blockDim.x) o[v] = r[v];
+  }
 }
 
 // ------------------------------------------------------------------ transpose

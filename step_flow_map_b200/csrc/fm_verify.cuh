@@ -23,7 +23,8 @@ __global__ void __launch_bounds__(VG_THREADS)
 k_verify_greedy(const float* __restrict__ tgt, const int* __restrict__ draft, int B, int N,
                 int K, int V, int chunks, float* __restrict__ pv, int* __restrict__ pi,
                 unsigned* __restrict__ counter, int* __restrict__ n_acc,
-                int* __restrict__ branch, int* __restrict__ out) {
+                int* __restrict__ branch, int* __restrict__ out,
+                const int* __restrict__ rowmap) {
   pdl_wait();
   pdl_trigger();
   __shared__ float shv[32];
@@ -36,7 +37,8 @@ k_verify_greedy(const float* __restrict__ tgt, const int* __restrict__ draft, in
   const int b = row / rows_b;
   const int per = (V + chunks - 1) / chunks;
   const int v0 = min(V, c * per), v1 = min(V, v0 + per);
-  const float* r = tgt + (size_t)row * V;
+  // a tree's rows come through its row map (shared prefixes share a row)
+  const float* r = tgt + (size_t)(rowmap ? rowmap[row] : row) * V;
   ArgMax a{-INFINITY, 0x7fffffff};
   // eight strided loads in flight per thread before they are compared (the
   // comparison is order-independent: ties go to the lowest index)
@@ -110,32 +112,51 @@ k_verify_greedy(const float* __restrict__ tgt, const int* __restrict__ draft, in
 
 // ------------------------------------------------------------------ stochastic
 // Pass 1: per (row, chunk) the chunk max m_c and S_c = sum exp((l - m_c)/T)
-// in fp64, for every target row and, when present, every draft row.
+// in fp64, for every target row and, when present, every draft row.  One
+// read of the chunk: each thread keeps a running max and a sum relative to
+// it (rescaled by exp((m_old - m_new)/T) when the max grows, which after
+// the first few elements is rare), then the block takes the largest max
+// and rescales every thread's sum to it.
 constexpr int VS_THREADS = 256;
 
 __global__ void __launch_bounds__(VS_THREADS)
 k_row_stats(const float* __restrict__ tgt, const float* __restrict__ dlog, int n_tgt_rows,
             int n_rows, int V, int chunks, float T, float* __restrict__ pm,
-            double* __restrict__ ps) {
+            double* __restrict__ ps, const int* __restrict__ rowmap) {
   pdl_wait();
   pdl_trigger();
   __shared__ float shf[32];
   __shared__ double shd[32];
   const int row = blockIdx.x / chunks, c = blockIdx.x - row * chunks;
-  const float* r = (row < n_tgt_rows) ? tgt + (size_t)row * V
+  const float* r = (row < n_tgt_rows) ? tgt + (size_t)(rowmap ? rowmap[row] : row) * V
                                       : dlog + (size_t)(row - n_tgt_rows) * V;
   const int per = (V + chunks - 1) / chunks;
   const int v0 = min(V, c * per), v1 = min(V, v0 + per);
+  const double iT = 1.0 / (double)T;
   float mx = -INFINITY;
-  for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x) mx = fmaxf(mx, r[v]);
-  mx = block_max(mx, shf);
   double s = 0.0;
-  const double dm = (double)mx, iT = 1.0 / (double)T;
-  for (int v = v0 + threadIdx.x; v < v1; v += blockDim.x) s += exp(((double)r[v] - dm) * iT);
-  s = block_sum_d(s, shd);
+  for (int base = v0 + (int)threadIdx.x; base < v1; base += 4 * (int)blockDim.x) {
+    float x[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int v = base + u * (int)blockDim.x;
+      x[u] = v < v1 ? __ldcs(r + v) : -INFINITY;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (x[u] > mx) {
+        s = (mx == -INFINITY) ? 0.0 : s * exp(((double)mx - (double)x[u]) * iT);
+        mx = x[u];
+      }
+      if (x[u] > -INFINITY) s += exp(((double)x[u] - (double)mx) * iT);
+    }
+  }
+  const float M = block_max(mx, shf);
+  double sc = (mx == -INFINITY) ? 0.0 : s * exp(((double)mx - (double)M) * iT);
+  sc = block_sum_d(sc, shd);
   if (threadIdx.x == 0) {
-    pm[(size_t)row * chunks + c] = mx;
-    ps[(size_t)row * chunks + c] = s;
+    pm[(size_t)row * chunks + c] = M;
+    ps[(size_t)row * chunks + c] = sc;
   }
 }
 
@@ -172,7 +193,8 @@ k_verify_sample_decide(const float* __restrict__ tgt, const float* __restrict__ 
                        const double* __restrict__ ua, const double* __restrict__ ures,
                        const float* __restrict__ pm, const double* __restrict__ ps, int chunks,
                        double* __restrict__ resid, int* __restrict__ n_acc,
-                       int* __restrict__ branch, int* __restrict__ out) {
+                       int* __restrict__ branch, int* __restrict__ out,
+                       const int* __restrict__ rowmap) {
   pdl_wait();
   pdl_trigger();
   __shared__ double shd[32];
@@ -189,7 +211,7 @@ k_verify_sample_decide(const float* __restrict__ tgt, const float* __restrict__ 
   for (int i = 0; i < K; ++i) {
     r0 = __ffs(alive) - 1;
     const int trow = (b * N + r0) * (K + 1) + i;
-    const float* tp = tgt + (size_t)trow * V;
+    const float* tp = tgt + (size_t)(rowmap ? rowmap[trow] : trow) * V;
     if (tid < 32) {
       RowStat st = warp_combine_stats(pm, ps, trow, chunks, dT, tid);
       if (tid == 0) { s_mp = st.m; s_Sp = st.S; s_mode = 0; s_buf = 0; s_accept = -1; }
@@ -269,7 +291,7 @@ k_verify_sample_decide(const float* __restrict__ tgt, const float* __restrict__ 
   if (n_done == K) {
     r0 = __ffs(alive) - 1;
     const int trow = (b * N + r0) * (K + 1) + K;
-    const float* tp = tgt + (size_t)trow * V;
+    const float* tp = tgt + (size_t)(rowmap ? rowmap[trow] : trow) * V;
     if (tid < 32) {
       RowStat st = warp_combine_stats(pm, ps, trow, chunks, dT, tid);
       if (tid == 0) { s_mp = st.m; s_Sp = st.S; }
@@ -287,6 +309,202 @@ k_verify_sample_decide(const float* __restrict__ tgt, const float* __restrict__ 
     n_acc[b] = n_done;
     branch[b] = r0;
   }
+}
+
+// ------------------------------------------------------------------ stochastic, one draft
+// With one draft per sequence the walk needs no materialised residual: the
+// first rejected depth fixes what is sampled -- normalise(max(0, p - q)) at
+// that depth, or p of row K when every depth is accepted -- so the walk is
+// one warp per sequence, and the weights of that one draw are summed and
+// searched by many CTAs per sequence (VS1_CHUNKS vocabulary chunks each)
+// instead of one.
+constexpr int VS1_CHUNKS = 16;
+
+// Per sequence: 0 depth of the draw (n accepted), 1 rejected token (-1 when
+// every depth accepted), 2 target row, 3 draft row (-1 without draft
+// logits); and fp64 (m_p, S_p, m_q, S_q).
+struct Vs1Plan {
+  int n, y, trow, drow;
+  double mp, Sp, mq, Sq;
+};
+
+// One warp per sequence: accept while u q(y) < p(y) (fp64), write the
+// accepted tokens, the counts and the -1 padding, and the draw's plan.
+__global__ void __launch_bounds__(128)
+k_vs1_walk(const float* __restrict__ tgt, const float* __restrict__ dlog,
+           const int* __restrict__ draft, int B, int K, int V, float T,
+           const double* __restrict__ ua, const float* __restrict__ pm,
+           const double* __restrict__ ps, int chunks, Vs1Plan* __restrict__ plan,
+           int* __restrict__ n_acc, int* __restrict__ branch, int* __restrict__ out,
+           const int* __restrict__ rowmap) {
+  pdl_wait();
+  pdl_trigger();
+  const int b = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (b >= B) return;
+  const double dT = (double)T;
+  const int n_tgt_rows = B * (K + 1);
+  int* o = out + (size_t)b * (K + 1);
+  int i = 0;
+  RowStat sp{0.0, 1.0}, sq{0.0, 1.0};
+  int y = -1;
+  for (; i < K; ++i) {
+    const int trow = b * (K + 1) + i, drow = b * K + i;
+    sp = warp_combine_stats(pm, ps, trow, chunks, dT, lane);
+    if (dlog) sq = warp_combine_stats(pm, ps, n_tgt_rows + drow, chunks, dT, lane);
+    y = draft[(size_t)b * K + i];
+    int acc = 0;
+    if (lane == 0) {
+      const float* tp = tgt + (size_t)(rowmap ? rowmap[trow] : trow) * V;
+      const double py = exp(((double)tp[y] - sp.m) / dT) / sp.S;
+      const double qy = dlog ? exp(((double)dlog[(size_t)drow * V + y] - sq.m) / dT) / sq.S : 1.0;
+      acc = (ua[(size_t)b * K + i] * qy < py) ? 1 : 0;
+      if (acc) o[i] = y;
+    }
+    acc = __shfl_sync(0xffffffffu, acc, 0);
+    if (!acc) break;
+  }
+  if (lane == 0) {
+    Vs1Plan pl;
+    pl.n = i;
+    if (i < K) {
+      pl.y = y;
+      pl.trow = b * (K + 1) + i;
+      pl.drow = dlog ? b * K + i : -1;
+      pl.mp = sp.m; pl.Sp = sp.S; pl.mq = sq.m; pl.Sq = sq.S;
+    } else {
+      const int trow = b * (K + 1) + K;
+      pl.y = -1;
+      pl.trow = trow;
+      pl.drow = -1;
+      pl.mp = pl.Sp = pl.mq = pl.Sq = 0.0;
+    }
+    plan[b] = pl;
+    for (int k = i + 1; k <= K; ++k) o[k] = -1;
+    n_acc[b] = i;
+    branch[b] = 0;
+  }
+  if (i == K) {
+    // the bonus row's statistics
+    RowStat st = warp_combine_stats(pm, ps, b * (K + 1) + K, chunks, dT, lane);
+    if (lane == 0) { plan[b].mp = st.m; plan[b].Sp = st.S; }
+  }
+}
+
+// Weight of token v in a draw: max(0, p - q) for a rejected depth (q the
+// draft distribution, or the point mass on the rejected token), p itself
+// for the bonus row; `use_p` forces p (a residual whose mass rounded to 0
+// leaves p unchanged).
+struct Vs1Weight {
+  const float* tp;
+  const float* qp;
+  double mp, iSp, mq, iSq, iT;
+  int y;
+  bool resid;
+  __device__ __forceinline__ double p(int v) const { return exp(((double)tp[v] - mp) * iT) * iSp; }
+  __device__ __forceinline__ double operator()(int v) const {
+    const double pv = p(v);
+    if (!resid) return pv;
+    const double qv = qp ? exp(((double)qp[v] - mq) * iT) * iSq : (v == y ? 1.0 : 0.0);
+    return fmax(pv - qv, 0.0);
+  }
+};
+
+__device__ __forceinline__ Vs1Weight vs1_weight(const Vs1Plan& pl, const float* tgt,
+                                                const float* dlog, int V, float T,
+                                                const int* rowmap) {
+  Vs1Weight w;
+  w.tp = tgt + (size_t)(rowmap ? rowmap[pl.trow] : pl.trow) * V;
+  w.qp = pl.drow >= 0 ? dlog + (size_t)pl.drow * V : nullptr;
+  w.mp = pl.mp;
+  w.iSp = 1.0 / pl.Sp;
+  w.mq = pl.mq;
+  w.iSq = pl.drow >= 0 ? 1.0 / pl.Sq : 0.0;
+  w.iT = 1.0 / (double)T;
+  w.y = pl.y;
+  w.resid = pl.y >= 0;
+  return w;
+}
+
+// (sum of the draw's weights, sum of p) over chunk c of sequence b.
+__global__ void __launch_bounds__(256)
+k_vs1_sums(const float* __restrict__ tgt, const float* __restrict__ dlog, int V, float T,
+           const Vs1Plan* __restrict__ plan, double* __restrict__ csum,
+           const int* __restrict__ rowmap) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ double shd[32];
+  const int b = blockIdx.x / VS1_CHUNKS, c = blockIdx.x - b * VS1_CHUNKS;
+  const Vs1Plan pl = plan[b];
+  const Vs1Weight w = vs1_weight(pl, tgt, dlog, V, T, rowmap);
+  const int per = (V + VS1_CHUNKS - 1) / VS1_CHUNKS;
+  const int v0 = min(V, c * per), v1 = min(V, v0 + per);
+  double sw = 0.0, sp = 0.0;
+  for (int v = v0 + (int)threadIdx.x; v < v1; v += blockDim.x) {
+    const double pv = w.p(v);
+    sp += pv;
+    if (w.resid) {
+      const double qv = w.qp ? exp(((double)w.qp[v] - w.mq) * w.iT) * w.iSq : (v == w.y ? 1.0 : 0.0);
+      sw += fmax(pv - qv, 0.0);
+    }
+  }
+  sw = block_sum_d(sw, shd);
+  sp = block_sum_d(sp, shd);
+  if (threadIdx.x == 0) {
+    csum[((size_t)b * VS1_CHUNKS + c) * 2] = w.resid ? sw : sp;
+    csum[((size_t)b * VS1_CHUNKS + c) * 2 + 1] = sp;
+  }
+}
+
+// One CTA per sequence: the chunk holding u * total (chunk sums in fixed
+// order), then the token inside it by inverse CDF; writes the drawn token.
+__global__ void __launch_bounds__(512)
+k_vs1_pick(const float* __restrict__ tgt, const float* __restrict__ dlog, int K, int V, float T,
+           const double* __restrict__ ures, const Vs1Plan* __restrict__ plan,
+           const double* __restrict__ csum, int* __restrict__ out,
+           const int* __restrict__ rowmap) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ int s_c;
+  __shared__ double s_u;
+  const int b = blockIdx.x;
+  const Vs1Plan pl = plan[b];
+  Vs1Weight w = vs1_weight(pl, tgt, dlog, V, T, rowmap);
+  const double* cs = csum + (size_t)b * VS1_CHUNKS * 2;
+  if (threadIdx.x == 0) {
+    double tot = 0.0;
+    for (int c = 0; c < VS1_CHUNKS; ++c) tot += cs[c * 2];
+    int col = 0;                           // the sums to use: the draw's weights, or p
+    if (w.resid && !(tot > 0.0)) {
+      col = 1;
+      tot = 0.0;
+      for (int c = 0; c < VS1_CHUNKS; ++c) tot += cs[c * 2 + 1];
+    }
+    const double target = ures[b] * tot;
+    double pre = 0.0;
+    int own = -1, last_pos = 0;
+    for (int c = 0; c < VS1_CHUNKS; ++c) {
+      const double sc = cs[c * 2 + col];
+      if (sc > 0.0) last_pos = c;
+      if (own < 0 && pre + sc > target) own = c;
+      else if (own < 0) pre += sc;
+    }
+    if (own < 0) {                        // rounding: the last chunk with mass
+      own = last_pos;
+      pre = 0.0;
+      for (int c = 0; c < own; ++c) pre += cs[c * 2 + col];
+    }
+    const double sc = cs[own * 2 + col];
+    s_c = own | (col << 16);
+    s_u = sc > 0.0 ? fmin(fmax((target - pre) / sc, 0.0), 1.0) : 0.0;
+  }
+  __syncthreads();
+  const int own = s_c & 0xffff;
+  if (s_c >> 16) w.resid = false;
+  const int per = (V + VS1_CHUNKS - 1) / VS1_CHUNKS;
+  const int v0 = min(V, own * per), v1 = min(V, v0 + per);
+  auto wf = [&](int v) { return w(v0 + v); };
+  const int tok = v0 + block_sample(wf, v1 - v0, s_u);
+  if (threadIdx.x == 0) out[(size_t)b * (K + 1) + pl.n] = tok;
 }
 
 }  // namespace fm

@@ -9,8 +9,8 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (FM_BF16, FM_F32, fm_draft, fm_free, fm_load_weights, fm_project_context,
-               fm_verify_greedy, fm_verify_sample)
+from . import (FM_BF16, FM_F32, fm_draft, fm_draft_factorised, fm_free, fm_load_weights,
+               fm_project_context, fm_verify_greedy, fm_verify_sample)
 
 TORCH_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16}
 FM_DTYPE = {"f32": FM_F32, "bf16": FM_BF16}
@@ -67,6 +67,17 @@ class Context:
                       if logits else None)
         fm_draft(self.ctx, seq_ids, noise, n_noise, t_grid, temps, u_draft, tokens, out_logits,
                  stream)
+        return tokens, out_logits
+
+    def draft_factorised(self, seq_ids, noise: torch.Tensor, t_grid, temps, u_draft=None,
+                         logits=True, stream=None):
+        """noise [n_seqs, K, K, V]: position i of each block from noise block i."""
+        n_seqs, K, _, V = noise.shape
+        tokens = torch.empty((n_seqs, K), dtype=torch.int32, device=noise.device)
+        out_logits = (torch.empty((n_seqs, K, V), dtype=torch.float32, device=noise.device)
+                      if logits else None)
+        fm_draft_factorised(self.ctx, seq_ids, noise, t_grid, temps, u_draft, tokens, out_logits,
+                            stream)
         return tokens, out_logits
 
     def verify_greedy(self, target: torch.Tensor, draft: torch.Tensor, stream=None):

@@ -132,20 +132,23 @@ def test_nan_logit_never_wins():
     W64 = {k: v.astype(np.float64) for k, v in W.items()}
     rows = np.concatenate([fs.prefill_hidden(w, 0), fs.round_inputs(w, 0).new_hidden[0]], axis=0)
     _, kv = om.project_context(W64, w.shape.n_blocks, rows)
-    ri = fs.round_inputs(w, 0)
-    ref = om.draft(W64, w.shape, kv, ri.noise[0], w.t_grid)
-    assert (ref["tokens"] != vstar).all()
-    clean = np.where(np.isnan(ref["logits"]), -np.inf, ref["logits"])
-    sure = om.margins(clean) > gu.MARGIN
-    assert sure.sum() >= 4
+    refs = [om.draft(W64, w.shape, kv, fs.round_inputs(w, r).noise[0], w.t_grid) for r in range(4)]
+    checked = 0
     for logits in (False, True):
         ctx = Context(w.shape, w.dtype, W, max_ctx=w.ctx + 40, max_seqs=1, max_noise=1, max_new=64)
         gu.gpu_prefill(ctx, w, [0], max_new=64)
         gu.gpu_new_rows(ctx, w, 0, [0])
-        tok, _ = ctx.draft([0], to_device(ri.noise, "bf16"), w.t_grid, w.temps, logits=logits)
-        torch.cuda.synchronize()
-        fm_device_status(ctx.ctx)
-        got = gu.to_np(tok)[0]
-        assert (got != vstar).all(), logits
-        np.testing.assert_array_equal(got[sure], ref["tokens"][sure])
+        for r, ref in enumerate(refs):
+            ri = fs.round_inputs(w, r)
+            assert (ref["tokens"] != vstar).all()
+            tok, _ = ctx.draft([0], to_device(ri.noise, "bf16"), w.t_grid, w.temps, logits=logits)
+            torch.cuda.synchronize()
+            fm_device_status(ctx.ctx)
+            got = gu.to_np(tok)[0]
+            assert (got != vstar).all(), (logits, r)
+            clean = np.where(np.isnan(ref["logits"]), -np.inf, ref["logits"])
+            sure = om.margins(clean) > gu.MARGIN
+            np.testing.assert_array_equal(got[sure], ref["tokens"][sure])
+            checked += int(sure.sum())
         ctx.close()
+    assert checked >= 4

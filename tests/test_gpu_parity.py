@@ -351,3 +351,34 @@ def test_argument_errors():
             f()
         assert e.value.status == FM_ERR_ARG
     ctx.close()
+
+
+# ------------------------------------------------------------------ factorised drafting
+@pytest.mark.parametrize("name,T", [("tiny_f32", 0.0), ("tiny_f32", 0.8)])
+def test_factorised_draft_matches_per_position_oracle(name, T):
+    # position i from its own noise block: the oracle drafts each block and
+    # keeps its position i
+    w = dataclasses.replace(fs.WORKLOADS[name], temps=(T,))
+    K = w.shape.K
+    ctx = gu.make_ctx(dataclasses.replace(w, n_noise=K))
+    gu.gpu_prefill(ctx, w, [0])
+    kv = gu.oracle_kv(w, 0, None)
+    W = gu.weights64(w.shape, w.dtype)
+    for r in range(2):
+        X = fs.factorised_noise(w, r)
+        u = fs.uniform(6000 + r, (1, K))
+        tok, lg = ctx.draft_factorised([0], to_device(X, w.dtype), w.t_grid, w.temps,
+                                       u_draft=to_device(u) if T > 0 else None)
+        tok, lg = gu.to_np(tok)[0], gu.to_np(lg)[0]
+        ref = om.draft(W, w.shape, kv, X[0], w.t_grid)
+        want_logits = np.stack([ref["logits"][i, i] for i in range(K)])
+        gu.assert_logits_close(lg, want_logits, w.dtype, f"round {r}")
+        for i in range(K):
+            if T == 0:
+                if om.margins(want_logits[i]) > gu.MARGIN:
+                    assert tok[i] == om.argmax_lowest(want_logits[i]), (r, i)
+            else:
+                y, sure = gu.sampled_token_sure(want_logits[i], T, u[0, i])
+                if sure:
+                    assert tok[i] == y, (r, i)
+    ctx.close()

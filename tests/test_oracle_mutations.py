@@ -128,3 +128,30 @@ def test_temperature_mutation_is_caught(name, monkeypatch):
 def test_argmax_mutation_is_caught(name, monkeypatch):
     _patch_all(_mutated(ARGMAX_MUTATIONS[name]), monkeypatch)
     assert _fails(TA.test_nan_never_wins)
+
+
+# ---- the prefix trie of the noise drafts ----
+from oracle import tree as ot              # noqa: E402
+import test_oracle_tree as TR              # noqa: E402
+
+TREE_SRC = inspect.getsource(ot)
+TREE_MUTATIONS = {
+    "node key without its parent": (
+        "key = (draft_node[j][i - 1] if i > 0 else -1, drafts[j][i])", "key = (-1, drafts[j][i])"),
+    "a node is not its own ancestor": ("        u = v\n", "        u = parent[v]\n"),
+    "node rows off by one": ("out[j, i] = node_rows[1 + draft_node[j][i - 1]]",
+                             "out[j, i] = node_rows[draft_node[j][i - 1]]"),
+}
+
+
+@pytest.mark.parametrize("name", list(TREE_MUTATIONS))
+def test_tree_mutation_is_caught(name, monkeypatch):
+    a, b = TREE_MUTATIONS[name]
+    assert a in TREE_SRC
+    ns = {}
+    exec(compile(TREE_SRC.replace(a, b), "<mutant>", "exec"), ns)
+    for f in ("build_trie", "ancestors", "tree_attention", "draft_rows"):
+        monkeypatch.setattr(ot, f, ns[f])
+    checks = [TR.test_hand_built_trie, lambda: TR.test_trie_matches_brute_force_prefixes(3),
+              TR.test_tree_attention_equals_causal_attention_on_each_path]
+    assert any(_fails(c) for c in checks)
