@@ -628,19 +628,28 @@ fm_status dit_persistent(fm_ctx* c, const float* mods, int slot, int ctx_len, bo
   am.cnt = c->attn_cnt;
   am.slot[0] = slot;
   am.len[0] = ctx_len;
-  int s_ctx = G / g.n_heads - 1;
-  s_ctx = std::min(s_ctx, (ctx_len + fm::AM_CHUNK - 1) / fm::AM_CHUNK);
-  s_ctx = std::max(s_ctx, 1);
+  // context rows this pass appends (keys/values written by its QKV phases)
+  P.attn_safe = ctx_len;
+  for (int q = 0; q < (P.n_ctx ? P.ctx_map.n_seqs : 0); ++q)
+    if (P.ctx_map.slot[q] == slot) P.attn_safe = std::min(P.attn_safe, P.ctx_map.pos0[q]);
+  // context splits of whole 64-row chunks below the appended rows, at least
+  // a full ring (two chunks) each, so a split's first chunks load before its
+  // queries exist; the rows from the last whole chunk on (appended rows
+  // included) ride with the block's own rows
+  const int s_max = G / g.n_heads - 1;
+  if (s_max < 1) return FM_ERR_UNSUPPORTED;
+  const int base = P.attn_safe / fm::AM_CHUNK * fm::AM_CHUNK;
+  const int per = (base + s_max * fm::AM_CHUNK - 1) / (s_max * fm::AM_CHUNK) * fm::AM_CHUNK;
+  am.split_rows = std::max(fm::DIT_ATTN_ST * fm::AM_CHUNK, per);
+  am.tail0 = base;
+  int s_ctx = std::max(1, (base + am.split_rows - 1) / am.split_rows);
+  if (ctx_len - base + 16 > fm::DIT_ATTN_ST * fm::AM_CHUNK) return FM_ERR_UNSUPPORTED;
   if (g.n_heads * (s_ctx + 1) > G) return FM_ERR_UNSUPPORTED;
   if ((size_t)g.n_heads * (s_ctx + 1) * 16 * fm::AM_PSTRIDE > c->attn_part_elems)
     return FM_ERR_UNSUPPORTED;
   // a head's split partials are merged in shared memory
   if ((size_t)(s_ctx + 1) * 16 * fm::AM_PSTRIDE * 4 > (size_t)fm::DIT_UNION) return FM_ERR_UNSUPPORTED;
   am.n_ctx_splits = s_ctx;
-  // context rows this pass appends (keys/values written by its QKV phases)
-  P.attn_safe = ctx_len;
-  for (int q = 0; q < (P.n_ctx ? P.ctx_map.n_seqs : 0); ++q)
-    if (P.ctx_map.slot[q] == slot) P.attn_safe = std::min(P.attn_safe, P.ctx_map.pos0[q]);
   P.splits[fm::DIT_ATTN] = s_ctx;
   FM_CUDA(cudaMemsetAsync(c->dit_flags, 0, c->dit_flags_n * sizeof(unsigned), st));
   cudaLaunchConfig_t cfg = {};
@@ -694,6 +703,8 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
   fm::AttnMmaArgs am;
   int max_len = 0;
   if (use_mma_attn) {
+    am.split_rows = 0;
+    am.tail0 = 0;
     am.n_seqs = n_seqs;
     am.n_noise = n_noise;
     am.K = K;
@@ -1265,8 +1276,7 @@ extern "C" fm_status fm_device_status(fm_ctx* c, fm_stream stream) {
   if (v) {
     // a kernel that gave up may have left arrival counters mid-count: they
     // return to zero here, so the context's next call starts clean (the
-    // persistent pass's handoff words need no reset: their flags name the
-    // launch that wrote them)
+    // persistent pass's completion counters are zeroed before each launch)
     FM_CUDA(cudaMemsetAsync(c->tc.err, 0, sizeof(int), st));
     FM_CUDA(cudaMemsetAsync(c->tile_cnt, 0, c->tile_cnt_n * sizeof(unsigned), st));
     FM_CUDA(cudaMemsetAsync(c->attn_cnt, 0, c->attn_pairs_max * sizeof(unsigned), st));

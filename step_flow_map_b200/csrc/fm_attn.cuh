@@ -30,6 +30,11 @@ constexpr int AM_PSTRIDE = AM_DH + 4;  // floats per partial row: O[128], m, l, 
 
 struct AttnMmaArgs {
   int n_seqs, n_noise, K, d, n_heads, max_ctx, n_ctx_splits;
+  // split_rows == 0: the context splits divide [0, len) evenly.  split_rows
+  // > 0 (one sequence, one noise draft): split s covers rows
+  // [s split_rows, (s + 1) split_rows) of [0, tail0), and the block-row item
+  // also takes the context rows [tail0, len) (at most 112 of them)
+  int split_rows, tail0;
   float scale_log2;    // log2(e) / sqrt(dh)
   float* part;         // [pairs][n_ctx_splits + 1][N*16][AM_PSTRIDE]
   unsigned* cnt;       // [pairs], zero between launches
@@ -174,17 +179,23 @@ struct AttnRange {
 __device__ __forceinline__ AttnRange attn_range(const AttnMmaArgs& a, int b, int h, int split) {
   AttnRange r;
   const int L = a.len[b];
-  r.k0 = (int)((long)split * L / a.n_ctx_splits);
-  r.k1 = (int)((long)(split + 1) * L / a.n_ctx_splits);
+  if (a.split_rows > 0) {
+    r.k0 = min(split * a.split_rows, a.tail0);
+    r.k1 = min(r.k0 + a.split_rows, a.tail0);
+  } else {
+    r.k0 = (int)((long)split * L / a.n_ctx_splits);
+    r.k1 = (int)((long)(split + 1) * L / a.n_ctx_splits);
+  }
   r.n_chunks = (r.k1 - r.k0 + AM_CHUNK - 1) / AM_CHUNK;
   r.base = (size_t)a.slot[b] * a.max_ctx * a.d + h * AM_DH;
   return r;
 }
 
-// Issue the first ST - 1 context chunks of a split (one cp.async commit group
-// each, empty past the end) into the K/V ring.  A caller may run this before
-// the queries exist, when those rows are not written by the same pass.
-template <int N, int ST>
+// Issue the first NPRE (ST - 1, or the whole ring: ST) context chunks of a
+// split (one cp.async commit group each, empty past the end) into the K/V
+// ring.  A caller may run this before the queries exist, when those rows are
+// not written by the same pass.
+template <int N, int ST, int NPRE = ST - 1>
 __device__ __forceinline__ void attn_ctx_prologue(const bf16* __restrict__ Kc,
                                                   const bf16* __restrict__ Vc,
                                                   const AttnMmaArgs& a, int pair, int split,
@@ -194,7 +205,7 @@ __device__ __forceinline__ void attn_ctx_prologue(const bf16* __restrict__ Kc,
   const int b = pair / a.n_heads, h = pair - b * a.n_heads;
   const AttnRange rg = attn_range(a, b, h, split);
 #pragma unroll
-  for (int c = 0; c < ST - 1; ++c) {
+  for (int c = 0; c < NPRE; ++c) {
     if (c < rg.n_chunks) {
       const int r0 = rg.k0 + c * AM_CHUNK, nr = min(AM_CHUNK, rg.k1 - r0);
       load_rows(sK + c * AM_CHUNK * AM_LD, Kc + rg.base + (size_t)r0 * a.d, a.d, nr, AM_CHUNK, tid);
@@ -220,7 +231,10 @@ struct AttnBulkMerge {
 // One work item -- (sequence, head) pair `pair`, split `split` -- run by
 // AM_THREADS threads (tid 0..AM_THREADS-1, four whole warps) that
 // synchronise with `sync()`.  ST context chunks are in flight; `smem_raw`
-// holds attn_mma_smem<N, ST>() bytes; `s_last` is one shared int.
+// holds attn_mma_smem<N, ST>() bytes; `s_last` is one shared int.  BULK
+// (the persistent pass): the prologue fills the whole ring (ST chunks, so a
+// split of at most ST chunks needs no load after its queries exist) and the
+// split partials are merged through one bulk copy.
 template <int N, int ST, bool BULK, class Sync>
 __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf16* __restrict__ Kc,
                                           const bf16* __restrict__ Vc, bf16* __restrict__ out,
@@ -268,7 +282,8 @@ __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf
     };
     // one commit group per chunk (empty past the end) keeps the group count
     // fixed: ST - 1 chunks are always in flight ahead of the one used
-    if (!prologue_done) attn_ctx_prologue<N, ST>(Kc, Vc, a, pair, split, smem_raw, tid);
+    constexpr int NPRE = BULK ? ST : ST - 1;
+    if (!prologue_done) attn_ctx_prologue<N, ST, NPRE>(Kc, Vc, a, pair, split, smem_raw, tid);
     // queries of all drafts of the sequence (the newest group)
     load_rows(sQ, qkv + (size_t)row0 * d3 + h * AM_DH, d3, NQ, NQ, tid);
     cp_commit();
@@ -276,8 +291,12 @@ __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf
     sync();
     q_fragments();
     for (int c = 0; c < n_chunks; ++c) {
-      if (c + ST - 1 < n_chunks) load_chunk(c + ST - 1);
-      cp_commit();
+      if constexpr (!BULK) {
+        if (c + ST - 1 < n_chunks) load_chunk(c + ST - 1);
+        cp_commit();
+      }
+      // one commit group per iteration: chunk c's group is older than the
+      // ST - 1 most recent ones
       cp_wait<ST - 1>();
       sync();
       const int buf = c % ST;
@@ -289,7 +308,33 @@ __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf
       const bf16* vs = sV + buf * AM_CHUNK * AM_LD + kw0 * AM_LD;
       if (nk > 0) attn_block<KW / 8>(st, qa, ks, vs, nk, a.scale_log2);
       sync();
+      if constexpr (BULK) {
+        // the whole ring was prefetched: chunk c + ST goes into the buffer
+        // just read
+        if (c + ST < n_chunks) load_chunk(c + ST);
+        cp_commit();
+      }
     }
+  } else if (a.split_rows > 0) {
+    // one sequence, one noise draft: the context rows [tail0, len) and the
+    // block's own 16 rows, as one key range [tail rows; own rows] spread
+    // over the four warps
+    static_assert(N == 1 || BULK == false, "tail rows need one noise draft");
+    const int L = a.len[b], nt = L - a.tail0, nkey = nt + 16;
+    const size_t base = (size_t)a.slot[b] * a.max_ctx * a.d + h * AM_DH;
+    load_rows(sQ, qkv + (size_t)row0 * d3 + h * AM_DH, d3, NQ, NQ, tid);
+    load_rows(sK, Kc + base + (size_t)a.tail0 * a.d, a.d, nt, nt, tid);
+    load_rows(sV, Vc + base + (size_t)a.tail0 * a.d, a.d, nt, nt, tid);
+    const int pad = (nkey + 31) / 32 * 32;
+    load_rows(sK + nt * AM_LD, qkv + (size_t)row0 * d3 + a.d + h * AM_DH, d3, 16, pad - nt, tid);
+    load_rows(sV + nt * AM_LD, qkv + (size_t)row0 * d3 + 2 * a.d + h * AM_DH, d3, 16, pad - nt, tid);
+    cp_commit();
+    cp_wait<0>();
+    sync();
+    q_fragments();
+    const int kw0 = warp * 32, nk = max(0, min(32, nkey - kw0));
+    if (nk > 0) attn_block<4>(st, qa, sK + kw0 * AM_LD, sV + kw0 * AM_LD, nk, a.scale_log2);
+    sync();
   } else {
     load_rows(sQ, qkv + (size_t)row0 * d3 + h * AM_DH, d3, NQ, NQ, tid);
     // each draft's own block rows: keys/values of rows row0 + mt*16 .. +16
@@ -313,7 +358,9 @@ __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf
     sync();
   }
 
-  // ---- merge the warps of each query tile in smem, write this split's partial
+  // ---- merge the warps of each query tile: per-row (max, sum) of every warp
+  // through shared memory; each warp rescales its own O in registers; the
+  // partial is the sum of the rescaled warp tiles
   float l_tot[2];
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
@@ -321,41 +368,61 @@ __device__ __forceinline__ void attn_item(const bf16* __restrict__ qkv, const bf
     l_tot[r] += __shfl_xor_sync(0xffffffffu, l_tot[r], 1);
     l_tot[r] += __shfl_xor_sync(0xffffffffu, l_tot[r], 2);
   }
-  float* sO = (float*)sK;                           // [4 warps][16][AM_DH + 2] fp32 (reuse)
+  constexpr int OLD = AM_DH + 4;                    // row stride of a warp's O tile (16-byte rows)
+  float* sML = (float*)sK;                          // [4 warps][16][2]: row max, row sum
+  float* sO = sML + 4 * 16 * 2;                     // [4 warps][16][OLD] rescaled O
   const int g = lane >> 2, t = lane & 3;
-  float* wo = sO + warp * 16 * (AM_DH + 2);
+  if (t == 0) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      sML[(warp * 16 + g + 8 * r) * 2] = st.m[r];
+      sML[(warp * 16 + g + 8 * r) * 2 + 1] = l_tot[r];
+    }
+  }
+  sync();
+  float Mrow[2], Lrow[2], f[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int row = g + 8 * r;
+    float M = -INFINITY;
+#pragma unroll
+    for (int s2 = 0; s2 < WPM; ++s2) M = fmaxf(M, sML[((s2 * N + mt) * 16 + row) * 2]);
+    float L = 0.f;
+#pragma unroll
+    for (int s2 = 0; s2 < WPM; ++s2) {
+      const float mm = sML[((s2 * N + mt) * 16 + row) * 2];
+      if (mm != -INFINITY) L += exp2f(mm - M) * sML[((s2 * N + mt) * 16 + row) * 2 + 1];
+    }
+    f[r] = (st.m[r] == -INFINITY) ? 0.f : exp2f(st.m[r] - M);
+    Mrow[r] = M;
+    Lrow[r] = L;
+  }
+  float* wo = sO + warp * 16 * OLD;
 #pragma unroll
   for (int n = 0; n < 16; ++n) {
     const int c = n * 8 + 2 * t;
-    wo[g * (AM_DH + 2) + c] = st.o[n][0];
-    wo[g * (AM_DH + 2) + c + 1] = st.o[n][1];
-    wo[(g + 8) * (AM_DH + 2) + c] = st.o[n][2];
-    wo[(g + 8) * (AM_DH + 2) + c + 1] = st.o[n][3];
-  }
-  if (t == 0) {
-    wo[g * (AM_DH + 2) + AM_DH] = st.m[0];
-    wo[g * (AM_DH + 2) + AM_DH + 1] = l_tot[0];
-    wo[(g + 8) * (AM_DH + 2) + AM_DH] = st.m[1];
-    wo[(g + 8) * (AM_DH + 2) + AM_DH + 1] = l_tot[1];
+    *(float2*)(wo + g * OLD + c) = make_float2(st.o[n][0] * f[0], st.o[n][1] * f[0]);
+    *(float2*)(wo + (g + 8) * OLD + c) = make_float2(st.o[n][2] * f[1], st.o[n][3] * f[1]);
   }
   sync();
   float* part = a.part + ((size_t)pair * S_all + split) * NQ * AM_PSTRIDE;
-  for (int e = tid; e < NQ * AM_DH; e += AM_THREADS) {
-    const int q = e / AM_DH, c = e % AM_DH;
+  for (int e = tid; e < NQ * (AM_DH / 4); e += AM_THREADS) {
+    const int q = e / (AM_DH / 4), c4 = (e % (AM_DH / 4)) * 4;
     const int tile = q / 16, rr = q % 16;
-    float M = -INFINITY;
-    for (int s2 = 0; s2 < WPM; ++s2) M = fmaxf(M, sO[((s2 * N + tile) * 16 + rr) * (AM_DH + 2) + AM_DH]);
-    float o = 0.f, l = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
     for (int s2 = 0; s2 < WPM; ++s2) {
-      const float* w = sO + ((s2 * N + tile) * 16 + rr) * (AM_DH + 2);
-      const float f = (w[AM_DH] == -INFINITY) ? 0.f : exp2f(w[AM_DH] - M);
-      o += f * w[c];
-      l += f * w[AM_DH + 1];
+      const float4 v = *(const float4*)(sO + ((s2 * N + tile) * 16 + rr) * OLD + c4);
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
     }
-    part[q * AM_PSTRIDE + c] = o;
-    if (c == 0) {
-      part[q * AM_PSTRIDE + AM_DH] = M;
-      part[q * AM_PSTRIDE + AM_DH + 1] = l;
+    *(float4*)(part + (size_t)q * AM_PSTRIDE + c4) = acc;
+  }
+  if (sub == 0 && t == 0) {
+    // one warp per query tile writes its rows' (max, sum)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int q = mt * 16 + g + 8 * r;
+      *(float2*)(part + (size_t)q * AM_PSTRIDE + AM_DH) = make_float2(Mrow[r], Lrow[r]);
     }
   }
   sync();

@@ -86,7 +86,7 @@ struct DitParams {
 };
 
 struct DitShared {                    // after the ring and the union region
-  uint64_t full[DIT_RING], empty[DIT_RING], tfull[2], tempty[2], bready, rbar;
+  uint64_t full[DIT_RING], empty[DIT_RING], tfull[2], tempty[2], bready[2], rbar;
   uint32_t tmem;
   int abort, last, ok[2], attn_last;
   float stat[2 * DIT_BROWS_MAX];      // mean, rstd per row
@@ -309,14 +309,15 @@ __device__ __forceinline__ void dit_row_stats(const DitParams& P, int et, DitSha
 // of x, QKV rows M .. M+n_ctx-1 are copied context rows; kind O/DOWN: rows
 // < M are copied from o / u.  Other rows are zero.
 // Shift and scale of a LayerNorm phase for this CTA's columns [c0, c0 + ncol)
-// into shared memory, all loads in flight at once.  The adaLN modulation is
-// fixed for the whole pass, so this runs before the phase's grid barrier.
-__device__ __forceinline__ void dit_stage_mods(const DitParams& P, int kind, int l, int c0,
-                                               int ncol, int et, DitShared* sh) {
+// into shared memory, all loads in flight at once (loaded by
+// dit_mods_load, stored by dit_mods_store, so other loads can be issued in
+// between).  The adaLN modulation is fixed for the whole pass, so this runs
+// before the phase's wait.
+__device__ __forceinline__ void dit_mods_load(const DitParams& P, int kind, int l, int c0,
+                                              int ncol, int et, float (&hv)[8], float (&cv)[8]) {
   const float* ml = P.mods + (size_t)l * 6 * P.d;
   const float* shift = kind == DIT_QKV ? ml : ml + 3 * P.d;
   const float* scale = kind == DIT_QKV ? ml + P.d : ml + 4 * P.d;
-  float hv[8], cv[8];
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
     const int c = et + 128 * u;
@@ -326,6 +327,10 @@ __device__ __forceinline__ void dit_stage_mods(const DitParams& P, int kind, int
       cv[u] = __ldg(scale + c0 + c);
     }
   }
+}
+
+__device__ __forceinline__ void dit_mods_store(int ncol, int et, const float (&hv)[8],
+                                               const float (&cv)[8], DitShared* sh) {
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
     const int c = et + 128 * u;
@@ -342,37 +347,52 @@ __device__ __forceinline__ void dit_stage_mods(const DitParams& P, int kind, int
 __device__ __forceinline__ void dit_fill_extra(const DitParams& P, uint8_t* sB, int kb0, int nkb,
                                                int brows, int Kd, int et) {
   const int tile_bytes = brows * 128;
-  const int M = P.M, xrows = brows - M;
-  const int items_x = nkb * xrows * 8;
-  for (int i0 = 0; i0 < items_x; i0 += 128 * 8) {
-    uint4 cp[8];
+  const int M = P.M, nr = P.n_ctx;                 // nr >= 1
+  // the context rows, sixteen loads per thread in flight per batch (one
+  // batch up to 16 rows x 16 k-blocks)
+  const int items = nkb * nr * 8;
+  for (int i0 = 0; i0 < items; i0 += 128 * 16) {
+    uint4 cp[16];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 16; ++u) {
       const int idx = i0 + u * 128 + et;
-      const int kbi = idx / (xrows * 8), rem = idx - kbi * (xrows * 8);
+      const int kbi = idx / (nr * 8), rem = idx - kbi * (nr * 8);
       const int r = rem >> 3, col = (kb0 + kbi) * TC_BK + (rem & 7) * 8;
       cp[u] = make_uint4(0, 0, 0, 0);
-      if (idx < items_x && r < P.n_ctx && col < Kd)
-        cp[u] = __ldcg((const uint4*)(P.ctx_rows + (size_t)r * P.d + col));
+      if (idx < items && col < Kd) cp[u] = __ldcg((const uint4*)(P.ctx_rows + (size_t)r * P.d + col));
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 16; ++u) {
       const int idx = i0 + u * 128 + et;
-      if (idx >= items_x) break;
-      const int kbi = idx / (xrows * 8), rem = idx - kbi * (xrows * 8);
+      if (idx >= items) break;
+      const int kbi = idx / (nr * 8), rem = idx - kbi * (nr * 8);
       const int row = M + (rem >> 3), ch = rem & 7;
       *(uint4*)(sB + kbi * tile_bytes + row * 128 + ((ch ^ (row & 7)) << 4)) = cp[u];
     }
   }
+  // rows past the context rows up to the tile height: zeros
+  const int pr = brows - M - nr;
+  const int zitems = nkb * pr * 8;
+  for (int idx = et; idx < zitems; idx += 128) {
+    const int kbi = idx / (pr * 8), rem = idx - kbi * (pr * 8);
+    const int row = M + nr + (rem >> 3), ch = rem & 7;
+    *(uint4*)(sB + kbi * tile_bytes + row * 128 + ((ch ^ (row & 7)) << 4)) = make_uint4(0, 0, 0, 0);
+  }
 }
 
 // B operand rows 0 .. M-1 (M = 16: 128 items per k-block, so each batch of
-// 1024 items is 8 k-blocks).  Every batch is published on `bready` (all 128
+// 1024 items is 8 k-blocks).  Batch i is published on bready[i] (all 128
 // threads arrive) as soon as it is stored, so the MMAs of its k-blocks, and
-// the ring refills they free, overlap the rest of the fill.
+// the ring refills they free, overlap the rest of the fill.  One barrier per
+// batch: each completes at most once per GEMM phase, and the MMA warp
+// observes that completion before the epilogue can reach the next phase's
+// fill (the epilogue first waits for this phase's accumulator), so a waiter
+// polling by parity never misses a phase.  (With one barrier for both
+// batches, two completions in quick succession could pass between two polls
+// and leave the MMA warp waiting on the wrong phase.)
 __device__ __forceinline__ void dit_fill_b(const DitParams& P, int kind, uint8_t* sB, int kb0,
                                            int nkb, int brows, int Kd, int et, DitShared* sh,
-                                           uint32_t bready) {
+                                           const uint64_t* bready) {
   // one loop per kind of row, so each unrolled batch holds one code path
   const int tile_bytes = brows * 128;
   const int M = P.M;
@@ -418,32 +438,34 @@ __device__ __forceinline__ void dit_fill_b(const DitParams& P, int kind, uint8_t
         put(kbi, row, ch, packed);
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive(bready);
+      mbar_arrive(smem_u32(&bready[i0 >> 10]));
     }
   } else {
-    // copied rows: attention output (O) or MLP hidden (down)
+    // copied rows: attention output (O) or MLP hidden (down); brows == M
     const bf16* src = kind == DIT_O ? P.o : P.u;
     const int items = nkb * brows * 8;
-    for (int i0 = 0; i0 < items; i0 += 128 * 8) {
-      uint4 cp[8];
+    uint4 cp[16];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int idx = i0 + u * 128 + et;
-        const int kbi = idx / (brows * 8), rem = idx - kbi * (brows * 8);
-        const int row = rem >> 3, col = (kb0 + kbi) * TC_BK + (rem & 7) * 8;
-        cp[u] = make_uint4(0, 0, 0, 0);
-        if (idx < items && row < M && col < Kd)
-          cp[u] = __ldcg((const uint4*)(src + (size_t)row * Kd + col));
-      }
+    for (int u = 0; u < 16; ++u) {
+      const int idx = u * 128 + et;
+      const int kbi = idx / (brows * 8), rem = idx - kbi * (brows * 8);
+      const int row = rem >> 3, col = (kb0 + kbi) * TC_BK + (rem & 7) * 8;
+      cp[u] = make_uint4(0, 0, 0, 0);
+      if (idx < items && row < M && col < Kd)
+        cp[u] = __ldcg((const uint4*)(src + (size_t)row * Kd + col));
+    }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int idx = i0 + u * 128 + et;
+    for (int half = 0; half < 2; ++half) {
+      if (half * 1024 >= items) break;
+#pragma unroll
+      for (int u = 8 * half; u < 8 * half + 8; ++u) {
+        const int idx = u * 128 + et;
         if (idx >= items) break;
         const int kbi = idx / (brows * 8), rem = idx - kbi * (brows * 8);
         put(kbi, rem >> 3, rem & 7, cp[u]);
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive(bready);
+      mbar_arrive(smem_u32(&bready[half]));
     }
   }
 }
@@ -511,7 +533,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
       mbar_init(smem_u32(&sh->tfull[i]), 1);
       mbar_init(smem_u32(&sh->tempty[i]), 128);
     }
-    mbar_init(smem_u32(&sh->bready), 128);
+    mbar_init(smem_u32(&sh->bready[0]), 128);
+    mbar_init(smem_u32(&sh->bready[1]), 128);
     mbar_init(smem_u32(&sh->rbar), 1);
     sh->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -539,7 +562,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
       uint32_t phase = 0;
       unsigned long long t_prog = gtimer();
       while (ld.valid && !*abort) {
-        if (mbar_try(smem_u32(&sh->empty[stage]), phase ^ 1)) {
+        // with no L2 prefetch to issue, the wait for a free stage suspends
+        if (P.l2_ahead > 0 ? mbar_try(smem_u32(&sh->empty[stage]), phase ^ 1)
+                           : mbar_try_suspend(smem_u32(&sh->empty[stage]), phase ^ 1)) {
           const uint32_t fb = smem_u32(&sh->full[stage]);
           mbar_expect_tx(fb, 16384);
           tma_load_2d(smem_u32(sA + stage * 16384), dit_wmap(P, ld), ld.kb * TC_BK, ld.nt * TC_BM, fb);
@@ -563,7 +588,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
     // ---------------- MMA issuer
     if (lane == 0) {
       int stage = 0, acc = 0;
-      uint32_t phase = 0, acc_phase = 0, b_phase = 0;
+      uint32_t phase = 0, acc_phase = 0, b_phase[2] = {0u, 0u};
       for (int p = 1; p < n_phases - 1 && !*abort; ++p) {
         int l = 0;
         const int kind = dit_phase_kind(p, nb, &l);
@@ -584,8 +609,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
         for (int kb = kb0; kb < kb1; ++kb) {
           if (((kb - kb0) & 7) == 0) {
             // the next 8 k-blocks of the B operand are in shared memory
-            if (!mbar_wait(smem_u32(&sh->bready), b_phase, abort)) { ok = false; break; }
-            b_phase ^= 1;
+            const int bi = (kb - kb0) >> 3;   // batch 0 or 1 (at most 16 k-blocks)
+            if (!mbar_wait(smem_u32(&sh->bready[bi]), b_phase[bi], abort)) { ok = false; break; }
+            b_phase[bi] ^= 1;
             tc_fence_after();
           }
           if (!mbar_wait(smem_u32(&sh->full[stage]), phase, abort)) { ok = false; break; }
@@ -617,20 +643,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
     uint32_t acc_phase = 0, r_phase = 0;
     int it = 0;
     for (int p = 0; p < n_phases; ++p) {
-      {
-        int l0 = 0;
-        const int k0 = dit_phase_kind(p, nb, &l0);
-        if (k0 == DIT_QKV || k0 == DIT_UP) {
-          int N, Kd;
-          dit_gemm_shape(P, k0, &N, &Kd);
-          const int S = P.splits[k0], kbs = Kd / TC_BK;
-          if (cta < (N / TC_BM) * S) {
-            const int z = cta % S;
-            const int kb0 = z * kbs / S, kb1 = (z + 1) * kbs / S;
-            dit_stage_mods(P, k0, l0, kb0 * TC_BK, (kb1 - kb0) * TC_BK, et, sh);
-          }
-        }
-      }
       int l = 0;
       const int kind = dit_phase_kind(p, nb, &l);
       if (kind == -2 && P.skip_final) continue;
@@ -650,16 +662,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
         const int h = cta % P.attn.n_heads, split = cta / P.attn.n_heads;
         if (split < P.attn.n_ctx_splits) {
           const AttnRange rg = attn_range(P.attn, 0, h, split);
-          kv_pre = rg.k0 + min(AM_CHUNK * (DIT_ATTN_ST - 1), rg.k1 - rg.k0) <= P.attn_safe;
-          if (kv_pre) attn_ctx_prologue<1, DIT_ATTN_ST>(P.Kc[l], P.Vc[l], P.attn, h, split, sU, et);
+          kv_pre = rg.k0 + min(AM_CHUNK * DIT_ATTN_ST, rg.k1 - rg.k0) <= P.attn_safe;
+          if (kv_pre)
+            attn_ctx_prologue<1, DIT_ATTN_ST, DIT_ATTN_ST>(P.Kc[l], P.Vc[l], P.attn, h, split, sU, et);
         }
       }
-      if (kind == DIT_QKV && P.n_ctx > 0) {
+      if (kind == DIT_QKV || kind == DIT_UP) {
+        // work that needs nothing this phase waits for: the adaLN shift and
+        // scale of this CTA's columns, and (QKV) the appended context rows
+        // of the B operand, their loads in flight together
         int N, Kd;
         dit_gemm_shape(P, kind, &N, &Kd);
         const int S = P.splits[kind], kbs = Kd / TC_BK, z = cta % S;
         const int kb0 = z * kbs / S, kb1 = (z + 1) * kbs / S;
-        dit_fill_extra(P, sU, kb0, kb1 - kb0, dit_brows(P, kind), Kd, et);
+        float hv[8], cv[8];
+        dit_mods_load(P, kind, l, kb0 * TC_BK, (kb1 - kb0) * TC_BK, et, hv, cv);
+        if (kind == DIT_QKV && P.n_ctx > 0)
+          dit_fill_extra(P, sU, kb0, kb1 - kb0, dit_brows(P, kind), Kd, et);
+        dit_mods_store((kb1 - kb0) * TC_BK, et, hv, cv, sh);
       }
       if (kind != -1) {
         // wait for the units whose outputs this one reads
@@ -713,7 +733,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
           const int nt = cta / S, z = cta % S;
           const int kb0 = z * kbs / S, kb1 = (z + 1) * kbs / S;
           const int brows = dit_brows(P, kind);
-          dit_fill_b(P, kind, sU, kb0, kb1 - kb0, brows, Kd, et, sh, smem_u32(&sh->bready));
+          dit_fill_b(P, kind, sU, kb0, kb1 - kb0, brows, Kd, et, sh, sh->bready);
           const int n = nt * TC_BM + r;
           // residual phases: x and the gate, loaded while the MMAs run
           const bool resid = (kind == DIT_O || kind == DIT_DOWN);

@@ -77,12 +77,27 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// As mbar_try, but a thread whose phase is not complete yet is suspended
+// until the phase completes or about 20 us have passed (the time hint), so
+// a waiting warp takes no issue slots from the warps that share its
+// scheduler.
+__device__ __forceinline__ bool mbar_try_suspend(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(20000u)
+      : "memory");
+  return ok != 0;
+}
 // Waits for the phase with the given parity; false when it timed out or
 // another role of the CTA already gave up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
   if (mbar_try(bar, parity)) return true;
   const unsigned long long t0 = gtimer();
-  while (!mbar_try(bar, parity)) {
+  while (!mbar_try_suspend(bar, parity)) {
     if (*abort) return false;
     if (gtimer() - t0 > TC_TIMEOUT_NS) {
       *abort = 1;
