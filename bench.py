@@ -25,7 +25,6 @@ import json
 import os
 import statistics
 import sys
-import threading
 import time
 
 import numpy as np
@@ -69,59 +68,87 @@ def peaks():
 
 
 # ---------------------------------------------------------------- clocks
+def _clock_child(bus: str, conn, stop) -> None:
+    """Sampler process: SM clock and throttle reasons through NVML as fast as
+    the calls return (a separate process, so the timing loop's GIL does not
+    starve it); sends [(t_before, t_after, mhz, reasons)] on stop."""
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        conn.send(("ready", pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)))
+    except Exception as e:  # pragma: no cover
+        conn.send(("error", str(e)))
+        return
+    out = []
+    while not stop.is_set():
+        t0 = time.monotonic()
+        try:
+            mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+            r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+        except Exception:
+            continue
+        out.append((t0, time.monotonic(), mhz, r))
+        time.sleep(0.0002)
+    conn.send(out)
+
+
 class ClockSampler:
-    """Samples SM clock and throttle reasons through NVML while running."""
+    """SM clock and throttle reasons sampled during the timed region by a
+    separate NVML process; only samples taken inside [enter, exit] count."""
 
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, torch_dev: int, period=0.002):
-        self.samples, self.reasons, self.ok = [], set(), False
-        self.period, self.stop_ev = period, threading.Event()
+    def __init__(self, torch_dev: int):
+        self.samples, self.reasons, self.ok, self.window = [], set(), False, 0.0
+        self.err = ""
         try:
-            import pynvml
+            import multiprocessing as mp
             import torch
-            pynvml.nvmlInit()
             pr = torch.cuda.get_device_properties(torch_dev)
             bus = "%08X:%02X:%02X.0" % (int(pr.pci_domain_id), int(pr.pci_bus_id),
                                         int(pr.pci_device_id))
-            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
-            self.nv = pynvml
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            mctx = mp.get_context("spawn")
+            self.stop = mctx.Event()
+            self.conn, child = mctx.Pipe()
+            self.proc = mctx.Process(target=_clock_child, args=(bus, child, self.stop), daemon=True)
+            self.proc.start()
+            if not self.conn.poll(60):
+                raise RuntimeError("clock sampler did not start")
+            tag, val = self.conn.recv()
+            if tag != "ready":
+                raise RuntimeError(val)
+            self.max_mhz = val
             self.ok = True
         except Exception as e:  # pragma: no cover
             self.err = str(e)
 
-    def _run(self):
-        nv = self.nv
-        while not self.stop_ev.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
-                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for bit, name in self.REASONS.items():
-                    if r & bit:
-                        self.reasons.add(name)
-            except Exception:
-                pass
-            time.sleep(self.period)
-
     def __enter__(self):
-        if self.ok:
-            self.t = threading.Thread(target=self._run, daemon=True)
-            self.t.start()
+        self.t0 = time.monotonic()
         return self
 
     def __exit__(self, *a):
-        if self.ok:
-            self.stop_ev.set()
-            self.t.join()
+        self.t1 = time.monotonic()
+        if not self.ok:
+            return
+        self.stop.set()
+        raw = self.conn.recv() if self.conn.poll(30) else []
+        self.proc.join(10)
+        self.window = self.t1 - self.t0
+        for tb, ta, mhz, r in raw:
+            if tb >= self.t0 and ta <= self.t1:
+                self.samples.append(mhz)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
 
     def summary(self):
         if not self.ok:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable: " + self.err]}
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
-                "samples": len(self.samples)}
+                "samples": len(self.samples), "window_ms": round(1e3 * self.window, 1)}
 
 
 # ---------------------------------------------------------------- algorithmic bytes

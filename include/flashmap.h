@@ -309,6 +309,14 @@ fm_status fm_profile(fm_ctx *ctx, int mask);
  * arrays have FM_PROF_N entries.  Waits for the recorded events. */
 fm_status fm_profile_read(fm_ctx *ctx, double *ms, int64_t *launches, int reset);
 
+/* Self-check of the fp64 exponential the stochastic verify sums with
+ * (Tang's table-driven method; valid for arguments <= 0, the softmax
+ * weights exp((l - max)/T)).  Device arrays: e[n] (arguments), mine[n]
+ * (that function) and ref[n] (CUDA's exp of the same argument).  No
+ * context needed; FM_ERR_ARG for NULL pointers or n < 0.  Asynchronous
+ * on `stream`. */
+fm_status fm_selftest_exp(const double *e, double *mine, double *ref, int n, fm_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

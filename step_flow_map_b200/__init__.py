@@ -26,7 +26,7 @@ EXPORTS = (
     "fm_load_weights", "fm_free", "fm_last_error", "fm_project_context",
     "fm_draft", "fm_verify_greedy", "fm_verify_sample", "fm_profile", "fm_profile_read", "fm_device_status",
     "fm_verify_greedy_noalloc", "fm_draft_factorised", "fm_build_tree", "fm_tree_attention",
-    "fm_verify_greedy_tree", "fm_verify_sample_tree",
+    "fm_verify_greedy_tree", "fm_verify_sample_tree", "fm_selftest_exp",
 )
 FM_PROF = {"embed": 0, "dit_gemm": 1, "attn": 2, "norm": 3, "lm_head": 4, "context": 5,
            "verify": 6, "other": 7}
@@ -100,6 +100,8 @@ def load_library(path: str = LIB_PATH):
     lib.fm_verify_greedy_noalloc.argtypes = [p, p, i, i, i, i, p, p, p, st]
     lib.fm_device_status.restype = i
     lib.fm_device_status.argtypes = [p, st]
+    lib.fm_selftest_exp.restype = i
+    lib.fm_selftest_exp.argtypes = [p, p, p, i, st]
     lib.fm_profile.restype = i
     lib.fm_profile.argtypes = [p, i]
     lib.fm_profile_read.restype = i
@@ -254,6 +256,11 @@ def fm_profile_read(ctx, reset: bool = False, times: bool = True):
     n = (ctypes.c_int64 * FM_PROF_N)()
     _check(load_library().fm_profile_read(ctx, ms, n, int(bool(reset))))
     return (list(ms) if times else None), list(n)
+
+
+def fm_selftest_exp(e, mine, ref, stream=None) -> None:
+    """The verify's fp64 exp (arguments <= 0) and CUDA's exp of fp64 device array e."""
+    _check(load_library().fm_selftest_exp(_ptr(e), _ptr(mine), _ptr(ref), e.numel(), _stream(stream)))
 
 
 def fm_device_status(ctx, stream=None) -> None:

@@ -66,6 +66,7 @@ struct fm_ctx {
   size_t esz = 4;
   fm_weights w;
   std::vector<const void*> wqkv, wo, wup, wdown, wada;
+  void* wkv_all = nullptr;       // every block's key and value weights stacked [nb][2d][d] (bf16)
   std::vector<void*> owned;  // every cudaMalloc of the context
   void* Et = nullptr;        // E transposed, [d][V]
   std::vector<void*> Kc, Vc; // per block [max_seqs][max_ctx][d]
@@ -413,6 +414,18 @@ fm_status load_impl(fm_ctx* c, cudaStream_t st) {
                             c->wup.data(), c->wdown.data(), g.n_blocks, g.d, g.mlp, g.V,
                             g.n_taps * g.target_hidden, g_err, sizeof(g_err)))
         return FM_ERR_CUDA;
+      // the keys and values of appended context rows for every block come
+      // from one GEMM over the stacked key/value weights (one launch, and
+      // enough output tiles to fill the SMs even for a few rows)
+      if (g.n_blocks <= 8) {
+        const size_t per = (size_t)2 * d * d;
+        FM_TRY(dalloc(c, &c->wkv_all, (size_t)g.n_blocks * per * sizeof(T)));
+        for (int l = 0; l < g.n_blocks; ++l)
+          FM_CUDA(cudaMemcpyAsync((T*)c->wkv_all + (size_t)l * per, (const T*)c->wqkv[l] + (size_t)d * d,
+                                  per * sizeof(T), cudaMemcpyDeviceToDevice, st));
+        if (!fm::tc_weight_map(c->tc.kv_all, c->wkv_all, g.n_blocks * 2 * d, d, g_err, sizeof(g_err)))
+          return FM_ERR_CUDA;
+      }
     }
   }
   if constexpr (sizeof(T) == 2) {
@@ -453,6 +466,22 @@ fm_status flush_pending(fm_ctx* c, cudaStream_t st) {
   if (c->pending_rows == 0) return FM_OK;
   const fm_config& g = c->cfg;
   const int d = g.d, R = c->pending_rows;
+  if constexpr (sizeof(T) == 2) {
+   if (c->use_tc && c->tc.kv_all.valid) {
+    fm::EpiCtxKVAll<T> ea;
+    for (int l = 0; l < g.n_blocks; ++l) {
+      ea.Kc[l] = (T*)c->Kc[l];
+      ea.Vc[l] = (T*)c->Vc[l];
+    }
+    ea.d = d;
+    ea.max_ctx = g.max_ctx;
+    ea.map = c->pending_map;
+    FM_TRY(gemm_w<T>(c, FM_PROF_CONTEXT, (const T*)c->c_norm, d, (const T*)c->wkv_all, R,
+                     g.n_blocks * 2 * d, d, ea, st, &c->tc.kv_all));
+    c->pending_rows = 0;
+    return FM_OK;
+   }
+  }
   fm::EpiCtxKV<T> epi;
   epi.d = d;
   epi.max_ctx = g.max_ctx;
@@ -1264,6 +1293,16 @@ extern "C" fm_status fm_profile_read(fm_ctx* c, double* ms, int64_t* launches, i
     for (int k = 0; k < FM_PROF_N; ++k) c->launches[k] = 0;
     c->ev_used = 0;
   }
+  return FM_OK;
+}
+
+extern "C" fm_status fm_selftest_exp(const double* e, double* mine, double* ref, int n,
+                                     fm_stream stream) {
+  if (!e || !mine || !ref || n < 0) return set_err(FM_ERR_ARG, "NULL argument or n < 0");
+  if (n == 0) return FM_OK;
+  fm::k_selftest_exp<<<grid_1d((size_t)n, 256), 256, 0, (cudaStream_t)stream>>>(e, mine, ref, n);
+  const cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return set_err(FM_ERR_CUDA, "self-test launch: %s", cudaGetErrorString(err));
   return FM_OK;
 }
 

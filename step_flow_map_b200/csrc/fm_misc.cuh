@@ -60,21 +60,91 @@ k_adaln(const TI* __restrict__ x, int d, const float* __restrict__ shift,
   __shared__ float sh[32];
   const int m = blockIdx.x;
   const TI* row = x + (size_t)m * d;
+  const int T = blockDim.x;
+  // rows up to 16 T wide stay in registers: one read, all loads in flight
+  constexpr int CACHE = 16;
+  float xv[CACHE];
+  const bool cached = d <= CACHE * T;
   float s = 0.f;
-  for (int c = threadIdx.x; c < d; c += blockDim.x) s += to_f(row[c]);
+  if (cached) {
+#pragma unroll
+    for (int i = 0; i < CACHE; ++i) {
+      const int c = threadIdx.x + i * T;
+      xv[i] = c < d ? to_f(row[c]) : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < CACHE; ++i) s += xv[i];
+  } else {
+    for (int c = threadIdx.x; c < d; c += T) s += to_f(row[c]);
+  }
   const float mean = block_sum(s, sh) / (float)d;
   float v = 0.f;
-  for (int c = threadIdx.x; c < d; c += blockDim.x) {
-    float t = to_f(row[c]) - mean;
-    v = fmaf(t, t, v);
+  if (cached) {
+#pragma unroll
+    for (int i = 0; i < CACHE; ++i) {
+      if (threadIdx.x + i * T < d) {
+        const float t = xv[i] - mean;
+        v = fmaf(t, t, v);
+      }
+    }
+  } else {
+    for (int c = threadIdx.x; c < d; c += T) {
+      float t = to_f(row[c]) - mean;
+      v = fmaf(t, t, v);
+    }
   }
   const float var = block_sum(v, sh) / (float)d;
   const float rstd = rsqrtf(var + 1e-6f);
-  for (int c = threadIdx.x; c < d; c += blockDim.x) {
-    float y = (to_f(row[c]) - mean) * rstd;
-    if (scale) y = y * (1.f + scale[c]) + shift[c];
-    out[(size_t)m * d + c] = from_f<TO>(y);
+  if (cached) {
+#pragma unroll
+    for (int i = 0; i < CACHE; ++i) {
+      const int c = threadIdx.x + i * T;
+      if (c < d) {
+        float y = (xv[i] - mean) * rstd;
+        if (scale) y = y * (1.f + scale[c]) + shift[c];
+        out[(size_t)m * d + c] = from_f<TO>(y);
+      }
+    }
+  } else {
+    for (int c = threadIdx.x; c < d; c += T) {
+      float y = (to_f(row[c]) - mean) * rstd;
+      if (scale) y = y * (1.f + scale[c]) + shift[c];
+      out[(size_t)m * d + c] = from_f<TO>(y);
+    }
   }
+}
+
+// Calls f(v, x) for every v in [v0, v1) of `row`, the bulk through 16-byte
+// loads with four in flight per thread (elements before the first 16-byte
+// boundary and after the last one one by one).  Visiting order differs from
+// index order; callers combine order-independently or break ties by index.
+template <class F>
+__device__ __forceinline__ void for_row_range(const float* __restrict__ row, int v0, int v1, F f) {
+  int a = v0;
+  while (a < v1 && ((reinterpret_cast<uintptr_t>(row + a) & 15) != 0)) {
+    if (a - v0 == (int)threadIdx.x) f(a, row[a]);
+    ++a;
+  }
+  const int nv = (v1 - a) >> 2;                     // whole float4 groups
+  const float4* r4 = reinterpret_cast<const float4*>(row + a);
+  const int T = blockDim.x;
+  int i = threadIdx.x;
+  for (; i + 3 * T < nv; i += 4 * T) {
+    float4 x[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) x[k] = __ldcs(r4 + i + k * T);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int v = a + 4 * (i + k * T);
+      f(v, x[k].x); f(v + 1, x[k].y); f(v + 2, x[k].z); f(v + 3, x[k].w);
+    }
+  }
+  for (; i < nv; i += T) {
+    const float4 x = __ldcs(r4 + i);
+    const int v = a + 4 * i;
+    f(v, x.x); f(v + 1, x.y); f(v + 2, x.z); f(v + 3, x.w);
+  }
+  for (int v = a + 4 * nv + (int)threadIdx.x; v < v1; v += T) f(v, row[v]);
 }
 
 // ------------------------------------------------------------------ softmax rows
@@ -88,14 +158,14 @@ k_softmax_rows(const float* __restrict__ logits, int V, TO* __restrict__ D) {
   __shared__ float sh[32];
   const float* row = logits + (size_t)blockIdx.x * V;
   float mx = -INFINITY;
-  for (int v = threadIdx.x; v < V; v += blockDim.x) mx = fmaxf(mx, row[v]);
+  for_row_range(row, 0, V, [&](int, float x) { mx = fmaxf(mx, x); });
   mx = block_max(mx, sh);
   float s = 0.f;
-  for (int v = threadIdx.x; v < V; v += blockDim.x) s += __expf(row[v] - mx);
+  for_row_range(row, 0, V, [&](int, float x) { s += __expf(x - mx); });
   s = block_sum(s, sh);
   const float inv = 1.f / s;
   TO* out = D + (size_t)blockIdx.x * V;
-  for (int v = threadIdx.x; v < V; v += blockDim.x) out[v] = from_f<TO>(__expf(row[v] - mx) * inv);
+  for_row_range(row, 0, V, [&](int v, float x) { out[v] = from_f<TO>(__expf(x - mx) * inv); });
 }
 
 // ------------------------------------------------------------------ inverse CDF
@@ -234,8 +304,9 @@ k_select_tokens(const float* __restrict__ logits, int V, const float* __restrict
       }
     } else {
       const float* row = logits + (size_t)m * V;
-      for (int v = threadIdx.x; v < V; v += blockDim.x)
-        if (am_better(row[v], v, a.v, a.i)) { a.v = row[v]; a.i = v; }
+      for_row_range(row, 0, V, [&](int v, float x) {
+        if (am_better(x, v, a.v, a.i)) { a.v = x; a.i = v; }
+      });
     }
     a = block_argmax(a, shv, shi);
     if (threadIdx.x == 0) tokens[m] = (a.i == 0x7fffffff) ? 0 : a.i;
@@ -273,7 +344,7 @@ k_sample_chunk_max(const float* __restrict__ logits, int V, TempArgs ta, float* 
   const int v0 = min(V, c * per), v1 = min(V, v0 + per);
   const float* row = logits + (size_t)m * V;
   float mx = -INFINITY;
-  for (int v = v0 + (int)threadIdx.x; v < v1; v += blockDim.x) mx = fmaxf(mx, row[v]);
+  for_row_range(row, v0, v1, [&](int, float x) { mx = fmaxf(mx, x); });
   mx = block_max(mx, sh);
   if (threadIdx.x == 0) cmax[(size_t)m * SAMPLE_CHUNKS + c] = mx;
 }
@@ -294,7 +365,7 @@ k_sample_chunk_sum(const float* __restrict__ logits, int V, TempArgs ta,
   const float* row = logits + (size_t)m * V;
   const float iT = 1.f / T;
   double s = 0.0;
-  for (int v = v0 + (int)threadIdx.x; v < v1; v += blockDim.x) s += (double)expf((row[v] - mx) * iT);
+  for_row_range(row, v0, v1, [&](int, float x) { s += (double)expf((x - mx) * iT); });
   s = block_sum_d(s, sh);
   if (threadIdx.x == 0) csum[(size_t)m * SAMPLE_CHUNKS + c] = s;
 }

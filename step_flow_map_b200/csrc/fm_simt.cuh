@@ -106,6 +106,24 @@ struct EpiCtxKV {
   }
 };
 
+// Keys and values of every block in one GEMM over the blocks' stacked key
+// and value weights (column n: block n / (2d), then keys [0, d), values
+// [d, 2d) of that block); rows map to cache positions as in EpiCtxKV.
+template <typename TO>
+struct EpiCtxKVAll {
+  TO* Kc[8];  // [max_seqs][max_ctx][d] of each block
+  TO* Vc[8];
+  int d, max_ctx;
+  RowMap map;
+  __device__ __forceinline__ void operator()(int r, int n, float v) const {
+    const int l = n / (2 * d), nn = n - l * 2 * d;
+    int q = r / map.n_new, k = r - q * map.n_new;
+    size_t row = (size_t)map.slot[q] * max_ctx + map.pos0[q] + k;
+    if (nn < d) Kc[l][row * d + nn] = from_f<TO>(v);
+    else Vc[l][row * d + (nn - d)] = from_f<TO>(v);
+  }
+};
+
 // QKV of the block rows plus, in the same GEMM, the keys and values of
 // context rows appended after them (rows >= M_draft; their query columns
 // are not needed and are dropped).

@@ -7,6 +7,7 @@
 // rejection, trying the drafts of a tree in index order.
 #pragma once
 #include "fm_misc.cuh"
+#include "fm_exp.cuh"
 
 namespace fm {
 
@@ -40,21 +41,11 @@ k_verify_greedy(const float* __restrict__ tgt, const int* __restrict__ draft, in
   // a tree's rows come through its row map (shared prefixes share a row)
   const float* r = tgt + (size_t)(rowmap ? rowmap[row] : row) * V;
   ArgMax a{-INFINITY, 0x7fffffff};
-  // eight strided loads in flight per thread before they are compared (the
-  // comparison is order-independent: ties go to the lowest index)
-  for (int base = v0 + (int)threadIdx.x; base < v1; base += 8 * (int)blockDim.x) {
-    float x[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int v = base + u * (int)blockDim.x;
-      x[u] = v < v1 ? __ldcs(r + v) : -INFINITY;
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int v = base + u * (int)blockDim.x;
-      if (v < v1 && am_better(x[u], v, a.v, a.i)) { a.v = x[u]; a.i = v; }
-    }
-  }
+  // 16-byte loads, four in flight per thread, compared in any order (ties go
+  // to the lowest index)
+  for_row_range(r, v0, v1, [&](int v, float x) {
+    if (am_better(x, v, a.v, a.i)) { a.v = x; a.i = v; }
+  });
   a = block_argmax(a, shv, shi);
   if (threadIdx.x == 0) {
     pv[(size_t)row * chunks + c] = a.v;
@@ -135,28 +126,30 @@ k_row_stats(const float* __restrict__ tgt, const float* __restrict__ dlog, int n
   const double iT = 1.0 / (double)T;
   float mx = -INFINITY;
   double s = 0.0;
-  for (int base = v0 + (int)threadIdx.x; base < v1; base += 4 * (int)blockDim.x) {
-    float x[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int v = base + u * (int)blockDim.x;
-      x[u] = v < v1 ? __ldcs(r + v) : -INFINITY;
+  // 16-byte loads, four in flight per thread: the row pass is bound by the
+  // bytes in flight, not by the fp64 arithmetic
+  for_row_range(r, v0, v1, [&](int, float x) {
+    if (x > mx) {
+      s = (mx == -INFINITY) ? 0.0 : s * exp_nonpos(((double)mx - (double)x) * iT);
+      mx = x;
     }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      if (x[u] > mx) {
-        s = (mx == -INFINITY) ? 0.0 : s * exp(((double)mx - (double)x[u]) * iT);
-        mx = x[u];
-      }
-      if (x[u] > -INFINITY) s += exp(((double)x[u] - (double)mx) * iT);
-    }
-  }
+    if (x > -INFINITY) s += exp_nonpos(((double)x - (double)mx) * iT);
+  });
   const float M = block_max(mx, shf);
-  double sc = (mx == -INFINITY) ? 0.0 : s * exp(((double)mx - (double)M) * iT);
+  double sc = (mx == -INFINITY) ? 0.0 : s * exp_nonpos(((double)mx - (double)M) * iT);
   sc = block_sum_d(sc, shd);
   if (threadIdx.x == 0) {
     pm[(size_t)row * chunks + c] = M;
     ps[(size_t)row * chunks + c] = sc;
+  }
+}
+
+// Both exponentials of each argument, for the self-check entry point.
+__global__ void k_selftest_exp(const double* __restrict__ e, double* __restrict__ mine,
+                               double* __restrict__ ref, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    mine[i] = exp_nonpos(e[i]);
+    ref[i] = exp(e[i]);
   }
 }
 
@@ -175,7 +168,7 @@ __device__ __forceinline__ RowStat warp_combine_stats(const float* pm, const dou
   double S = 0.0;
   for (int c = lane; c < chunks; c += 32) {
     const double mc = (double)pm[(size_t)row * chunks + c];
-    if (mc > -INFINITY) S += ps[(size_t)row * chunks + c] * exp((mc - m) / T);
+    if (mc > -INFINITY) S += ps[(size_t)row * chunks + c] * exp_nonpos((mc - m) / T);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
@@ -243,8 +236,8 @@ k_verify_sample_decide(const float* __restrict__ tgt, const float* __restrict__ 
       const double iSp = 1.0 / s_Sp, iSq = qp ? 1.0 / s_Sq : 0.0;
       double local = 0.0;
       for (int v = tid; v < V; v += blockDim.x) {
-        double p = (mode == 0) ? exp(((double)tp[v] - mp) * iT) * iSp : buf[src][v];
-        double q = qp ? exp(((double)qp[v] - mq) * iT) * iSq : (v == y ? 1.0 : 0.0);
+        double p = (mode == 0) ? exp_nonpos(((double)tp[v] - mp) * iT) * iSp : buf[src][v];
+        double q = qp ? exp_nonpos(((double)qp[v] - mq) * iT) * iSq : (v == y ? 1.0 : 0.0);
         double r = fmax(p - q, 0.0);
         buf[dst][v] = r;
         local += r;
@@ -257,7 +250,7 @@ k_verify_sample_decide(const float* __restrict__ tgt, const float* __restrict__ 
         if (tid == 0) { s_mode = 1; s_buf = dst; }
       } else if (mode == 0) {
         // p' stays the target row itself: materialise it for later steps
-        for (int v = tid; v < V; v += blockDim.x) buf[dst][v] = exp(((double)tp[v] - mp) * iT) * iSp;
+        for (int v = tid; v < V; v += blockDim.x) buf[dst][v] = exp_nonpos(((double)tp[v] - mp) * iT) * iSp;
         __syncthreads();
         if (tid == 0) { s_mode = 1; s_buf = dst; }
       }
@@ -271,7 +264,7 @@ k_verify_sample_decide(const float* __restrict__ tgt, const float* __restrict__ 
       int tok;
       if (s_mode == 0) {
         const double mp = s_mp, iSp = 1.0 / s_Sp;
-        auto wf = [&](int v) { return exp(((double)tp[v] - mp) * iT) * iSp; };
+        auto wf = [&](int v) { return exp_nonpos(((double)tp[v] - mp) * iT) * iSp; };
         tok = block_sample(wf, V, u);
       } else {
         const double* pb = buf[s_buf];
@@ -298,7 +291,7 @@ k_verify_sample_decide(const float* __restrict__ tgt, const float* __restrict__ 
     }
     __syncthreads();
     const double mp = s_mp, iSp = 1.0 / s_Sp, u = ures[b];
-    auto wf = [&](int v) { return exp(((double)tp[v] - mp) * iT) * iSp; };
+    auto wf = [&](int v) { return exp_nonpos(((double)tp[v] - mp) * iT) * iSp; };
     int tok = block_sample(wf, V, u);
     if (tid == 0) o[K] = tok;
   } else {
@@ -400,11 +393,11 @@ struct Vs1Weight {
   double mp, iSp, mq, iSq, iT;
   int y;
   bool resid;
-  __device__ __forceinline__ double p(int v) const { return exp(((double)tp[v] - mp) * iT) * iSp; }
+  __device__ __forceinline__ double p(int v) const { return exp_nonpos(((double)tp[v] - mp) * iT) * iSp; }
   __device__ __forceinline__ double operator()(int v) const {
     const double pv = p(v);
     if (!resid) return pv;
-    const double qv = qp ? exp(((double)qp[v] - mq) * iT) * iSq : (v == y ? 1.0 : 0.0);
+    const double qv = qp ? exp_nonpos(((double)qp[v] - mq) * iT) * iSq : (v == y ? 1.0 : 0.0);
     return fmax(pv - qv, 0.0);
   }
 };
@@ -443,7 +436,7 @@ k_vs1_sums(const float* __restrict__ tgt, const float* __restrict__ dlog, int V,
     const double pv = w.p(v);
     sp += pv;
     if (w.resid) {
-      const double qv = w.qp ? exp(((double)w.qp[v] - w.mq) * w.iT) * w.iSq : (v == w.y ? 1.0 : 0.0);
+      const double qv = w.qp ? exp_nonpos(((double)w.qp[v] - w.mq) * w.iT) * w.iSq : (v == w.y ? 1.0 : 0.0);
       sw += fmax(pv - qv, 0.0);
     }
   }
