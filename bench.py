@@ -363,19 +363,20 @@ def run_fm(args, w, rank, world, local_rank):
     out_tok = torch.empty((B, K + 1), dtype=torch.int32, device="cuda")
     g, h0 = len(greedy), len(greedy)
 
-    def step(rd, n_acc, st):
+    def step(rd, n_acc, st, outs=None):
+        br, ot = outs if outs is not None else (branch, out_tok)
         if w.new_rows:
             fmb.fm_project_context(ctx.ctx, seqs, rd["hidden"], w.new_rows, [w.ctx] * B, st)
         fmb.fm_draft(ctx.ctx, seqs, rd["noise"], N, w.t_grid, w.temps, rd["u_draft"], tokens, dlog,
                      st)
         tgt = rd["target"]
         if g:
-            fmb.fm_verify_greedy(ctx.ctx, tgt, tokens, g, N, K, V, n_acc, branch, out_tok, st)
+            fmb.fm_verify_greedy(ctx.ctx, tgt, tokens, g, N, K, V, n_acc, br, ot, st)
         if sampled:
             ns = B - g
             fmb.fm_verify_sample(ctx.ctx, tgt[h0:], dlog[h0:], tokens[h0:], ns, N, K, V,
                                  w.temps[h0], rd["u_accept"][h0:], rd["u_res"][h0:],
-                                 n_acc[h0:], branch[h0:], out_tok[h0:], st)
+                                 n_acc[h0:], br[h0:], ot[h0:], st)
 
     def barrier():
         torch.cuda.synchronize()
@@ -567,7 +568,12 @@ def run_fm(args, w, rank, world, local_rank):
         # last read its buffer, and each step after its upload)
         dev_in = [{k: (torch.empty_like(v) if v is not None else None) for k, v in rounds[0].items()}
                   for _ in range(2)]
-        n_stage = torch.zeros(B, dtype=torch.int32, device="cuda")
+        # two sets of device outputs, one per input buffer: the copy stream
+        # reads step k's results (accepted lengths and tokens) back while
+        # step k + 1 writes the other set
+        n_stage = [torch.zeros(B, dtype=torch.int32, device="cuda") for _ in range(2)]
+        outs = [(torch.empty(B, dtype=torch.int32, device="cuda"),
+                 torch.empty((B, K + 1), dtype=torch.int32, device="cuda")) for _ in range(2)]
         host_n = torch.empty((args.steps, B), dtype=torch.int32).pin_memory()
         host_tok = torch.empty((args.steps, B, K + 1), dtype=torch.int32).pin_memory()
         h2d = sum(v.numel() * v.element_size() for v in pin[0].values() if v is not None)
@@ -580,12 +586,13 @@ def run_fm(args, w, rank, world, local_rank):
                         dev_in[bi][key].copy_(v)
                 gstage[bi] = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(gstage[bi]):
-                    step(dev_in[bi], n_stage, torch.cuda.current_stream())
+                    step(dev_in[bi], n_stage[bi], torch.cuda.current_stream(), outs[bi])
         torch.cuda.synchronize()
         barrier()
         cs = torch.cuda.Stream()
         copied = [torch.cuda.Event(), torch.cuda.Event()]
         used = [torch.cuda.Event(), torch.cuda.Event()]
+        read = [torch.cuda.Event(), torch.cuda.Event()]
 
         def upload(k: int, bi: int):
             with torch.cuda.stream(cs):
@@ -596,6 +603,13 @@ def run_fm(args, w, rank, world, local_rank):
                         dev_in[bi][key].copy_(v, non_blocking=True)
                 copied[bi].record(cs)
 
+        def download(k: int, bi: int):
+            with torch.cuda.stream(cs):
+                cs.wait_event(used[bi])
+                host_n[k].copy_(n_stage[bi], non_blocking=True)
+                host_tok[k].copy_(outs[bi][1], non_blocking=True)
+                read[bi].record(cs)
+
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         cs.wait_event(e0)
@@ -605,13 +619,15 @@ def run_fm(args, w, rank, world, local_rank):
             if k + 1 < args.steps:
                 upload(k + 1, 1 - bi)
             stream.wait_event(copied[bi])
+            if k >= 2:
+                stream.wait_event(read[bi])     # step k - 2's results are read
             if gstage[bi] is not None:
                 gstage[bi].replay()
             else:
-                step(dev_in[bi], n_stage, stream)
+                step(dev_in[bi], n_stage[bi], stream, outs[bi])
             used[bi].record(stream)
-            host_n[k].copy_(n_stage, non_blocking=True)
-            host_tok[k].copy_(out_tok, non_blocking=True)
+            download(k, bi)
+        stream.wait_stream(cs)
         e1.record(stream)
         torch.cuda.synchronize()
         ems = max_over_ranks(e0.elapsed_time(e1))
