@@ -9,7 +9,8 @@
 // exact value) and exp(r) from its Taylor series through r^6 (the remainder
 // is below 4e-18 relative for |r| <= ln2/64).  ln2/32 is split into a
 // 37-bit head (k * head is exact for |k| < 2^16) and a tail, so r keeps full
-// precision.  Below e = -700 the weight (< 1e-304) is returned as 0: it
+// precision; k is rounded with the 1.5 * 2^52 shifter (Cody and Waite's
+// trick) instead of conversion instructions.  Below e = -700 the weight (< 1e-304) is returned as 0: it
 // cannot change a row sum that holds exp(0) = 1.  -inf gives 0, NaN gives
 // NaN.  About a dozen fp64 operations instead of a general exp's range
 // handling; the GPU tests compare it with CUDA's exp over [-700, 0].
@@ -32,7 +33,12 @@ __device__ const double g_exp2_32[32] = {
 
 __device__ __forceinline__ double exp_nonpos(double e) {
   if (!(e > -700.0)) return (e == e) ? 0.0 : e;
-  const double kf = rint(e * 0x1.71547652b82fep+5);               // e * 32 / ln2
+  // k = round(e * 32 / ln2) by adding 1.5 * 2^52 (the sum's unit in the last
+  // place is 1, so the addition rounds to the nearest integer and its low
+  // word holds k in two's complement): no conversion instructions
+  const double t = fma(e, 0x1.71547652b82fep+5, 0x1.8p52);
+  const double kf = t - 0x1.8p52;
+  const int k = __double2loint(t);
   const double r = fma(-kf, 0x1.cf79abc9e3b3ap-45, fma(-kf, 0x1.62e42fefa0000p-6, e));
   double p = 1.0 / 720.0;
   p = fma(p, r, 1.0 / 120.0);
@@ -41,7 +47,6 @@ __device__ __forceinline__ double exp_nonpos(double e) {
   p = fma(p, r, 0.5);
   p = fma(p, r, 1.0);
   p = fma(p, r, 1.0);
-  const int k = (int)kf;
   const int j = k & 31, q = k >> 5;                                 // q = floor(k / 32)
   // scale by 2^q through the exponent field (the result stays normal)
   return __longlong_as_double(__double_as_longlong(p * __ldg(&g_exp2_32[j])) + ((long long)q << 52));

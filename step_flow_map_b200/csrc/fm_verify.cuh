@@ -125,16 +125,60 @@ k_row_stats(const float* __restrict__ tgt, const float* __restrict__ dlog, int n
   const int v0 = min(V, c * per), v1 = min(V, v0 + per);
   const double iT = 1.0 / (double)T;
   float mx = -INFINITY;
+  double mxd = -INFINITY;   // mx as a double
   double s = 0.0;
-  // 16-byte loads, four in flight per thread: the row pass is bound by the
-  // bytes in flight, not by the fp64 arithmetic
-  for_row_range(r, v0, v1, [&](int, float x) {
+  // one element: running max, the sum rescaled when the max grows
+  auto one = [&](float x) {
+    const double xd = (double)x;
     if (x > mx) {
-      s = (mx == -INFINITY) ? 0.0 : s * exp_nonpos(((double)mx - (double)x) * iT);
+      s = (mx == -INFINITY) ? 0.0 : s * exp_nonpos((mxd - xd) * iT);
       mx = x;
+      mxd = xd;
     }
-    if (x > -INFINITY) s += exp_nonpos(((double)x - (double)mx) * iT);
-  });
+    if (x > -INFINITY) s += exp_nonpos((xd - mxd) * iT);
+  };
+  // the bulk: sixteen values per thread from four 16-byte loads in flight;
+  // the max of the sixteen first (one rescale at most), then sixteen
+  // independent exponentials into four partial sums (NaN never raises the
+  // max -- fmaxf ignores it -- and adds nothing, as in `one`)
+  int a = v0;
+  while (a < v1 && ((reinterpret_cast<uintptr_t>(r + a) & 15) != 0)) {
+    if (a - v0 == (int)threadIdx.x) one(r[a]);
+    ++a;
+  }
+  const int nv = (v1 - a) >> 2;
+  const float4* r4 = reinterpret_cast<const float4*>(r + a);
+  const int TT = blockDim.x;
+  int i = threadIdx.x;
+  for (; i + 3 * TT < nv; i += 4 * TT) {
+    float x[16];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float4 q = __ldcs(r4 + i + k * TT);
+      x[4 * k] = q.x; x[4 * k + 1] = q.y; x[4 * k + 2] = q.z; x[4 * k + 3] = q.w;
+    }
+    float bm = x[0];
+#pragma unroll
+    for (int k = 1; k < 16; ++k) bm = fmaxf(bm, x[k]);
+    if (bm > mx) {
+      const double bd = (double)bm;
+      s = (mx == -INFINITY) ? 0.0 : s * exp_nonpos((mxd - bd) * iT);
+      mx = bm;
+      mxd = bd;
+    }
+    if (mx > -INFINITY) {
+      double acc[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        if (x[k] > -INFINITY) acc[k & 3] += exp_nonpos(((double)x[k] - mxd) * iT);
+      s += (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    }
+  }
+  for (; i < nv; i += TT) {
+    const float4 q = __ldcs(r4 + i);
+    one(q.x); one(q.y); one(q.z); one(q.w);
+  }
+  for (int v = a + 4 * nv + (int)threadIdx.x; v < v1; v += TT) one(r[v]);
   const float M = block_max(mx, shf);
   double sc = (mx == -INFINITY) ? 0.0 : s * exp_nonpos(((double)mx - (double)M) * iT);
   sc = block_sum_d(sc, shd);
