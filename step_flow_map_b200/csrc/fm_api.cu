@@ -114,6 +114,12 @@ struct fm_ctx {
   float* vs_pm = nullptr;
   double* vs_ps = nullptr;
   double* vs_resid = nullptr;
+  // the tree's stochastic verify over many CTAs per sequence: per-chunk
+  // partial sums [max_seqs][VT_MAX_CHUNKS], abort word + one barrier
+  // counter per sequence, resident CTAs of that kernel per SM
+  double* vt_part = nullptr;
+  unsigned* vt_bar = nullptr;
+  int vt_per_sm = 0;
   fm::Vs1Plan* vs1_plan = nullptr;   // one-draft stochastic verify: the draw of each sequence
   double* vs1_csum = nullptr;        //   and its per-chunk weight sums
   bool use_tc = false;
@@ -402,6 +408,15 @@ fm_status load_impl(fm_ctx* c, cudaStream_t st) {
   FM_TRY(dalloc_t(c, &c->vs_pm, vrows * c->v_chunks));
   FM_TRY(dalloc_t(c, &c->vs_ps, vrows * c->v_chunks));
   FM_TRY(dalloc_t(c, &c->vs_resid, (size_t)g.max_seqs * 2 * g.V));
+  FM_TRY(dalloc_t(c, &c->vt_part, (size_t)g.max_seqs * fm::VT_MAX_CHUNKS));
+  FM_TRY(dalloc_t(c, &c->vt_bar, (size_t)g.max_seqs + 1));
+  {
+    int coop = 0;
+    cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, c->dev);
+    if (coop)
+      FM_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&c->vt_per_sm, fm::k_vtree,
+                                                            fm::VT_THREADS, 0));
+  }
   FM_TRY(dalloc_t(c, &c->vs1_plan, (size_t)g.max_seqs));
   FM_TRY(dalloc_t(c, &c->vs1_csum, (size_t)g.max_seqs * fm::VS1_CHUNKS * 2));
   FM_TRY(dalloc_t(c, &c->tc.err, 1));
@@ -1153,6 +1168,29 @@ static fm_status verify_sample_impl(fm_ctx* c, const float* target_logits,
     FM_LAUNCH(c, FM_PROF_VERIFY, fm::k_vs1_pick, B, 512, 0, st, target_logits, draft_logits, K, V,
               temperature, u_res, (const fm::Vs1Plan*)c->vs1_plan, (const double*)c->vs1_csum,
               out_tokens, rowmap);
+    return FM_OK;
+  }
+  // the tree: C CTAs per sequence share each pass over the vocabulary
+  // (cooperative launch, so the CTAs that wait on one another are resident)
+  const long capacity = (long)c->sms * c->vt_per_sm;
+  const int C = (int)std::min<long>({(long)fm::VT_MAX_CHUNKS, capacity / B, std::max(1, V / 1024)});
+  if (C >= 2) {
+    FM_CUDA(cudaMemsetAsync(c->vt_bar, 0, (size_t)(B + 1) * sizeof(unsigned), st));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(B * C));
+    cfg.blockDim = dim3(fm::VT_THREADS);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    FM_CUDA(cudaLaunchKernelEx(&cfg, fm::k_vtree, target_logits, draft_logits, draft, B, N, K, V,
+                               temperature, u_accept, u_res, (const float*)c->vs_pm,
+                               (const double*)c->vs_ps, ch, c->vs_resid, C, c->vt_part, c->vt_bar,
+                               c->tc.err, n_acc, branch, out_tokens, rowmap));
+    c->launches[FM_PROF_VERIFY]++;
     return FM_OK;
   }
   FM_LAUNCH(c, FM_PROF_VERIFY, (fm::k_verify_sample_decide), B, fm::VS_DECIDE_THREADS, 0, st,

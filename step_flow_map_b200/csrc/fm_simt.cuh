@@ -122,7 +122,28 @@ struct EpiCtxKVAll {
     if (nn < d) Kc[l][row * d + nn] = from_f<TO>(v);
     else Vc[l][row * d + (nn - d)] = from_f<TO>(v);
   }
+  // rows r0 .. r0 + count - 1 (count <= 16) of column n: the block, the
+  // key/value half and the first row's sequence are found once, the later
+  // rows step through the sequences' row ranges
+  __device__ __forceinline__ void chunk16(int r0, int n, const float* v, int count) const {
+    const int l = n / (2 * d), nn = n - l * 2 * d;
+    TO* col = nn < d ? Kc[l] + nn : Vc[l] + (nn - d);
+    int q = r0 / map.n_new, k = r0 - q * map.n_new;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (j < count) {
+        col[((size_t)map.slot[q] * max_ctx + map.pos0[q] + k) * d] = from_f<TO>(v[j]);
+        if (++k == map.n_new) {
+          k = 0;
+          ++q;
+        }
+      }
+    }
+  }
 };
+
+template <typename TO>
+struct has_chunk16<EpiCtxKVAll<TO>> : std::true_type {};
 
 // QKV of the block rows plus, in the same GEMM, the keys and values of
 // context rows appended after them (rows >= M_draft; their query columns

@@ -8,6 +8,7 @@
 #pragma once
 #include "fm_misc.cuh"
 #include "fm_exp.cuh"
+#include "fm_tc.cuh"
 
 namespace fm {
 
@@ -342,6 +343,227 @@ k_verify_sample_decide(const float* __restrict__ tgt, const float* __restrict__ 
     r0 = __ffs(alive) - 1;
   }
   if (tid == 0) {
+    for (int i = n_done + 1; i <= K; ++i) o[i] = -1;
+    n_acc[b] = n_done;
+    branch[b] = r0;
+  }
+}
+
+// ------------------------------------------------------------------ stochastic, tree, many CTAs
+// The same walk as k_verify_sample_decide, run by C CTAs per sequence
+// (cooperative launch: every CTA resident).  Each CTA owns one vocabulary
+// chunk of the sequence's residual buffers and computes every decision of
+// the walk itself from the same inputs, so all of them take the same path;
+// a full-vocabulary quantity (a residual's mass, the sampled distribution's
+// chunk sums) is a per-chunk partial, summed by every CTA in chunk order
+// after a barrier of the sequence's CTAs.  One barrier per pass, so a
+// rejection costs two short passes over 1/C of the vocabulary instead of
+// full-vocabulary passes on one SM.
+constexpr int VT_THREADS = 256;
+constexpr int VT_MAX_CHUNKS = 128;
+
+// Barrier of the C CTAs of one sequence: the k-th call returns once all C
+// have arrived for the k-th time (target C k on a counter zeroed before the
+// launch), after at most TC_TIMEOUT_NS; false when it gave up or another
+// CTA did (the abort word), with the error word set.
+__device__ __forceinline__ bool vt_barrier(unsigned* bar, unsigned target, int* abort_g, int* err) {
+  __shared__ int s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    red_add_release_gpu(bar, 1u);
+    const unsigned long long t0 = gtimer();
+    int ok = 1;
+    for (unsigned n = 1;; ++n) {
+      unsigned v;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
+      if (v >= target) break;
+      if ((n & 31) == 0) {
+        if (*(volatile int*)abort_g) { ok = 0; break; }
+        if (gtimer() - t0 > TC_TIMEOUT_NS) {
+          atomicExch(abort_g, 1);
+          atomicExch(err, TC_ERR_TIMEOUT);
+          ok = 0;
+          break;
+        }
+      }
+    }
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0;
+}
+
+__global__ void __launch_bounds__(VT_THREADS)
+k_vtree(const float* __restrict__ tgt, const float* __restrict__ dlog, const int* __restrict__ draft,
+        int B, int N, int K, int V, float T, const double* __restrict__ ua,
+        const double* __restrict__ ures, const float* __restrict__ pm, const double* __restrict__ ps,
+        int chunks, double* __restrict__ resid, int C, double* __restrict__ vpart,
+        unsigned* __restrict__ vbar, int* __restrict__ err, int* __restrict__ n_acc,
+        int* __restrict__ branch, int* __restrict__ out, const int* __restrict__ rowmap) {
+  __shared__ double shd[32];
+  __shared__ int s_accept, s_own;
+  __shared__ double s_mp, s_Sp, s_mq, s_Sq, s_Z, s_u;
+  const int b = blockIdx.x / C, g = blockIdx.x - b * C, tid = threadIdx.x;
+  int* abort_g = (int*)vbar;
+  unsigned* bar = vbar + 1 + b;
+  unsigned epoch = 0;
+  const double dT = (double)T, iT = 1.0 / dT;
+  const int n_tgt_rows = B * N * (K + 1);
+  const int per = (V + C - 1) / C;
+  const int v0 = min(V, g * per), v1 = min(V, v0 + per);
+  double* part = vpart + (size_t)b * C;
+  double* buf[2] = {resid + (size_t)b * 2 * V, resid + (size_t)b * 2 * V + V};
+  int* o = out + (size_t)b * (K + 1);
+  unsigned alive = (N >= 32) ? 0xffffffffu : ((1u << N) - 1u);
+  int n_done = K, r0 = 0;
+  bool ok = true;
+
+  // draws a token from the current distribution p' (mode 0: the target row
+  // given by (tp, mp, Sp); mode 1: buf[cur]) at u: chunk sums, a barrier,
+  // then the chunk holding u * total (fixed chunk order) is searched by its
+  // owner, which writes o[pos]
+  auto sample = [&](const float* tp, int mode, int cur, double u, int pos) -> bool {
+    const double mp = s_mp, iSp = 1.0 / s_Sp;
+    double local = 0.0;
+    for (int v = v0 + tid; v < v1; v += VT_THREADS)
+      local += (mode == 0) ? exp_nonpos(((double)tp[v] - mp) * iT) * iSp : buf[cur][v];
+    local = block_sum_d(local, shd);
+    if (tid == 0) part[g] = local;
+    if (!vt_barrier(bar, (unsigned)C * ++epoch, abort_g, err)) return false;
+    if (tid == 0) {
+      double tot = 0.0;
+      for (int k = 0; k < C; ++k) tot += part[k];
+      const double target = u * tot;
+      double pre = 0.0;
+      int own = -1, last_pos = 0;
+      for (int k = 0; k < C; ++k) {
+        const double sc = part[k];
+        if (sc > 0.0) last_pos = k;
+        if (own < 0 && pre + sc > target) own = k;
+        else if (own < 0) pre += sc;
+      }
+      if (own < 0) {                       // rounding: the last chunk with mass
+        own = last_pos;
+        pre = 0.0;
+        for (int k = 0; k < own; ++k) pre += part[k];
+      }
+      const double sc = part[own];
+      s_own = own;
+      s_u = sc > 0.0 ? fmin(fmax((target - pre) / sc, 0.0), 1.0) : 0.0;
+    }
+    __syncthreads();
+    if (s_own == g) {
+      int tok;
+      if (mode == 0) {
+        auto wf = [&](int v) { return exp_nonpos(((double)tp[v0 + v] - mp) * iT) * iSp; };
+        tok = v0 + block_sample(wf, v1 - v0, s_u);
+      } else {
+        const double* pb = buf[cur] + v0;
+        auto wf = [&](int v) { return pb[v]; };
+        tok = v0 + block_sample(wf, v1 - v0, s_u);
+      }
+      if (tid == 0) o[pos] = tok;
+    }
+    return true;
+  };
+
+  for (int i = 0; i < K && ok; ++i) {
+    r0 = __ffs(alive) - 1;
+    const int trow = (b * N + r0) * (K + 1) + i;
+    const float* tp = tgt + (size_t)(rowmap ? rowmap[trow] : trow) * V;
+    if (tid < 32) {
+      RowStat st = warp_combine_stats(pm, ps, trow, chunks, dT, tid);
+      if (tid == 0) { s_mp = st.m; s_Sp = st.S; }
+    }
+    __syncthreads();
+    int mode = 0, cur = 0, acc = -1;
+    for (int j = 0; j < N; ++j) {
+      if (!((alive >> j) & 1u)) continue;
+      const int y = draft[((size_t)b * N + j) * K + i];
+      const int drow = (b * N + j) * K + i;
+      const float* qp = dlog ? dlog + (size_t)drow * V : nullptr;
+      if (tid < 32) {
+        RowStat sq{0.0, 1.0};
+        if (qp) sq = warp_combine_stats(pm, ps, n_tgt_rows + drow, chunks, dT, tid);
+        if (tid == 0) {
+          double qy = 1.0;
+          if (qp) {
+            s_mq = sq.m; s_Sq = sq.S;
+            qy = exp(((double)qp[y] - sq.m) / dT) / sq.S;
+          }
+          const double py = (mode == 0) ? exp(((double)tp[y] - s_mp) / dT) / s_Sp : buf[cur][y];
+          s_accept = (ua[((size_t)b * N + j) * K + i] * qy < py) ? y : -1;
+        }
+      }
+      __syncthreads();
+      acc = s_accept;
+      if (acc >= 0) break;
+      // residual r = max(0, p' - q_j) on this CTA's chunk, its mass summed
+      // over the chunks, then p' = r / mass
+      const int dst = mode == 0 ? 0 : 1 - cur;
+      const double mp = s_mp, mq = s_mq;
+      const double iSp = 1.0 / s_Sp, iSq = qp ? 1.0 / s_Sq : 0.0;
+      double local = 0.0;
+      for (int v = v0 + tid; v < v1; v += VT_THREADS) {
+        const double pv = (mode == 0) ? exp_nonpos(((double)tp[v] - mp) * iT) * iSp : buf[cur][v];
+        const double qv = qp ? exp_nonpos(((double)qp[v] - mq) * iT) * iSq : (v == y ? 1.0 : 0.0);
+        const double rv = fmax(pv - qv, 0.0);
+        buf[dst][v] = rv;
+        local += rv;
+      }
+      local = block_sum_d(local, shd);
+      if (tid == 0) part[g] = local;
+      if (!vt_barrier(bar, (unsigned)C * ++epoch, abort_g, err)) { ok = false; break; }
+      if (tid == 0) {
+        double Z = 0.0;
+        for (int k = 0; k < C; ++k) Z += part[k];
+        s_Z = Z;
+      }
+      __syncthreads();
+      const double Z = s_Z;
+      if (Z > 0.0) {
+        const double iZ = 1.0 / Z;
+        for (int v = v0 + tid; v < v1; v += VT_THREADS) buf[dst][v] *= iZ;
+        mode = 1;
+        cur = dst;
+      } else if (mode == 0) {
+        // p' stays the target row itself: materialise it for later steps
+        for (int v = v0 + tid; v < v1; v += VT_THREADS)
+          buf[dst][v] = exp_nonpos(((double)tp[v] - mp) * iT) * iSp;
+        mode = 1;
+        cur = dst;
+      }
+      // buf[cur] complete on every chunk before any CTA reads an entry of
+      // another's (the next accept test), and the partials are free again
+      if (!vt_barrier(bar, (unsigned)C * ++epoch, abort_g, err)) { ok = false; break; }
+    }
+    if (!ok) break;
+    if (acc < 0) {
+      if (!sample(tp, mode, cur, ures[b], i)) { ok = false; break; }
+      n_done = i;
+      break;
+    }
+    if (g == 0 && tid == 0) o[i] = acc;
+    unsigned keep = 0u;
+    for (int j = 0; j < N; ++j)
+      if (((alive >> j) & 1u) && draft[((size_t)b * N + j) * K + i] == acc) keep |= 1u << j;
+    alive = keep;
+  }
+  if (!ok) return;
+  if (n_done == K) {
+    r0 = __ffs(alive) - 1;
+    const int trow = (b * N + r0) * (K + 1) + K;
+    const float* tp = tgt + (size_t)(rowmap ? rowmap[trow] : trow) * V;
+    if (tid < 32) {
+      RowStat st = warp_combine_stats(pm, ps, trow, chunks, dT, tid);
+      if (tid == 0) { s_mp = st.m; s_Sp = st.S; }
+    }
+    __syncthreads();
+    if (!sample(tp, 0, 0, ures[b], K)) return;
+  } else {
+    r0 = __ffs(alive) - 1;
+  }
+  if (g == 0 && tid == 0) {
     for (int i = n_done + 1; i <= K; ++i) o[i] = -1;
     n_acc[b] = n_done;
     branch[b] = r0;
