@@ -729,11 +729,19 @@ fm_status tc_launch(const TcMap& wm, const bf16* A, int lda, int M, Epi epi, flo
   a.k_blocks = (wm.Kd + TC_BK - 1) / TC_BK;
   const int tiles = a.n_tiles * a.m_tiles;
   // K splits only while tiles leave SMs idle (measured: more splits than
-  // that lose to the serial reduction of their partial tiles)
+  // that lose to the serial reduction of their partial tiles), and no more
+  // than balance a split's weight stream against the last arrival's pull of
+  // all partial tiles: with per-split weight bytes W/S and S partial tiles of
+  // P bytes, S ~ sqrt(W/P) (the O projection at 64 rows: 4 splits of its
+  // 512 KB weight tile instead of 9, each partial 32 KB)
   int splits = 1;
   if (tiles < sms) {
     splits = sms / tiles;
     splits = splits > a.k_blocks ? a.k_blocks : splits;
+    const double w_tile = (double)a.k_blocks * TC_BK * TC_BM * 2.0;
+    const double p_tile = (double)TC_BM * BN * 4.0;
+    const int s_bal = (int)ceil(sqrt(w_tile / p_tile));
+    if (splits > s_bal) splits = s_bal;
     while (splits > 1 && (size_t)splits * tiles * TC_BM * BN > partial_elems) --splits;
   }
   if (splits > 1 && tiles > tile_cnt_n) splits = 1;
