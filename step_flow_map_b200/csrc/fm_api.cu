@@ -384,7 +384,7 @@ fm_status load_impl(fm_ctx* c, cudaStream_t st) {
   c->tile_cnt_n = 1 << 16;
   FM_TRY(dalloc_t(c, &c->tile_cnt, c->tile_cnt_n));
   FM_CUDA(cudaMemsetAsync(c->tile_cnt, 0, c->tile_cnt_n * sizeof(unsigned), st));
-  c->attn_pairs_max = call_seqs * g.n_heads;
+  c->attn_pairs_max = call_seqs * g.max_noise * g.n_heads;
   c->attn_part_elems = (size_t)(2 * c->sms + 2 * c->attn_pairs_max) * g.max_noise * 16 * fm::AM_PSTRIDE;
   FM_TRY(dalloc_t(c, &c->attn_part, c->attn_part_elems));
   FM_TRY(dalloc_t(c, &c->attn_cnt, (size_t)c->attn_pairs_max));
@@ -444,6 +444,9 @@ fm_status load_impl(fm_ctx* c, cudaStream_t st) {
     }
   }
   if constexpr (sizeof(T) == 2) {
+    // diagnostic: split-K GEMMs reduce through global memory only
+    const char* ncl = getenv("FM_DISABLE_TC_CLUSTER");
+    fm::tc_cluster_ok = !(ncl && *ncl == '1');
     int coop = 0;
     cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, c->dev);
     const char* off = getenv("FM_DISABLE_PERSISTENT");  // diagnostic: per-kernel DiT path
@@ -558,10 +561,35 @@ fm_status attn_mma_launch(fm_ctx* c, const fm::AttnMmaArgs& am, dim3 grid, const
   return FM_OK;
 }
 
+// Whether attn_mma can run every noise draft of n_seqs sequences as its own
+// one-draft sequence.
+static bool attn_split_drafts_ok(const fm_ctx* c, int n_seqs, int n_noise) {
+  return n_seqs * n_noise <= 256 && n_seqs * n_noise * c->cfg.n_heads <= c->attn_pairs_max;
+}
+
 // Split count: about two CTAs per SM over all (sequence, head) pairs, at
 // most one 64-row chunk per split when the context is short.
 fm_status attn_mma(fm_ctx* c, int n_noise, fm::AttnMmaArgs am, const bf16* qkv, const bf16* Kc,
                    const bf16* Vc, bf16* o, int n_seqs, int max_len, cudaStream_t st) {
+  // Few sequences with several noise drafts: one CTA per (draft, head,
+  // split) instead of one per (sequence, head, split).  The drafts' rows are
+  // consecutive [sequence][draft][K], so draft j of sequence b is "sequence"
+  // b n_noise + j of one draft with b's context; the CTAs of a context slice
+  // run together and share its reads in L2, and each head's merge covers
+  // 16 query rows instead of n_noise * 16.
+  const bool tiled = n_noise == 1 || n_noise == 2 || n_noise == 4;
+  if (n_noise > 1 && attn_split_drafts_ok(c, n_seqs, n_noise) &&
+      (!tiled || n_seqs * am.n_heads < c->sms)) {
+    for (int q = n_seqs - 1; q >= 0; --q)
+      for (int j = n_noise - 1; j >= 0; --j) {
+        am.slot[q * n_noise + j] = am.slot[q];
+        am.len[q * n_noise + j] = am.len[q];
+      }
+    n_seqs *= n_noise;
+    n_noise = 1;
+    am.n_seqs = n_seqs;
+    am.n_noise = 1;
+  }
   const int pairs = n_seqs * am.n_heads;
   // at most about two CTAs per SM, and at least four 64-row chunks per split:
   // every extra split adds a partial to the final merge
@@ -695,6 +723,10 @@ fm_status dit_persistent(fm_ctx* c, const float* mods, int slot, int ctx_len, bo
   if ((size_t)(s_ctx + 1) * 16 * fm::AM_PSTRIDE * 4 > (size_t)fm::DIT_UNION) return FM_ERR_UNSUPPORTED;
   am.n_ctx_splits = s_ctx;
   P.splits[fm::DIT_ATTN] = s_ctx;
+  // Measured: a programmatic launch (the pass's weight stream starting
+  // under x.E's tail, the LM head's under the pass's) with the flags cleared
+  // by the pass's last CTA instead of this memset made the pass 3.6 us
+  // slower and the end-to-end round 20-35 us slower
   FM_CUDA(cudaMemsetAsync(c->dit_flags, 0, c->dit_flags_n * sizeof(unsigned), st));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(G);
@@ -743,7 +775,8 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
   }
   // tensor-core (mma.sync) split-KV attention for bf16, head width 128
   const bool use_mma_attn = sizeof(T) == 2 && d / g.n_heads == fm::AM_DH && K == 16 &&
-                            (n_noise == 1 || n_noise == 2 || n_noise == 4);
+                            (n_noise == 1 || n_noise == 2 || n_noise == 4 ||
+                             attn_split_drafts_ok(c, n_seqs, n_noise));
   fm::AttnMmaArgs am;
   int max_len = 0;
   if (use_mma_attn) {

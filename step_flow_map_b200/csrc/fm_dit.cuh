@@ -842,8 +842,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_dit_persistent(const __grid_c
 
   // ---------------- teardown
   tc_fence_before();
-  __syncthreads();
-  if (*abort || *(volatile int*)P.abort_g) {
+  // one barrier that also ORs every thread's view of the abort words, so
+  // every thread takes the same branch
+  if (__syncthreads_or((*abort || *(volatile int*)P.abort_g) ? 1 : 0)) {
     if (threadIdx.x == 0) atomicExch(P.err, TC_ERR_TIMEOUT);
     const unsigned long long t0 = gtimer();
     while (gtimer() - t0 < 50000ull) {

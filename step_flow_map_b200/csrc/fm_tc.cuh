@@ -220,6 +220,10 @@ struct TcArgs {
   int M_ln;             // rows [0, M_ln) come from x; rows [M_ln, M) are copied from ln_extra
   const bf16* ln_extra; // [M - M_ln][Kd] bf16, already normalised
   int b_kb;             // k-blocks of the shared-memory-resident B operand
+  // > 1: the grid runs in clusters of this many CTAs, one unit each, that
+  // are the K splits of one output tile (one activation tile); their partial
+  // tiles are summed through distributed shared memory, not global memory
+  int cluster = 0;
 };
 
 // Ring depth: "deep" (about 200 KB, one CTA per SM) for long weight streams
@@ -234,6 +238,13 @@ __host__ __device__ constexpr int tc_stages(bool deep) {
               : (100 * 1024) / (TC_BM * TC_BK * 2 + BN * TC_BK * 2);
 }
 
+// barriers and flags of a GEMM CTA (after the operand tiles)
+constexpr int TC_BAR_BYTES = 256;
+
+// Whether split-K GEMMs of one activation tile may run as clusters that
+// reduce in distributed shared memory (diagnostic switch, set by the host).
+inline bool tc_cluster_ok = true;
+
 template <int BN, int STAGES_>
 struct TcCfg {
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;  // 16 KB
@@ -241,7 +252,7 @@ struct TcCfg {
   static constexpr int STAGE = A_BYTES + B_BYTES;
   static constexpr int STAGES = STAGES_;
   static constexpr int TMEM_COLS = (2 * BN) < 32 ? 32 : 2 * BN;
-  static constexpr int SMEM = STAGES * STAGE + 1024 /*align*/ + 256 /*barriers*/ + 8 * BN * 4;
+  static constexpr int SMEM = STAGES * STAGE + 1024 /*align*/ + TC_BAR_BYTES + 8 * BN * 4;
 };
 
 template <int BN, class Epi>
@@ -275,6 +286,140 @@ __device__ __forceinline__ void tc_finish_chunk(const Epi& epi, const TcArgs& a,
       if (m < a.M) epi(m, n, v[j]);
     }
   }
+}
+
+// ---- thread-block clusters: distributed shared memory and cluster-scope
+// barrier arrivals (rank = this CTA's index within its cluster)
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// All threads of every CTA of the cluster (kernel start only: nothing can
+// give up before it, so every thread reaches it).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
+                   "memory");
+}
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t dsmem_addr(uint32_t local, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(local), "r"(rank));
+  return a;
+}
+__device__ __forceinline__ float dsmem_ld(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+// One arrival, with release at cluster scope, on the barrier at `local` in
+// CTA `rank`.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t local, uint32_t rank) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+                   dsmem_addr(local, rank))
+               : "memory");
+}
+// Bounded wait, with acquire at cluster scope, for the phase of parity 0.
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, unsigned long long limit_ns) {
+  const unsigned long long t0 = gtimer();
+  for (;;) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(0u), "r"(20000u)
+        : "memory");
+    if (ok) return true;
+    if (gtimer() - t0 > limit_ns) return false;
+  }
+}
+
+// Rows m .. m + count - 1 (count <= 16) of feature n0 + r through the
+// epilogue (not the argmax epilogue).
+template <class Epi>
+__device__ __forceinline__ void tc_finish_rows(const Epi& epi, const TcArgs& a, int n0, int r, int m,
+                                               int count, const float* v) {
+  const int n = n0 + r;
+  if (n >= a.N) return;
+  if constexpr (has_chunk16<Epi>::value) {
+    epi.chunk16(m, n, v, count);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j < count) epi(m + j, n, v[j]);
+  }
+}
+
+// Split-K reduction of one output tile inside its cluster (a.cluster CTAs,
+// CTA z of the cluster holds K split z).  Every CTA stores its partial tile
+// [BN][128] fp32 in its own shared memory `sP`, arrives on every CTA's
+// `crdy`, waits for its own, then sums rows [z M / S, (z + 1) M / S) over
+// the cluster's tiles in split order (as the global-memory reduction does)
+// and finishes them; last, it arrives on every CTA's `cfree` and waits for
+// its own, so no CTA leaves while another may still read its tile.  A CTA
+// whose accumulator never arrived (`have` false) still makes every arrival,
+// so the others' waits end; it returns false and writes nothing.
+template <int BN, class Epi>
+__device__ __forceinline__ bool tc_cluster_finish(const Epi& epi, const TcArgs& a, int n0, int r,
+                                                  int et, uint32_t taddr, bool have, float* sP,
+                                                  uint64_t* crdy, uint64_t* cfree,
+                                                  volatile int* s_flag) {
+  const uint32_t S = (uint32_t)a.cluster, z = cluster_rank();
+  float v[16];
+  if (have) {
+    tc_fence_after();
+    for (int j0 = 0; j0 < BN; j0 += 16) {
+      tmem_ld16(taddr + j0, v);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) sP[(j0 + j) * TC_BM + r] = v[j];
+    }
+    tc_fence_before();
+  }
+  named_sync(1, 128);   // every thread's stores before the releasing arrivals
+  if (et == 0) {
+    for (uint32_t p = 0; p < S; ++p) mbar_arrive_cluster(smem_u32(crdy), p);
+    *s_flag = mbar_wait_cluster(smem_u32(crdy), TC_TIMEOUT_NS) ? 1 : 0;
+  }
+  named_sync(1, 128);
+  const bool ok = have && *s_flag != 0;
+  if (ok) {
+    (void)mbar_wait_cluster(smem_u32(crdy), TC_TIMEOUT_NS);   // complete: acquire for this thread
+    const int lo = (int)(z * (uint32_t)a.M / S), hi = (int)((z + 1) * (uint32_t)a.M / S);
+    const uint32_t mine = smem_u32(sP) + (uint32_t)r * 4u;
+    for (int m = lo; m < hi; m += 16) {
+      const int count = hi - m < 16 ? hi - m : 16;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = 0.f;
+      for (uint32_t p0 = 0; p0 < S; p0 += 4) {
+        // four splits' loads in flight; sums stay in split order
+        float t[4][16];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t pa = dsmem_addr(mine, p0 + u < S ? p0 + u : 0);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            t[u][j] = (p0 + u < S && j < count) ? dsmem_ld(pa + (uint32_t)((m + j) * TC_BM * 4)) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (p0 + u < S)
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] += t[u][j];
+      }
+      tc_finish_rows(epi, a, n0, r, m, count, v);
+    }
+  }
+  named_sync(1, 128);   // this CTA's reads of the other tiles are done
+  if (et == 0) {
+    for (uint32_t p = 0; p < S; ++p) mbar_arrive_cluster(smem_u32(cfree), p);
+    // longer than any wait before it, so a CTA that gave up late still
+    // finds the others resident when it arrives
+    if (!mbar_wait_cluster(smem_u32(cfree), 4ull * TC_TIMEOUT_NS)) *s_flag = 0;
+  }
+  named_sync(1, 128);
+  return ok && *s_flag != 0;
 }
 
 // Modulated LayerNorm of the activation rows, written straight into the
@@ -343,10 +488,14 @@ __device__ __forceinline__ void tc_ln_fill(uint8_t* sB, const TcArgs& a, int kb0
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-template <int BN, int STAGES, bool LNB, class Epi>
+// CL: launched in clusters of a.cluster CTAs that reduce their split-K
+// partials in distributed shared memory (a separate instantiation, so the
+// other launches carry none of its code)
+template <int BN, int STAGES, bool LNB, class Epi, bool CL = false>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 k_tc_gemm(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUtensorMap mapA,
           TcArgs a, Epi epi) {
+  static_assert(!CL || (!LNB && !is_argmax<Epi>::value), "cluster reduction: plain epilogues only");
   using C = TcCfg<BN, STAGES>;
   pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
@@ -366,7 +515,11 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUte
   volatile int* abort = (volatile int*)(tmem_slot + 1);
   int* s_last = (int*)(tmem_slot + 2);
   volatile int* s_ok = (volatile int*)(tmem_slot + 3);  // two slots
-  float* red_v = (float*)(base + data_bytes + 256);
+  float* red_v = (float*)(base + data_bytes + TC_BAR_BYTES);
+  // cluster reduction barriers: in the argmax scratch, which CL kernels
+  // never use (8-byte aligned)
+  uint64_t* crdy = (uint64_t*)red_v;
+  uint64_t* cfree = crdy + 1;
   int* red_i = (int*)(red_v + 4 * BN);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -380,6 +533,10 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUte
       mbar_init(smem_u32(&tempty[i]), 128);
     }
     mbar_init(smem_u32(bready), 128);
+    if constexpr (CL) {
+      mbar_init(smem_u32(crdy), (uint32_t)a.cluster);
+      mbar_init(smem_u32(cfree), (uint32_t)a.cluster);
+    }
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -390,6 +547,8 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUte
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // every CTA's barriers are initialised before another CTA can arrive on them
+  if constexpr (CL) cluster_sync_all();
   const uint32_t tmem = *tmem_slot;
   const int tiles = a.n_tiles * a.m_tiles;
 
@@ -503,9 +662,17 @@ k_tc_gemm(const __grid_constant__ CUtensorMap mapW, const __grid_constant__ CUte
       // next unit's value
       if (et == 0) s_ok[it & 1] = mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort) ? 1 : 0;
       named_sync(1, 128);
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + acc * BN;
+      if constexpr (CL) {
+        // this CTA's only unit: the ring is idle (every MMA has completed)
+        // and holds the partial tile the cluster reduces
+        if (!tc_cluster_finish<BN>(epi, a, n0, r, et, taddr, s_ok[it & 1] != 0, (float*)sA, crdy,
+                                   cfree, (volatile int*)s_last))
+          *abort = 1;
+        break;
+      }
       if (!s_ok[it & 1]) break;
       tc_fence_after();
-      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + acc * BN;
       float v[16];
       if (a.splits == 1) {
         for (int j0 = 0; j0 < BN; j0 += 16) {
@@ -702,12 +869,47 @@ template <int BN, int STAGES, class Epi, bool LNB = false>
 fm_status tc_launch_cfg(const TcMap& wm, const CUtensorMap& mapA, const TcArgs& a, int grid, Epi epi,
                         cudaStream_t st, char* err, size_t errlen, int* n_launch) {
   using C = TcCfg<BN, STAGES>;
-  const int smem = LNB ? C::STAGES * C::A_BYTES + a.b_kb * C::B_BYTES + 1024 + 256 + 8 * BN * 4
+  const int smem = LNB ? C::STAGES * C::A_BYTES + a.b_kb * C::B_BYTES + 1024 + TC_BAR_BYTES + 8 * BN * 4
                        : C::SMEM;
-  cudaError_t e = set_smem_once(k_tc_gemm<BN, STAGES, LNB, Epi>, LNB ? 227 * 1024 : C::SMEM);
-  if (e == cudaSuccess)
-    e = launch_pdl(k_tc_gemm<BN, STAGES, LNB, Epi>, dim3(grid), dim3(TC_THREADS), smem, st, wm.map,
-                   mapA, a, epi);
+  cudaError_t e = cudaSuccess;
+  bool launched = false;
+  if constexpr (!LNB && !is_argmax<Epi>::value && BN <= 128) {
+    if (a.cluster > 1) {
+      if (BN * TC_BM * 4 > C::STAGES * C::A_BYTES || 8 * BN * 4 < 16) {
+        snprintf(err, errlen, "tensor-core GEMM: no room for a cluster's partial tile");
+        return FM_ERR_UNSUPPORTED;
+      }
+      e = set_smem_once(k_tc_gemm<BN, STAGES, LNB, Epi, true>, C::SMEM);
+      // programmatic launch in clusters of a.cluster CTAs (the K splits of a tile)
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(grid);
+      cfg.blockDim = dim3(TC_THREADS);
+      cfg.dynamicSmemBytes = smem;
+      cfg.stream = st;
+      cudaLaunchAttribute attr[2];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      attr[1].id = cudaLaunchAttributeClusterDimension;
+      attr[1].val.clusterDim.x = (unsigned)a.cluster;
+      attr[1].val.clusterDim.y = 1;
+      attr[1].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 2;
+      if (e == cudaSuccess)
+        e = cudaLaunchKernelEx(&cfg, k_tc_gemm<BN, STAGES, LNB, Epi, true>, wm.map, mapA, a, epi);
+      launched = true;
+    }
+  }
+  if (!launched) {
+    if (a.cluster > 1) {
+      snprintf(err, errlen, "tensor-core GEMM: this epilogue has no cluster reduction");
+      return FM_ERR_UNSUPPORTED;
+    }
+    e = set_smem_once(k_tc_gemm<BN, STAGES, LNB, Epi>, LNB ? 227 * 1024 : C::SMEM);
+    if (e == cudaSuccess)
+      e = launch_pdl(k_tc_gemm<BN, STAGES, LNB, Epi>, dim3(grid), dim3(TC_THREADS), smem, st,
+                     wm.map, mapA, a, epi);
+  }
   if (e != cudaSuccess) {
     snprintf(err, errlen, "tensor-core GEMM launch: %s", cudaGetErrorString(e));
     return FM_ERR_CUDA;
@@ -734,18 +936,33 @@ fm_status tc_launch(const TcMap& wm, const bf16* A, int lda, int M, Epi epi, flo
   // all partial tiles: with per-split weight bytes W/S and S partial tiles of
   // P bytes, S ~ sqrt(W/P) (the O projection at 64 rows: 4 splits of its
   // 512 KB weight tile instead of 9, each partial 32 KB)
-  int splits = 1;
+  int splits = 1, cluster = 0;
   if (tiles < sms) {
     splits = sms / tiles;
     splits = splits > a.k_blocks ? a.k_blocks : splits;
     const double w_tile = (double)a.k_blocks * TC_BK * TC_BM * 2.0;
     const double p_tile = (double)TC_BM * BN * 4.0;
     const int s_bal = (int)ceil(sqrt(w_tile / p_tile));
-    if (splits > s_bal) splits = s_bal;
-    while (splits > 1 && (size_t)splits * tiles * TC_BM * BN > partial_elems) --splits;
+    // one activation tile: the K splits of a tile can form a cluster (at
+    // most 8 CTAs) and sum their partials in distributed shared memory, in
+    // parallel over the rows and with no global-memory round trip, so the
+    // balance cap does not apply; taken when it keeps at least as many
+    // splits as the global-memory reduction would (measured: the context fc
+    // at 17 rows in 8 clustered splits instead of 9 was no faster)
+    const int s_cl = splits < 8 ? splits : 8;
+    const int s_gm = splits > s_bal ? s_bal : splits;
+    if (tc_cluster_ok && !is_argmax<Epi>::value && a.m_tiles == 1 && BN <= 128 && s_cl >= 2 &&
+        s_cl >= s_gm) {
+      splits = s_cl;
+      cluster = s_cl;
+    } else {
+      splits = s_gm;
+      while (splits > 1 && (size_t)splits * tiles * TC_BM * BN > partial_elems) --splits;
+    }
   }
-  if (splits > 1 && tiles > tile_cnt_n) splits = 1;
+  if (!cluster && splits > 1 && tiles > tile_cnt_n) splits = 1;
   a.splits = splits < 1 ? 1 : splits;
+  a.cluster = cluster;
   a.units = tiles * a.splits;
   a.partial = partial;
   a.tile_cnt = tile_cnt;
@@ -825,7 +1042,7 @@ fm_status tc_launch_ln(const TcMap& wm, const float* x, const float* shift, cons
   const bool deep = per_cta >= 24;
   using CS = TcCfg<BN, 5>;
   using CD = TcCfg<BN, 8>;
-  if ((deep ? 8 * CD::A_BYTES : 5 * CS::A_BYTES) + a.b_kb * CS::B_BYTES + 1280 + 8 * BN * 4 >
+  if ((deep ? 8 * CD::A_BYTES : 5 * CS::A_BYTES) + a.b_kb * CS::B_BYTES + 1024 + TC_BAR_BYTES + 8 * BN * 4 >
       227 * 1024)
     return FM_ERR_UNSUPPORTED;
   if (deep)

@@ -30,16 +30,19 @@ def _workload(B, N, t_grid=(0.0, 1.0), temps=None, ctx=40):
                                temps=temps or tuple([0.0] * B))
 
 
-def _run(w, env_off=False, logits=True, no_persistent=False):
+def _run(w, env_off=False, logits=True, no_persistent=False, no_cluster=False):
     if env_off:
         os.environ["FM_DISABLE_TC"] = "1"
     if no_persistent:
         os.environ["FM_DISABLE_PERSISTENT"] = "1"
+    if no_cluster:
+        os.environ["FM_DISABLE_TC_CLUSTER"] = "1"
     try:
         ctx = gu.make_ctx(w, max_new=64)
     finally:
         os.environ.pop("FM_DISABLE_TC", None)
         os.environ.pop("FM_DISABLE_PERSISTENT", None)
+        os.environ.pop("FM_DISABLE_TC_CLUSTER", None)
     seqs = list(range(w.B))
     gu.gpu_prefill(ctx, w, seqs, max_new=64)
     gu.gpu_new_rows(ctx, w, 0, seqs)
@@ -99,6 +102,22 @@ def test_persistent_pass_context_rows_reach_the_cache():
         ref = om.draft(W, w.shape, kv, ri.noise[0], w.t_grid)
         gu.assert_logits_close(gu.to_np(lg)[0], ref["logits"], "bf16", f"round {r}")
     ctx.close()
+
+
+def test_cluster_splitk_matches_global_reduction():
+    # four noise drafts of one sequence: 64 activation rows, one activation
+    # tile, so the split-K GEMMs of the draft (x.E in 8 splits, QKV, O and
+    # the MLP) sum their partial tiles inside a thread-block cluster through
+    # distributed shared memory; the same draft with the partials reduced
+    # through global memory (other split counts) agrees to rounding, and
+    # both match the oracle
+    w = _workload(1, 4)
+    (tok_c, lg_c), _ = _run(w)
+    (tok_g, lg_g), _ = _run(w, no_cluster=True)
+    np.testing.assert_allclose(lg_c, lg_g, atol=2e-2, rtol=1e-2)
+    ref = gu.oracle_draft(w, 0, 0)
+    gu.assert_logits_close(lg_c[0], ref["logits"], "bf16", "cluster")
+    gu.assert_logits_close(lg_g[0], ref["logits"], "bf16", "global")
 
 
 def test_tc_matches_cuda_core_path():
