@@ -959,8 +959,14 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
     }
     Prof prof(c, FM_PROF_NORM, st);
     if (!last) {
-      FM_LAUNCH(c, FM_PROF_NORM, (fm::k_softmax_rows<T>), M, 1024, 0, st,
-              logits, V, (T*)c->D);
+      // a cluster of CTAs per row, up to four, about two CTAs per SM
+      const int C = std::max(1, std::min(4, 2 * c->sms / std::max(1, M)));
+      const cudaError_t e_ = fm::launch_pdl_cluster(fm::k_softmax_rows<T>, dim3(M * C), dim3(1024),
+                                                    0, st, (unsigned)C, (const float*)logits, V,
+                                                    (T*)c->D);
+      c->launches[FM_PROF_NORM]++;
+      if (e_ != cudaSuccess)
+        return set_err(FM_ERR_CUDA, "launch of k_softmax_rows failed: %s", cudaGetErrorString(e_));
     } else {
       // greedy rows (and, with few sampled rows, the sampled ones) one CTA
       // per row; many sampled rows through the chunked sampler

@@ -63,14 +63,17 @@ k_adaln(const TI* __restrict__ x, int d, const float* __restrict__ shift,
   const int T = blockDim.x;
   // rows up to 16 T wide stay in registers: one read, all loads in flight
   constexpr int CACHE = 16;
-  float xv[CACHE];
+  float xv[CACHE], cv[CACHE], hv[CACHE];
   const bool cached = d <= CACHE * T;
   float s = 0.f;
   if (cached) {
+    // the row, and the modulation of this thread's columns, in one round trip
 #pragma unroll
     for (int i = 0; i < CACHE; ++i) {
       const int c = threadIdx.x + i * T;
       xv[i] = c < d ? to_f(row[c]) : 0.f;
+      cv[i] = (scale && c < d) ? scale[c] : 0.f;
+      hv[i] = (scale && c < d) ? shift[c] : 0.f;
     }
 #pragma unroll
     for (int i = 0; i < CACHE; ++i) s += xv[i];
@@ -101,7 +104,7 @@ k_adaln(const TI* __restrict__ x, int d, const float* __restrict__ shift,
       const int c = threadIdx.x + i * T;
       if (c < d) {
         float y = (xv[i] - mean) * rstd;
-        if (scale) y = y * (1.f + scale[c]) + shift[c];
+        if (scale) y = y * (1.f + cv[i]) + hv[i];
         out[(size_t)m * d + c] = from_f<TO>(y);
       }
     }
@@ -149,23 +152,51 @@ __device__ __forceinline__ void for_row_range(const float* __restrict__ row, int
 
 // ------------------------------------------------------------------ softmax rows
 // D[m] = softmax(logits[m]) at temperature 1, stored as dtype (the flow-map
-// denoiser output used by the next step's embedding).
+// denoiser output used by the next step's embedding).  Launched in clusters
+// of C CTAs per row (C = 1 without a cluster; grid = rows x C): CTA z of a
+// row takes the vocabulary slice [z V / C, (z + 1) V / C).  One pass keeps a
+// running (max, sum of exp(x - max)) per thread; the CTA combines its
+// threads' pairs, the cluster its CTAs' pairs through distributed shared
+// memory, and a second pass writes exp(x - max) / sum.
 template <typename TO>
 __global__ void __launch_bounds__(1024)
 k_softmax_rows(const float* __restrict__ logits, int V, TO* __restrict__ D) {
   pdl_wait();
   pdl_trigger();
   __shared__ float sh[32];
-  const float* row = logits + (size_t)blockIdx.x * V;
+  __shared__ float s_ms[2];               // this CTA's (max, sum), read by the cluster
+  const uint32_t C = cluster_size(), z = cluster_rank();
+  const int r = blockIdx.x / (int)C;
+  const int v0 = (int)((long)z * V / C), v1 = (int)((long)(z + 1) * V / C);
+  const float* row = logits + (size_t)r * V;
+  float m = -INFINITY, s = 0.f;
+  for_row_range(row, v0, v1, [&](int, float x) {
+    if (x > m) {
+      s = s * __expf(m - x) + 1.f;
+      m = x;
+    } else if (x != -INFINITY) {
+      s += __expf(x - m);
+    }
+  });
+  const float mb = block_max(m, sh);
+  float sb = block_sum(m == -INFINITY ? 0.f : s * __expf(m - mb), sh);
+  if (threadIdx.x == 0) {
+    s_ms[0] = mb;
+    s_ms[1] = sb;
+  }
+  cluster_sync_all();                     // every CTA's pair is written
   float mx = -INFINITY;
-  for_row_range(row, 0, V, [&](int, float x) { mx = fmaxf(mx, x); });
-  mx = block_max(mx, sh);
-  float s = 0.f;
-  for_row_range(row, 0, V, [&](int, float x) { s += __expf(x - mx); });
-  s = block_sum(s, sh);
-  const float inv = 1.f / s;
-  TO* out = D + (size_t)blockIdx.x * V;
-  for_row_range(row, 0, V, [&](int v, float x) { out[v] = from_f<TO>(__expf(x - mx) * inv); });
+  for (uint32_t p = 0; p < C; ++p) mx = fmaxf(mx, dsmem_ld(dsmem_addr((uint32_t)__cvta_generic_to_shared(&s_ms[0]), p)));
+  float tot = 0.f;
+  for (uint32_t p = 0; p < C; ++p) {
+    const float mp = dsmem_ld(dsmem_addr((uint32_t)__cvta_generic_to_shared(&s_ms[0]), p));
+    const float sp = dsmem_ld(dsmem_addr((uint32_t)__cvta_generic_to_shared(&s_ms[1]), p));
+    if (mp != -INFINITY) tot += sp * __expf(mp - mx);
+  }
+  cluster_sync_all();                     // no CTA leaves while another reads its pair
+  const float inv = 1.f / tot;
+  TO* out = D + (size_t)r * V;
+  for_row_range(row, v0, v1, [&](int v, float x) { out[v] = from_f<TO>(__expf(x - mx) * inv); });
 }
 
 // ------------------------------------------------------------------ inverse CDF

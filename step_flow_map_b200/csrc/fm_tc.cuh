@@ -288,30 +288,7 @@ __device__ __forceinline__ void tc_finish_chunk(const Epi& epi, const TcArgs& a,
   }
 }
 
-// ---- thread-block clusters: distributed shared memory and cluster-scope
-// barrier arrivals (rank = this CTA's index within its cluster)
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// All threads of every CTA of the cluster (kernel start only: nothing can
-// give up before it, so every thread reaches it).
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
-                   "memory");
-}
-// Address of the same shared-memory location in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t dsmem_addr(uint32_t local, uint32_t rank) {
-  uint32_t a;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(local), "r"(rank));
-  return a;
-}
-__device__ __forceinline__ float dsmem_ld(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
-}
+// ---- cluster-scope barrier arrivals (the cluster helpers are in fm_common.cuh)
 // One arrival, with release at cluster scope, on the barrier at `local` in
 // CTA `rank`.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t local, uint32_t rank) {
