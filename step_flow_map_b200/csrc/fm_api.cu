@@ -959,10 +959,12 @@ fm_status draft_impl(fm_ctx* c, const int32_t* seq_ids, int n_seqs, const void* 
     }
     Prof prof(c, FM_PROF_NORM, st);
     if (!last) {
-      // a cluster of CTAs per row, up to four, about two CTAs per SM
+      // a cluster of CTAs per row, up to four, about two CTAs per SM; 512
+      // threads, so registers admit two CTAs per SM (measured: 1,024 threads
+      // of 44 registers fit one per SM and ran in two waves, 44 us)
       const int C = std::max(1, std::min(4, 2 * c->sms / std::max(1, M)));
-      const cudaError_t e_ = fm::launch_pdl_cluster(fm::k_softmax_rows<T>, dim3(M * C), dim3(1024),
-                                                    0, st, (unsigned)C, (const float*)logits, V,
+      const cudaError_t e_ = fm::launch_pdl_cluster(fm::k_softmax_rows<T>, dim3(M * C), dim3(512),
+                                                    0, st, (unsigned)C, (const float*)logits, V, M,
                                                     (T*)c->D);
       c->launches[FM_PROF_NORM]++;
       if (e_ != cudaSuccess)

@@ -160,13 +160,14 @@ __device__ __forceinline__ void for_row_range(const float* __restrict__ row, int
 // memory, and a second pass writes exp(x - max) / sum.
 template <typename TO>
 __global__ void __launch_bounds__(1024)
-k_softmax_rows(const float* __restrict__ logits, int V, TO* __restrict__ D) {
+k_softmax_rows(const float* __restrict__ logits, int V, int rows, TO* __restrict__ D) {
   pdl_wait();
   pdl_trigger();
   __shared__ float sh[32];
   __shared__ float s_ms[2];               // this CTA's (max, sum), read by the cluster
   const uint32_t C = cluster_size(), z = cluster_rank();
   const int r = blockIdx.x / (int)C;
+  if (r >= rows) return;                  // every CTA of the cluster: the same row
   const int v0 = (int)((long)z * V / C), v1 = (int)((long)(z + 1) * V / C);
   const float* row = logits + (size_t)r * V;
   float m = -INFINITY, s = 0.f;
