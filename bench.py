@@ -93,9 +93,25 @@ def _clock_child(bus: str, conn, stop) -> None:
     conn.send(out)
 
 
+def window_samples(raw, t0: float, t1: float, reasons: dict):
+    """SM clocks and throttle-reason names of the NVML samples taken in the
+    timed region [t0, t1].  A sample is the interval [before, after] of its
+    two NVML calls; one that overlaps the region counts (an NVML call can
+    take longer than a short timed region, which then holds no sample that
+    started and ended inside it)."""
+    mhz_in, names = [], set()
+    for tb, ta, mhz, r in raw:
+        if ta >= t0 and tb <= t1:
+            mhz_in.append(mhz)
+            for bit, name in reasons.items():
+                if r & bit:
+                    names.add(name)
+    return mhz_in, names
+
+
 class ClockSampler:
     """SM clock and throttle reasons sampled during the timed region by a
-    separate NVML process; only samples taken inside [enter, exit] count."""
+    separate NVML process; the samples overlapping [enter, exit] count."""
 
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
@@ -136,12 +152,8 @@ class ClockSampler:
         raw = self.conn.recv() if self.conn.poll(30) else []
         self.proc.join(10)
         self.window = self.t1 - self.t0
-        for tb, ta, mhz, r in raw:
-            if tb >= self.t0 and ta <= self.t1:
-                self.samples.append(mhz)
-                for bit, name in self.REASONS.items():
-                    if r & bit:
-                        self.reasons.add(name)
+        self.samples, self.reasons = window_samples(raw, self.t0, self.t1, self.REASONS)
+
 
     def summary(self):
         if not self.ok:

@@ -155,3 +155,33 @@ def test_8b_bs1_step_bytes_match_the_survey_count():
     assert not bench.persistent_pass(w5)
     d = w5.shape.d
     assert bench.algorithmic_bytes(w5)["context"] > 6 * 2 * d * d * 2   # separate K/V projection
+
+
+def test_clock_samples_of_the_timed_region():
+    # samples are (before, after, MHz, reason bits); those overlapping the
+    # region [10, 11] count, including one NVML call that spans all of it
+    R = bench.ClockSampler.REASONS
+    raw = [(9.0, 9.5, 1000, 0x0),        # before the region
+           (9.9, 10.1, 1965, 0x4),       # overlaps its start: sw_power_cap
+           (10.4, 10.5, 1965, 0x0),      # inside
+           (10.9, 11.2, 1900, 0x8),      # overlaps its end: hw_slowdown
+           (11.5, 11.6, 500, 0x20)]      # after
+    mhz, names = bench.window_samples(raw, 10.0, 11.0, R)
+    assert mhz == [1965, 1965, 1900]
+    assert names == {"sw_power_cap", "hw_slowdown"}
+    mhz, names = bench.window_samples([(9.0, 12.0, 1965, 0x0)], 10.0, 11.0, R)
+    assert mhz == [1965] and names == set()
+    assert bench.window_samples([], 10.0, 11.0, R) == ([], set())
+
+
+def test_clock_summary_of_a_sampler():
+    # the summary the bench line carries, without NVML: a sampler that
+    # could not start reports why; one with samples reports their median
+    c = bench.ClockSampler.__new__(bench.ClockSampler)
+    c.ok, c.err = False, "no NVML"
+    assert c.summary()["reasons"] == ["nvml unavailable: no NVML"]
+    c.ok, c.max_mhz, c.window = True, 1965, 0.05
+    c.samples, c.reasons = [1965, 1900, 1965], {"sw_power_cap"}
+    s = c.summary()
+    assert s["sm_mhz"] == 1965 and s["samples"] == 3 and s["reasons"] == ["sw_power_cap"]
+    assert s["window_ms"] == 50.0 and s["sm_max_mhz"] == 1965
